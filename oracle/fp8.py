@@ -1,0 +1,118 @@
+"""FP8-E4M3 codec and fine-grained block quantisation (test infrastructure).
+
+E4M3 follows the OCP 8-bit floating point format definition (OFP8, "E4M3"):
+1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+encodes subnormals (m/8 * 2^-6); there are no infinities and S.1111.111 is
+NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.  Encoding here is
+round-to-nearest-even with saturation to +-448 ("satfinite").
+
+Quantisation follows [P1] §4.1 (精细量化策略, 在线量化): activations are
+scaled per 1x128 tile and weights per 128x128 block, each scale computed
+online from the tile's current max-abs.  Reading taken: scale = amax/448 and
+its inverse 448/amax, both float32 (IEEE division); code =
+E4M3(float32(v * inverse)); dequantised value = code * scale; a tile whose
+amax is 0 gets scale 1 and all-zero codes.  The block-scaled GEMM keeps one
+float64 partial sum per 128-wide K slice and applies both scales to it, which
+is the exact value of sum_k (qa*sa)(qb*sb).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 bit patterns (uint8) -> float64 values (NaN for S.1111.111)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    E = (c >> 3) & 0xF
+    M = c & 0x7
+    mag = np.where(E == 0, (M / 8.0) * 2.0 ** -6, (1.0 + M / 8.0) * np.exp2(E - 7.0))
+    mag = np.where((E == 15) & (M == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_all_values() -> np.ndarray:
+    """Values of all 256 codes, index = code."""
+    return e4m3_decode(np.arange(256, dtype=np.uint8))
+
+
+_POS_VALUES = e4m3_all_values()[:127]          # codes 0x00..0x7E: 0 .. 448, increasing
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """float -> E4M3 code, round to nearest (ties to even mantissa),
+    saturating finite overflow to +-448; NaN -> 0x7F."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, e = np.frexp(a)                         # a = m * 2**e, 0.5 <= m < 1
+    step_exp = np.maximum(e - 4, -9)           # 3 mantissa bits; subnormal step 2^-9
+    r = np.ldexp(np.rint(np.ldexp(a, -step_exp)), step_exp)
+    r = np.minimum(r, 448.0)
+    code = np.searchsorted(_POS_VALUES, np.nan_to_num(r, nan=0.0)).astype(np.uint8)
+    assert np.all(np.isnan(r) | (_POS_VALUES[np.minimum(code, 126)] == r))
+    code = np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+    return np.where(np.isnan(v), np.uint8(0x7F), code).astype(np.uint8)
+
+
+def _quant_tiles(tiles32: np.ndarray):
+    """Quantise tiles [..., n] (float32 values), each with its own online
+    scale from its max-abs.  Returns (codes [..., n], scales [...])."""
+    amax = np.max(np.abs(tiles32), axis=-1).astype(np.float32)
+    zero = amax == 0
+    safe = np.where(zero, np.float32(1.0), amax).astype(np.float32)
+    scale = np.where(zero, np.float32(1.0), safe / np.float32(448.0)).astype(np.float32)
+    inv = (np.float32(448.0) / safe).astype(np.float32)
+    prod = (tiles32 * inv[..., None]).astype(np.float32)
+    codes = np.where(zero[..., None], np.uint8(0), e4m3_encode(prod)).astype(np.uint8)
+    return codes, scale
+
+
+def quant_rows_1x128(a):
+    """Per-row, per-128-column quantisation of activations [M, K] (K % 128 == 0).
+    Returns (codes uint8 [M, K], scales float32 [M, K/128])."""
+    a32 = np.asarray(a, dtype=np.float32)
+    M, K = a32.shape
+    codes, scales = _quant_tiles(a32.reshape(M, K // 128, 128))
+    return codes.reshape(M, K), scales
+
+
+def quant_blocks_128(w):
+    """Per-128x128-block quantisation of a weight matrix [R, C] (both % 128 == 0).
+    Returns (codes uint8 [R, C], scales float32 [R/128, C/128])."""
+    w32 = np.asarray(w, dtype=np.float32)
+    R, C = w32.shape
+    blocks = w32.reshape(R // 128, 128, C // 128, 128).transpose(0, 2, 1, 3)
+    codes, scales = _quant_tiles(blocks.reshape(R // 128, C // 128, 128 * 128))
+    codes = codes.reshape(R // 128, C // 128, 128, 128).transpose(0, 2, 1, 3).reshape(R, C)
+    return codes, scales
+
+
+def fp8_gemm_ref(codes_a, sa, codes_b, sb) -> np.ndarray:
+    """out[m, n] = sum_k (qa[m,k] sa[m,k/128]) (qb[n,k] sb[n/128,k/128]) in
+    float64, for A [M, K] (1x128 scales) and B [Nn, K] (128x128 scales)."""
+    qa = e4m3_decode(codes_a)
+    qb = e4m3_decode(codes_b)
+    M, K = qa.shape
+    Nn = qb.shape[0]
+    out = np.zeros((M, Nn), dtype=np.float64)
+    sbx = np.repeat(np.asarray(sb, np.float64), 128, axis=0)[:Nn]      # [Nn, K/128]
+    for kb in range(K // 128):
+        part = qa[:, kb * 128:(kb + 1) * 128] @ qb[:, kb * 128:(kb + 1) * 128].T
+        out += part * np.asarray(sa, np.float64)[:, kb:kb + 1] * sbx[:, kb][None, :]
+    return out
+
+
+def fp8_swiglu_expert(a, w1, w3, w2) -> np.ndarray:
+    """One SwiGLU expert with all three GEMMs in block-scaled E4M3 ([P1] §4.1):
+    the rows ``a`` (bf16 values) are quantised per 1x128 tile along d, W1, W3
+    ([f, d]) and W2 ([d, f]) per 128x128 block; the hidden activation
+    h = silu(a W1^T) * (a W3^T) is held in float32 (the accumulation
+    precision the pages name) and quantised per 1x128 tile along f before W2."""
+    from .moe import silu
+    qa, sa = quant_rows_1x128(a)
+    q1, s1 = quant_blocks_128(w1)
+    q3, s3 = quant_blocks_128(w3)
+    q2, s2 = quant_blocks_128(w2)
+    h = silu(fp8_gemm_ref(qa, sa, q1, s1)) * fp8_gemm_ref(qa, sa, q3, s3)
+    qh, sh = quant_rows_1x128(h.astype(np.float32))
+    return fp8_gemm_ref(qh, sh, q2, s2)

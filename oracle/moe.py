@@ -1,0 +1,249 @@
+"""Float64 oracle of the DeepSeekMoE layer forward (test infrastructure only).
+
+Each function is the plain definition of one step, written for a reader to
+check against the pages by eye; see the package docstring for the [P*] page
+keys.  All arithmetic is float64 unless a step names another precision.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# rounding helpers (storage precision of operands the method stores)
+# ---------------------------------------------------------------------------
+
+def round_bf16(v) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits,
+    ties to even), returned as float64.  Written as an exact power-of-two
+    rescale plus numpy's half-to-even ``rint`` (finite, in-range inputs)."""
+    v = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(v)                      # v = m * 2**e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                 # bf16 subnormal spacing is 2**-133
+    step_exp = e - 8                        # 8 significant bits
+    return np.ldexp(np.rint(np.ldexp(v, -step_exp)), step_exp)
+
+
+def silu(u):
+    """SiLU(u) = u * sigmoid(u) = u / (1 + exp(-u))."""
+    u = np.asarray(u, dtype=np.float64)
+    return u / (1.0 + np.exp(-u))
+
+
+# ---------------------------------------------------------------------------
+# routing: affinity, bias, group limit, top-K, gates, counts
+# ---------------------------------------------------------------------------
+
+def affinity(x, router) -> np.ndarray:
+    """s[t, i] = sigmoid(x_t . e_i) in float64 from the stored operands.
+
+    [P4] DeepSeekMoE paragraph: V3 computes the token-to-expert affinity with
+    a sigmoid (not a softmax)."""
+    z = np.asarray(x, dtype=np.float64) @ np.asarray(router, dtype=np.float64).T
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def biased_scores(s, bias) -> np.ndarray:
+    """s'[t, i] = s[t, i] + b_i, the score used only to choose experts.
+
+    [P2] Q3 and [P1] §1.2: a per-expert bias is added to the affinity score
+    to steer routing; it never enters the gate value."""
+    return np.asarray(s, dtype=np.float64) + np.asarray(bias, dtype=np.float64)[None, :]
+
+
+def group_scores(sb, G: int) -> np.ndarray:
+    """Score of each of G contiguous expert groups (expert i in group
+    i // (N/G)): the sum of the two largest biased scores in the group (the
+    whole group when it holds one expert).
+
+    [P1] §3.1 limits each token to at most 4 nodes; with experts laid out
+    contiguously over nodes a group is a node.  The top-2-sum group score is
+    the reading this library takes (the pages give no formula)."""
+    T, N = sb.shape
+    gs = N // G
+    out = np.empty((T, G), dtype=np.float64)
+    for g in range(G):
+        block = np.sort(sb[:, g * gs:(g + 1) * gs], axis=1)    # ascending
+        out[:, g] = block[:, -min(2, gs):].sum(axis=1)
+    return out
+
+
+def kept_groups(gscore, topG: int) -> np.ndarray:
+    """Indices of the topG highest-scoring groups per token (lower index wins
+    an exact tie), [T, topG]."""
+    order = np.argsort(-gscore, axis=1, kind="stable")
+    return order[:, :topG]
+
+
+def route(x, router, bias, G: int, topG: int, K: int) -> dict:
+    """Group-limited top-K routing with the bias-for-selection-only rule.
+
+    Steps (per token):
+      1. s = sigmoid(x . e_i)                             [P4]
+      2. s' = s + b                                       [P2] Q3, [P1] §1.2
+      3. keep the topG groups by group score (top-2 sum)  [P1] §3.1
+      4. idx = the K largest s' among experts of kept groups ([P5] §二(一)4
+         top-K by affinity); reported in ascending expert id
+      5. gate_k = s[idx_k] / sum_j s[idx_j] with the *un-biased* s
+         ([P4]: normalise over the selected affinities; [P2] Q3: the bias
+         does not affect the gate)
+      6. counts_i = number of tokens that selected expert i
+    Returns dict(idx [T,K] int64, gate [T,K] f64, counts [N] int64, s, sb)."""
+    s = affinity(x, router)
+    sb = biased_scores(s, bias)
+    T, N = sb.shape
+    allowed = np.zeros((T, N), dtype=bool)
+    gs = N // G
+    for t, groups in enumerate(kept_groups(group_scores(sb, G), topG)):
+        for g in groups:
+            allowed[t, g * gs:(g + 1) * gs] = True
+    masked = np.where(allowed, sb, -np.inf)
+    top = np.argsort(-masked, axis=1, kind="stable")[:, :K]
+    idx = np.sort(top, axis=1)
+    sel = np.take_along_axis(s, idx, axis=1)
+    gate = sel / sel.sum(axis=1, keepdims=True)
+    counts = np.bincount(idx.ravel(), minlength=N).astype(np.int64)
+    return dict(idx=idx.astype(np.int64), gate=gate, counts=counts, s=s, sb=sb)
+
+
+def route_margins(x, router, bias, G: int, topG: int, K: int) -> np.ndarray:
+    """Per token, the smaller of two gaps that decide the discrete routing:
+    (K-th minus (K+1)-th biased score among experts of the kept groups) and
+    (topG-th minus (topG+1)-th group score).  +inf where a gap does not exist
+    (K = number of allowed experts, or topG = G)."""
+    s = affinity(x, router)
+    sb = biased_scores(s, bias)
+    T, N = sb.shape
+    gsc = group_scores(sb, G)
+    gsorted = -np.sort(-gsc, axis=1)
+    gmargin = (gsorted[:, topG - 1] - gsorted[:, topG]) if topG < G else np.full(T, np.inf)
+    gs = N // G
+    emargin = np.full(T, np.inf)
+    for t, groups in enumerate(kept_groups(gsc, topG)):
+        vals = np.sort(np.concatenate([sb[t, g * gs:(g + 1) * gs] for g in groups]))[::-1]
+        if K < vals.size:
+            emargin[t] = vals[K - 1] - vals[K]
+    return np.minimum(gmargin, emargin)
+
+
+# ---------------------------------------------------------------------------
+# dispatch, experts, combine
+# ---------------------------------------------------------------------------
+
+def dispatch(idx, N: int) -> dict:
+    """Group the (token, expert) pairs by expert for the expert GEMMs
+    ([P1] §2.2: DISPATCH precedes MLP).
+
+    Row order: experts ascending, and within one expert tokens ascending.
+    offsets[i] = first row of expert i (exclusive prefix sum of the counts),
+    perm_tok[r] = token of row r, slot[t, k] = row holding (t, idx[t, k])."""
+    idx = np.asarray(idx)
+    T, K = idx.shape
+    counts = np.bincount(idx.ravel(), minlength=N)
+    offsets = np.zeros(N + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    perm_tok = np.empty(T * K, dtype=np.int64)
+    slot = np.empty((T, K), dtype=np.int64)
+    fill = offsets[:-1].copy()
+    for t in range(T):                      # tokens in ascending order
+        for k in range(K):
+            e = idx[t, k]
+            perm_tok[fill[e]] = t
+            slot[t, k] = fill[e]
+            fill[e] += 1
+    return dict(offsets=offsets, perm_tok=perm_tok, slot=slot, counts=counts)
+
+
+def swiglu_expert(a, w1, w3, w2, h_round: str = "none") -> np.ndarray:
+    """One expert FFN on the rows ``a`` [M, d]:
+    y = (silu(a W1^T) * (a W3^T)) W2^T, with W1, W3 [f, d] and W2 [d, f].
+
+    The expert is an FFN ([P1] §1.1, [P5]); its SwiGLU form is this library's
+    reading.  ``h_round='bf16'`` rounds the hidden activation to bf16 before
+    the W2 contraction (it is stored as a bf16 GEMM operand)."""
+    a = np.asarray(a, dtype=np.float64)
+    h = silu(a @ np.asarray(w1, np.float64).T) * (a @ np.asarray(w3, np.float64).T)
+    if h_round == "bf16":
+        h = round_bf16(h)
+    return h @ np.asarray(w2, np.float64).T
+
+
+def expert_outputs(x, idx, get_weights, N: int, tokens=None, h_round: str = "none",
+                   expert_fn=None) -> dict:
+    """Per-expert outputs for the selected tokens.
+
+    Returns {'shared': y_sh [len(tokens), d], 'routed': {(t, e): y [d]}} where
+    y_sh = E_N(x_t) is the always-on shared expert ([P1] §1.1: the shared
+    expert processes every token) and routed entries are E_e(x_t) for each
+    selected expert e of each token t.  ``get_weights(e)`` -> (W1, W3, W2);
+    ``expert_fn(a, w1, w3, w2)`` overrides the expert math (FP8 emulation)."""
+    x = np.asarray(x, dtype=np.float64)
+    tokens = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens)
+    fn = expert_fn or (lambda a, w1, w3, w2: swiglu_expert(a, w1, w3, w2, h_round))
+    routed = {}
+    users = {}
+    for t in tokens:
+        for e in idx[t]:
+            users.setdefault(int(e), []).append(int(t))
+    for e in sorted(users):
+        w1, w3, w2 = get_weights(e)
+        ts = users[e]
+        y = fn(x[ts], w1, w3, w2)
+        for j, t in enumerate(ts):
+            routed[(t, e)] = y[j]
+    w1, w3, w2 = get_weights(N)
+    shared = fn(x[tokens], w1, w3, w2)
+    return dict(shared=shared, routed=routed, tokens=tokens)
+
+
+def combine(shared, routed, idx, gate, tokens) -> np.ndarray:
+    """y_t = y_shared_t + sum_k gate[t,k] * E_{idx[t,k]}(x_t), float64
+    ([P1] §2.2 COMBINE; [P4] gate-weighted sum of the routed outputs)."""
+    out = np.array(shared, dtype=np.float64, copy=True)
+    for j, t in enumerate(tokens):
+        for k in range(idx.shape[1]):
+            out[j] += gate[t, k] * routed[(int(t), int(idx[t, k]))]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# auxiliary-loss-free bias update
+# ---------------------------------------------------------------------------
+
+def bias_update(bias, counts, T: int, K: int, gamma: float) -> np.ndarray:
+    """b_i <- b_i - gamma if expert i is overloaded, b_i + gamma if it is
+    under-loaded, unchanged if its load is exactly the mean T*K/N.  Computed
+    in float32 (the stored precision of b), one rounding per step.
+
+    [P4] DeepSeekMoE paragraph (decrease by gamma when overloaded, increase by
+    gamma when under-loaded; gamma is the bias update speed); [P1] §1.2 (the
+    bias is not a gradient update and is adjusted at every step)."""
+    b = np.asarray(bias, dtype=np.float32)
+    c = np.asarray(counts, dtype=np.int64)
+    N = b.size
+    g = np.float32(gamma)
+    out = b.copy()
+    for i in range(N):
+        if c[i] * N > T * K:          # c_i > T*K/N, compared exactly
+            out[i] = np.float32(b[i] - g)
+        elif c[i] * N < T * K:
+            out[i] = np.float32(b[i] + g)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the whole layer
+# ---------------------------------------------------------------------------
+
+def moe_forward(x, router, bias, get_weights, G: int, topG: int, K: int,
+                tokens=None, h_round: str = "none", expert_fn=None) -> dict:
+    """Routing for every token, then the layer output for ``tokens`` (all by
+    default): y = E_shared(x) + sum_k gate_k * E_{idx_k}(x), float64.
+    Forward order DISPATCH -> MLP -> COMBINE as in [P1] §2.2."""
+    N = np.asarray(router).shape[0]
+    r = route(x, router, bias, G, topG, K)
+    d = dispatch(r["idx"], N)
+    ex = expert_outputs(x, r["idx"], get_weights, N, tokens, h_round, expert_fn)
+    y = combine(ex["shared"], ex["routed"], r["idx"], r["gate"], ex["tokens"])
+    return dict(route=r, dispatch=d, y=y, tokens=ex["tokens"], shared=ex["shared"],
+                routed=ex["routed"])
