@@ -1,0 +1,349 @@
+"""Throughput of the DeepSeekMoE layer forward on B200 GPUs.
+
+A step is one whole forward of the layer over one batch (route -> dispatch
+-> experts -> combine) plus the bias update, on synthetic seeded inputs of the
+DeepSeek-V3 shape (T=8192 tokens, d=7168, 256 routed + 1 shared experts,
+K=8, 8 groups / top-4, f=2048, bf16).  `value` is tokens/s over all ranks
+with inputs resident in HBM; `e2e` adds the host->device copy of x and the
+device->host copy of y to every step.  Each rank is an independent replica
+(the layer needs no exchange on one GPU), so scaling is weak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth import BY_NAME, gen  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at 1 B200 (bf16, FP8) and % of tensor/HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", default="v3_bf16")
+    p.add_argument("--cpu-sample", type=int, default=4, help="tokens per oracle sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def workload_name(cfg):
+    return (f"{cfg.name}: T={cfg.T} d={cfg.d} N={cfg.N}+1 K={cfg.K} groups={cfg.G}/top{cfg.topG} "
+            f"f={cfg.f} {cfg.dtype}")
+
+
+def flops_per_forward(cfg):
+    """Algorithmic FLOPs: router 2*T*d*N, experts 6*d*f per (token, expert)
+    for the K routed experts and the shared one."""
+    return 2.0 * cfg.T * cfg.d * cfg.N + 6.0 * cfg.d * cfg.f * cfg.T * (cfg.K + 1)
+
+
+def ffn_flops(cfg):
+    return 6.0 * cfg.d * cfg.f * cfg.T * (cfg.K + 1)
+
+
+def bytes_per_forward(cfg, counts):
+    """Algorithmic HBM bytes: weights of the experts that received rows plus
+    the shared expert, x in, y out, the fp32 router (bf16 elements)."""
+    used = int(np.count_nonzero(counts)) + 1
+    wb = used * 3 * cfg.d * cfg.f * 2
+    return wb + 2 * cfg.T * cfg.d * 2 + cfg.N * cfg.d * 4
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def cpu_oracle_baseline(cfg, n_tokens, seed=0, rounds=1):
+    """The float64 oracle as it stands on this host's cores: routing plus the
+    expert and combine work of `n_tokens` sampled tokens per round (weight
+    generation is excluded from the time).  Returns (tokens/s, cores, note)."""
+    import oracle
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    cores = len(os.sched_getaffinity(0))
+    total_t, total_tok = 0.0, 0
+    for r in range(rounds):
+        x = gen.make_x(cfg, seed, batch=1000 + r)[:max(n_tokens, 1)]
+        gen_time = [0.0]
+
+        def get(e):
+            t0 = time.perf_counter()
+            w = tuple(gen.make_expert_weight(cfg, seed, w, e).astype(np.float64)
+                      for w in ("w1", "w3", "w2"))
+            gen_time[0] += time.perf_counter() - t0
+            return w
+
+        t0 = time.perf_counter()
+        oracle.moe_forward(x, R, b, get, cfg.G, cfg.topG, cfg.K,
+                           h_round="none" if cfg.dtype == "fp32" else "bf16")
+        total_t += time.perf_counter() - t0 - gen_time[0]
+        total_tok += x.shape[0]
+    note = (f"{total_tok} tokens of the {cfg.name} workload (full routing and expert math per "
+            f"token, weight generation excluded), numpy float64 on {cores} cores")
+    return total_tok / total_t, cores, note
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    return world, rank, local, pg
+
+
+def run_reference(args, cfg):
+    world, rank, local, pg = dist_setup(args)
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    times = []
+    n = max(1, args.cpu_sample)
+    for _ in range(args.warmup):
+        cpu_oracle_baseline(cfg, 1)
+    cores = len(os.sched_getaffinity(0))
+    note = ""
+    for _ in range(args.steps):
+        v, cores, note = cpu_oracle_baseline(cfg, n)
+        times.append(n / v)
+    value = n * len(times) / sum(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(cfg), "sample_tokens_per_step": n},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": note},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    cfg = BY_NAME[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import sparse_moe_layer_limited_b200 as M
+    from synth import device as sdev
+
+    world, rank, local, pg = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    s = M.shape(cfg.T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f,
+                {"fp32": M.DTYPE_FP32, "bf16": M.DTYPE_BF16, "e4m3": M.DTYPE_E4M3}[cfg.dtype])
+
+    # ---- inputs resident in HBM (weights generated on the device) ----
+    w1 = sdev.expert_weights_bf16(cfg, 0, "w1", dev)
+    w3 = sdev.expert_weights_bf16(cfg, 0, "w3", dev)
+    w13 = torch.empty(cfg.N + 1, 2 * cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
+    M.moe_pack_w13(s, w1, w3, w13)
+    del w1, w3
+    w2 = sdev.expert_weights_bf16(cfg, 0, "w2", dev)
+    router = torch.from_numpy(gen.make_router(cfg)).to(dev)
+    bias = torch.from_numpy(gen.make_bias(cfg)).to(dev)
+    x = sdev.x_bf16(cfg, 0, 0, dev)
+    layer = M.MoELayer(s, router, bias, w13, w2, gamma=cfg.gamma)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream(dev)
+    phases = ["route", "dispatch", "experts", "combine", "bias"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        M.moe_route(s, x, router, layer.bias, layer.topk_idx, layer.topk_gate, layer.counts,
+                    layer.ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        M.moe_dispatch(s, x, layer.topk_idx, layer.counts, layer.offsets, layer.perm_tok,
+                       layer.slot, layer.x_perm, layer.x_perm_scales, layer.ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        M.moe_expert_ffn(s, layer.x_perm, layer.x_perm_scales, layer.offsets, x, w13, w2,
+                         None, None, layer.y_perm, layer.y_shared, layer.ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        M.moe_combine(s, layer.y_perm, layer.y_shared, layer.slot, layer.topk_gate, layer.y,
+                      stream)
+        if ev is not None:
+            ev[4].record(stream)
+        M.moe_bias_update(s, layer.counts, layer.bias, cfg.gamma, stream)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            step(evs[k])
+        torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    per_phase = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]
+                 for i, p in enumerate(phases)}
+    total_ms = evs[0][0].elapsed_time(evs[-1][5])
+    counts = layer.counts.cpu().numpy()
+    status = layer.device_status()
+
+    # ---- end to end through the public API with host buffers ----
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+    x_dev2 = torch.empty_like(x)
+    for _ in range(2):
+        x_dev2.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev2, stream=stream)
+        y_host.copy_(layer.y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev2.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev2, stream=stream)
+        y_host.copy_(layer.y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if pg is not None:
+        t = torch.tensor([total_ms, e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms, e2e_ms = t.tolist()
+
+    if rank == 0:
+        P = peaks()
+        ms_step = total_ms / args.steps
+        value = world * cfg.T * args.steps / (total_ms / 1e3)
+        ffn_ms = statistics.mean(per_phase["experts"])
+        achieved = ffn_flops(cfg) / (ffn_ms / 1e3) / 1e12
+        fl = flops_per_forward(cfg)
+        by = bytes_per_forward(cfg, counts)
+        roof_ms = max(fl / (P["bf16"] * 1e12), by / (P["hbm"] * 1e9)) * 1e3
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
+            "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
+                       "l2": "inputs larger than L2: the 22.6 GB of expert weights stream "
+                             "through it every step",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, "
+                         "GEMM2)", "achieved": achieved, "peak": P["bf16"], "unit": "TFLOP/s",
+                         "frac": achieved / P["bf16"], "peak_source": P["source"] + " burst",
+                         "traffic": None},
+            "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step,
+                               "flops": fl, "bytes": by},
+            "phases_ms": {p: statistics.mean(v) for p, v in per_phase.items()},
+            "e2e": {"value": world * cfg.T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": cfg.T * cfg.d * 2,
+                    "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+            "gpu_launches": 8 * args.steps,
+            "clocks": clk.summary(),
+            "device_status": status,
+            "load_max_over_mean": float(counts.max() / counts.mean()),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, cores, note = cpu_oracle_baseline(cfg, args.cpu_sample)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
+                                    "kind": "oracle", "sample": note}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

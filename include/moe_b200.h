@@ -1,0 +1,210 @@
+/*
+ * moe_b200.h -- C ABI of the DeepSeekMoE layer forward for one NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer (per token t, N routed experts, one shared expert):
+ *   s_i   = sigmoid(x_t . e_i)                       affinity
+ *   s'_i  = s_i + b_i                                biased score, selection only
+ *   keep the topG of G contiguous expert groups by group score (sum of the two
+ *   largest s' in the group), then idx = the K largest s' inside kept groups
+ *   gate_k = s_{idx_k} / sum_j s_{idx_j}             un-biased, renormalised
+ *   y_t = E_shared(x_t) + sum_k gate_k * E_{idx_k}(x_t)
+ *   E(a) = (silu(a W1^T) * (a W3^T)) W2^T            SwiGLU expert
+ *   after the step: b_i -= gamma if expert i took more than T*K/N rows,
+ *                   b_i += gamma if it took fewer.
+ *
+ * Sources (web pages on DeepSeek-V3):
+ *   [P1] "DeepSeek-V3 高效训练关键技术分析" (mhpq.cn): §1.1 DeepSeekMoE (1 shared +
+ *        256 routed experts, 8 active), §1.2 auxiliary-loss-free balancing (bias
+ *        adjusted every step from the measured load), §2.2 forward order
+ *        DISPATCH -> MLP -> COMBINE, §3.1 each token reaches at most 4 nodes,
+ *        §4.1 FP8 GEMMs with 1x128 activation / 128x128 weight scaling and
+ *        online max-abs scales, FP32 accumulation.
+ *   [P2] "解读 DeepSeek-V3" reading notes (gkm0120.cn), Q3: the bias enters
+ *        routing only, never the gate value.
+ *   [P4] DeepSeek-V3 walk-through (kaiyunto.com), DeepSeekMoE paragraphs:
+ *        sigmoid affinity, gate = normalisation over the selected affinities,
+ *        bias -gamma when overloaded, +gamma when under-loaded.
+ *   [P5] "DeepSeek-V3核心技术解析" (wenxiaobai), §二(一)4: top-K by affinity,
+ *        the shared expert always participates.
+ * Readings where the pages are silent: top-2-sum group score, contiguous groups,
+ * SwiGLU without biases, no routed scaling factor, lower index wins exact ties,
+ * FP8 scale = amax/448 in fp32.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     16-byte aligned; the library allocates and frees nothing.
+ *   - `stream` is a cudaStream_t (passed as void*); every call only enqueues
+ *     work on it and returns without synchronising.
+ *   - Return value: MOE_OK or a negative MOE_ERR_* status; nothing is enqueued
+ *     when an argument check fails.  No exception or exit crosses the ABI.
+ *   - Device-side failures (a pipeline wait that gave up, an expert index out
+ *     of range, inconsistent counts) are OR-ed into the status word at the
+ *     start of the workspace; read it with moe_read_device_status().
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer shape.  dtype selects the expert-GEMM arithmetic:
+ *   MOE_DTYPE_FP32: x, weights, y fp32; SIMT fp32 experts.
+ *   MOE_DTYPE_BF16: x, weights, y bf16; tcgen05 bf16 MMAs, fp32 accumulate.
+ *   MOE_DTYPE_E4M3: x, y bf16; expert GEMMs in E4M3 with fp32 block scales
+ *                   (1x128 activations, 128x128 weights), fp32 accumulate.
+ * The router is fp32 in every mode. */
+typedef struct moe_shape {
+  int32_t T;     /* tokens */
+  int32_t d;     /* model width */
+  int32_t N;     /* routed experts (the shared expert is index N) */
+  int32_t K;     /* routed experts per token */
+  int32_t G;     /* expert groups (contiguous, N/G experts each) */
+  int32_t topG;  /* groups a token may reach */
+  int32_t f;     /* expert inner width */
+  int32_t dtype; /* MOE_DTYPE_* */
+} moe_shape;
+
+enum {
+  MOE_DTYPE_FP32 = 0,
+  MOE_DTYPE_BF16 = 1,
+  MOE_DTYPE_E4M3 = 2
+};
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = -1,         /* null pointer, non-positive size, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = -2, /* shape or dtype outside what the kernels handle */
+  MOE_ERR_WORKSPACE = -3,   /* workspace smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = -4,        /* a CUDA launch or API call failed */
+  MOE_ERR_DEVICE = -5       /* the device status word is non-zero */
+};
+
+/* Device status bits (moe_read_device_status). */
+enum {
+  MOE_DEV_WAIT_TIMEOUT = 1,   /* a tensor-core pipeline wait gave up after ~2 s */
+  MOE_DEV_COUNT_MISMATCH = 2, /* counts[] disagree with the expert indices */
+  MOE_DEV_BAD_INDEX = 4       /* an expert index outside [0, N) */
+};
+
+/* Human-readable text for a MOE_* status.  Never NULL; static storage. */
+const char* moe_status_string(int status);
+
+/* Check a shape: MOE_OK, MOE_ERR_ARG or MOE_ERR_UNSUPPORTED.
+ * Supported: T >= 1; 1 <= K <= min(32, topG*N/G); N <= 256; G divides N;
+ * 1 <= topG <= G; for BF16 and E4M3 also d % 256 == 0 and f % 128 == 0;
+ * for FP32 also d % 4 == 0. */
+int moe_check_shape(const moe_shape* shape);
+
+/* Bytes of scratch every entry point of this shape may use (one buffer serves
+ * all of them; calls on the same stream may share it).  The first 256 bytes
+ * hold the device status word: zero them once after allocating
+ * (moe_workspace_init) and read them with moe_read_device_status.
+ * Returns 0 for an invalid shape. */
+size_t moe_workspace_size(const moe_shape* shape);
+
+/* Zero the device status word of `ws` (enqueued on `stream`). */
+int moe_workspace_init(void* ws, void* stream);
+
+/* Synchronise `stream`, then copy the device status word of `ws` into
+ * *status_out (0 = no device-side failure).  When `clear` is non-zero the word
+ * is reset to 0 afterwards.  Returns MOE_OK, or MOE_ERR_DEVICE when the word
+ * was non-zero. */
+int moe_read_device_status(void* ws, void* stream, uint32_t* status_out, int clear);
+
+/* Routing: affinity, biased group-limited top-K, gates and per-expert counts.
+ * [P4] sigmoid affinity and gate normalisation; [P2] Q3 / [P1] §1.2 bias for
+ * selection only; [P1] §3.1 group limit; [P5] top-K by affinity.
+ *   x          [T, d]  fp32 (FP32 mode) or bf16 (BF16/E4M3 modes)
+ *   router_w   [N, d]  fp32, row i = e_i
+ *   bias       [N]     fp32
+ *   topk_idx   [T, K]  int32 out, ascending expert id per token
+ *   topk_gate  [T, K]  fp32 out, gate of topk_idx[t, k]; each row sums to 1
+ *   counts     [N]     int32 out, tokens routed to each expert (sum = T*K)
+ *   ws         workspace of moe_workspace_size(shape) bytes
+ * Scores are fp32 (dot products accumulated in fp32); an exact tie between
+ * two scores goes to the lower expert (or group) index. */
+int moe_route(const moe_shape* shape, const void* x, const float* router_w, const float* bias,
+              int32_t* topk_idx, float* topk_gate, int32_t* counts, void* ws, void* stream);
+
+/* Dispatch ([P1] §2.2 DISPATCH, single-GPU permutation): group the T*K
+ * (token, expert) pairs by expert.  Row order is experts ascending, tokens
+ * ascending within an expert, so the result is deterministic.
+ *   topk_idx   [T, K]  int32 (from moe_route)
+ *   counts     [N]     int32 (from moe_route)
+ *   offsets    [N+1]   int32 out, first row of each expert; offsets[N] = T*K
+ *   perm_tok   [T*K]   int32 out, token of each row
+ *   slot       [T, K]  int32 out, row holding (t, topk_idx[t, k])
+ *   x_perm     [T*K, d] out: bf16 copy of x rows (BF16), fp32 (FP32), or E4M3
+ *                      codes (E4M3 mode, one byte per element)
+ *   x_perm_scales [T*K, d/128] fp32 out, E4M3 mode only (NULL otherwise):
+ *                      per-1x128-tile scale amax/448 ([P1] §4.1)
+ * Sets MOE_DEV_COUNT_MISMATCH if counts disagree with topk_idx. */
+int moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                 const int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* slot,
+                 void* x_perm, float* x_perm_scales, void* ws, void* stream);
+
+/* Experts: the N routed SwiGLU experts on their dispatched rows and the shared
+ * expert (index N) on all T rows of x, in one pass per GEMM
+ * ([P1] §1.1, [P5]; SwiGLU is this library's reading of "FFN").
+ *   x_perm, x_perm_scales, offsets   from moe_dispatch
+ *   x          [T, d]  layer input (fp32 or bf16), input of the shared expert
+ *   w13        [N+1, 2f, d] packed W1/W3 (moe_pack_w13): for each 128-row block
+ *              j of W1 and W3, rows 256j..256j+127 are W1 rows 128j.. and rows
+ *              256j+128..256j+255 are W3 rows 128j..  (bf16 / fp32 / E4M3 codes)
+ *   w2         [N+1, d, f]  (bf16 / fp32 / E4M3 codes)
+ *   w13_scales [N+1, 2f/128, d/128], w2_scales [N+1, d/128, f/128] fp32,
+ *              E4M3 mode only (from moe_quantize_weights), else NULL
+ *   y_perm     [T*K, d] out (fp32 in FP32 mode, else bf16): E_{expert}(row)
+ *   y_shared   [T, d]   out: E_shared(x)
+ * The hidden activation h is held in the workspace as bf16 (BF16), fp32 (FP32)
+ * or E4M3 with 1x128 scales (E4M3). */
+int moe_expert_ffn(const moe_shape* shape, const void* x_perm, const float* x_perm_scales,
+                   const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                   const float* w13_scales, const float* w2_scales, void* y_perm,
+                   void* y_shared, void* ws, void* stream);
+
+/* Combine ([P1] §2.2 COMBINE): y[t] = y_shared[t] + sum_k gate[t,k] *
+ * y_perm[slot[t,k]], accumulated in fp32 in k order, rounded once to the
+ * output dtype (fp32 in FP32 mode, else bf16).  No atomics: deterministic. */
+int moe_combine(const moe_shape* shape, const void* y_perm, const void* y_shared,
+                const int32_t* slot, const float* topk_gate, void* y, void* stream);
+
+/* Auxiliary-loss-free bias update ([P4]; [P1] §1.2): for every expert,
+ * bias[i] -= gamma if counts[i] * N > T * K, += gamma if counts[i] * N < T * K,
+ * unchanged otherwise; fp32, in place. */
+int moe_bias_update(const moe_shape* shape, const int32_t* counts, float* bias, float gamma,
+                    void* stream);
+
+/* Weight preparation (not part of the timed forward).
+ * moe_pack_w13: w1, w3 [N+1, f, d] -> w13 [N+1, 2f, d] in the 128-row block
+ * interleave described at moe_expert_ffn (element type per shape->dtype; for
+ * E4M3 pass the bf16 weights here, then moe_quantize_weights). */
+int moe_pack_w13(const moe_shape* shape, const void* w1, const void* w3, void* w13, void* stream);
+
+/* moe_quantize_weights (E4M3 mode): per 128x128 block of each expert matrix,
+ * scale = amax/448 (fp32), codes = E4M3_RNE_satfinite(w * (448/amax)).
+ *   w13_bf16 [N+1, 2f, d] (packed), w2_bf16 [N+1, d, f]
+ *   w13_q / w2_q: E4M3 codes of the same shapes; scales as at moe_expert_ffn. */
+int moe_quantize_weights(const moe_shape* shape, const void* w13_bf16, const void* w2_bf16,
+                         void* w13_q, float* w13_scales, void* w2_q, float* w2_scales,
+                         void* stream);
+
+/* The whole forward in order: route, dispatch, experts, combine, then the bias
+ * update; intermediate buffers are caller-provided as in the calls above. */
+int moe_forward(const moe_shape* shape, const void* x, const float* router_w, float* bias,
+                float gamma, const void* w13, const void* w2, const float* w13_scales,
+                const float* w2_scales, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                int32_t* offsets, int32_t* perm_tok, int32_t* slot, void* x_perm,
+                float* x_perm_scales, void* y_perm, void* y_shared, void* y, void* ws,
+                void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

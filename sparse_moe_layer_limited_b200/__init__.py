@@ -1,0 +1,15 @@
+"""DeepSeekMoE layer forward for one NVIDIA B200 (sm_100a).
+
+The compute runs in ``libmoe_b200.so`` (hand-written CUDA, C ABI declared in
+``include/moe_b200.h``); this package only marshals arguments.  Import fails
+loudly when the library has not been built.
+"""
+from ._lib import (  # noqa: F401
+    DTYPE_BF16, DTYPE_E4M3, DTYPE_FP32, MoEError, MoEShape, check_shape, lib, moe_bias_update,
+    moe_combine, moe_dispatch, moe_expert_ffn, moe_forward, moe_pack_w13, moe_quantize_weights,
+    moe_read_device_status, moe_route, moe_workspace_init, shape, status_string,
+    workspace_size, x_torch_dtype, w_torch_dtype,
+)
+from .layer import MoELayer  # noqa: F401
+
+lib()

@@ -1,0 +1,204 @@
+"""ctypes binding of libmoe_b200.so: argument marshalling only.
+
+Each function takes torch tensors (device memory from PyTorch), checks their
+dtype/shape/placement, and calls the C entry point of the same name; every
+step of the computation runs in the library's CUDA kernels.  A missing
+library is an error: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB_PATH
+
+DTYPE_FP32, DTYPE_BF16, DTYPE_E4M3 = 0, 1, 2
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = 0, -1, -2, -3, -4, -5
+
+_c_p = ctypes.c_void_p
+
+
+class MoEShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("G", ctypes.c_int32), ("topG", ctypes.c_int32),
+                ("f", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "MoEShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        self.status = status
+
+
+_SIGS = {
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_check_shape": (ctypes.c_int, [ctypes.POINTER(MoEShape)]),
+    "moe_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
+    "moe_workspace_init": (ctypes.c_int, [_c_p, _c_p]),
+    "moe_read_device_status": (ctypes.c_int, [_c_p, _c_p, ctypes.POINTER(ctypes.c_uint32),
+                                              ctypes.c_int]),
+    "moe_route": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 8),
+    "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 10),
+    "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
+    "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
+    "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, ctypes.c_float,
+                                       _c_p]),
+    "moe_pack_w13": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 4),
+    "moe_quantize_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
+    "moe_forward": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, _c_p, ctypes.c_float]
+                    + [_c_p] * 17),
+}
+
+_lib = None
+
+
+def lib():
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} missing: build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def shape(T, d, N, K, G, topG, f, dtype) -> MoEShape:
+    return MoEShape(T, d, N, K, G, topG, f, dtype)
+
+
+def check_shape(s: MoEShape) -> int:
+    return lib().moe_check_shape(ctypes.byref(s))
+
+
+def workspace_size(s: MoEShape) -> int:
+    return lib().moe_workspace_size(ctypes.byref(s))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _call(name, *args):
+    rc = getattr(lib(), name)(*args)
+    if rc != OK:
+        raise MoEError(name, rc)
+
+
+def _expect(t, dtype, numel, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name}: expected {numel} elements, got {t.numel()}")
+
+
+def x_torch_dtype(s: MoEShape):
+    return torch.float32 if s.dtype == DTYPE_FP32 else torch.bfloat16
+
+
+def w_torch_dtype(s: MoEShape):
+    return {DTYPE_FP32: torch.float32, DTYPE_BF16: torch.bfloat16,
+            DTYPE_E4M3: torch.float8_e4m3fn}[s.dtype]
+
+
+def moe_workspace_init(ws, stream=None):
+    _call("moe_workspace_init", _ptr(ws), _stream(stream))
+
+
+def moe_read_device_status(ws, stream=None, clear=False) -> int:
+    v = ctypes.c_uint32(0)
+    rc = lib().moe_read_device_status(_ptr(ws), _stream(stream), ctypes.byref(v), int(clear))
+    if rc not in (OK, ERR_DEVICE):
+        raise MoEError("moe_read_device_status", rc)
+    return int(v.value)
+
+
+def moe_route(s, x, router_w, bias, topk_idx, topk_gate, counts, ws, stream=None):
+    _expect(x, x_torch_dtype(s), s.T * s.d, "x")
+    _expect(router_w, torch.float32, s.N * s.d, "router_w")
+    _expect(bias, torch.float32, s.N, "bias")
+    _expect(topk_idx, torch.int32, s.T * s.K, "topk_idx")
+    _expect(topk_gate, torch.float32, s.T * s.K, "topk_gate")
+    _expect(counts, torch.int32, s.N, "counts")
+    _call("moe_route", ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(topk_idx),
+          _ptr(topk_gate), _ptr(counts), _ptr(ws), _stream(stream))
+
+
+def moe_dispatch(s, x, topk_idx, counts, offsets, perm_tok, slot, x_perm, x_perm_scales, ws,
+                 stream=None):
+    _expect(offsets, torch.int32, s.N + 1, "offsets")
+    _expect(perm_tok, torch.int32, s.T * s.K, "perm_tok")
+    _expect(slot, torch.int32, s.T * s.K, "slot")
+    _expect(x_perm, w_torch_dtype(s) if s.dtype == DTYPE_E4M3 else x_torch_dtype(s),
+            s.T * s.K * s.d, "x_perm")
+    _call("moe_dispatch", ctypes.byref(s), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+          _ptr(perm_tok), _ptr(slot), _ptr(x_perm), _ptr(x_perm_scales), _ptr(ws),
+          _stream(stream))
+
+
+def moe_expert_ffn(s, x_perm, x_perm_scales, offsets, x, w13, w2, w13_scales, w2_scales,
+                   y_perm, y_shared, ws, stream=None):
+    _expect(w13, w_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "w13")
+    _expect(w2, w_torch_dtype(s), (s.N + 1) * s.d * s.f, "w2")
+    _expect(y_perm, x_torch_dtype(s), s.T * s.K * s.d, "y_perm")
+    _expect(y_shared, x_torch_dtype(s), s.T * s.d, "y_shared")
+    _call("moe_expert_ffn", ctypes.byref(s), _ptr(x_perm), _ptr(x_perm_scales), _ptr(offsets),
+          _ptr(x), _ptr(w13), _ptr(w2), _ptr(w13_scales), _ptr(w2_scales), _ptr(y_perm),
+          _ptr(y_shared), _ptr(ws), _stream(stream))
+
+
+def moe_combine(s, y_perm, y_shared, slot, topk_gate, y, stream=None):
+    _expect(y, x_torch_dtype(s), s.T * s.d, "y")
+    _call("moe_combine", ctypes.byref(s), _ptr(y_perm), _ptr(y_shared), _ptr(slot),
+          _ptr(topk_gate), _ptr(y), _stream(stream))
+
+
+def moe_bias_update(s, counts, bias, gamma, stream=None):
+    _expect(counts, torch.int32, s.N, "counts")
+    _expect(bias, torch.float32, s.N, "bias")
+    _call("moe_bias_update", ctypes.byref(s), _ptr(counts), _ptr(bias), ctypes.c_float(gamma),
+          _stream(stream))
+
+
+def moe_pack_w13(s, w1, w3, w13, stream=None):
+    _call("moe_pack_w13", ctypes.byref(s), _ptr(w1), _ptr(w3), _ptr(w13), _stream(stream))
+
+
+def moe_quantize_weights(s, w13_bf16, w2_bf16, w13_q, w13_scales, w2_q, w2_scales, stream=None):
+    _call("moe_quantize_weights", ctypes.byref(s), _ptr(w13_bf16), _ptr(w2_bf16), _ptr(w13_q),
+          _ptr(w13_scales), _ptr(w2_q), _ptr(w2_scales), _stream(stream))
+
+
+def moe_forward(s, x, router_w, bias, gamma, w13, w2, w13_scales, w2_scales, topk_idx,
+                topk_gate, counts, offsets, perm_tok, slot, x_perm, x_perm_scales, y_perm,
+                y_shared, y, ws, stream=None):
+    _call("moe_forward", ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(bias),
+          ctypes.c_float(gamma), _ptr(w13), _ptr(w2), _ptr(w13_scales), _ptr(w2_scales),
+          _ptr(topk_idx), _ptr(topk_gate), _ptr(counts), _ptr(offsets), _ptr(perm_tok),
+          _ptr(slot), _ptr(x_perm), _ptr(x_perm_scales), _ptr(y_perm), _ptr(y_shared), _ptr(y),
+          _ptr(ws), _stream(stream))

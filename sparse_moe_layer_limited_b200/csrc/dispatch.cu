@@ -1,0 +1,182 @@
+// Dispatch: deterministic grouping of the (token, expert) pairs by expert
+// and the gather of x rows into expert order (the DISPATCH step of the
+// forward order ATTN -> DISPATCH -> MLP -> COMBINE, mhpq.cn article §2.2; on
+// one GPU it is a permutation, not an all-to-all).
+//
+// Row of (t, e) = offsets[e] + #{t' < t : t' chose e}.  Computed without
+// atomics in three launches:
+//   1. per 32-token chunk, a histogram of the chosen experts;
+//   2. per expert (one CTA each), the exclusive prefix over experts of
+//      counts[] and over chunks of that expert's histogram column;
+//   3. per chunk, each pair's rank among the chunk's earlier tokens, the slot
+//      and perm_tok writes, then the row gather: one warp per token reads x
+//      once with 16-byte loads and writes it to its K destination rows
+//      (E4M3 mode: quantised per 1x128 tile on the way, mhpq.cn §4.1).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ idx, int T,
+                                                         int K, int N,
+                                                         int32_t* __restrict__ chunk_hist,
+                                                         uint32_t* __restrict__ status) {
+  __shared__ int h[kRouteMaxN];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < N; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const int t0 = c * kChunkTokens;
+  const int nt = min(kChunkTokens, T - t0);
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) {
+    const int e = idx[(size_t)t0 * K + p];
+    if (e < 0 || e >= N)
+      atomicOr(status, kErrBadIndex);
+    else
+      atomicAdd(&h[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) chunk_hist[(size_t)c * N + e] = h[e];
+}
+
+__device__ __forceinline__ int block_sum_256(int v, int* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  int s = 0;
+  for (int i = 0; i < 8; ++i) s += red[i];
+  return s;
+}
+
+// Exclusive scan of one int per thread over a 256-thread block.
+__device__ __forceinline__ int block_exclusive_scan_256(int v, int* red) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (l >= o) inc += n;
+  }
+  __syncthreads();
+  if (l == 31) red[w] = inc;
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < w; ++i) base += red[i];
+  return base + inc - v;
+}
+
+__global__ void __launch_bounds__(256) expert_scan_kernel(const int32_t* __restrict__ counts,
+                                                          const int32_t* __restrict__ chunk_hist,
+                                                          int nchunks, int N,
+                                                          int32_t* __restrict__ offsets,
+                                                          int32_t* __restrict__ chunk_base,
+                                                          uint32_t* __restrict__ status) {
+  __shared__ int red[8];
+  const int e = blockIdx.x;
+  int part = 0;
+  for (int i = threadIdx.x; i < e; i += blockDim.x) part += counts[i];
+  const int off_e = block_sum_256(part, red);
+
+  const int per = (nchunks + blockDim.x - 1) / blockDim.x;
+  const int c0 = threadIdx.x * per;
+  const int c1 = min(nchunks, c0 + per);
+  int mine = 0;
+  for (int c = c0; c < c1; ++c) mine += chunk_hist[(size_t)c * N + e];
+  int run = off_e + block_exclusive_scan_256(mine, red);
+  for (int c = c0; c < c1; ++c) {
+    chunk_base[(size_t)c * N + e] = run;
+    run += chunk_hist[(size_t)c * N + e];
+  }
+  const int total = block_sum_256(mine, red);
+  if (threadIdx.x == 0) {
+    const int ce = counts[e];
+    if (total != ce) atomicOr(status, kErrCountMismatch);
+    offsets[e] = off_e;
+    if (e == N - 1) offsets[N] = off_e + ce;
+  }
+}
+
+// Slots for one chunk, then the row gather (bf16 / fp32 rows copied verbatim).
+template <typename XT>
+__global__ void __launch_bounds__(256) scatter_gather_kernel(
+    const XT* __restrict__ x, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ chunk_base, int T, int d, int K, int N,
+    int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot, XT* __restrict__ x_perm) {
+  __shared__ int sidx[kChunkTokens * kMaxK];
+  __shared__ int sslot[kChunkTokens * kMaxK];
+  const int c = blockIdx.x;
+  const int t0 = c * kChunkTokens;
+  const int nt = min(kChunkTokens, T - t0);
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) sidx[p] = idx[(size_t)t0 * K + p];
+  __syncthreads();
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) {
+    const int tl = p / K;
+    const int e = sidx[p];
+    if (e < 0 || e >= N) {  // flagged by the histogram kernel; keep writes in bounds
+      sslot[p] = -1;
+      continue;
+    }
+    int rank = 0;
+    for (int q = 0; q < tl * K; ++q) rank += (sidx[q] == e) ? 1 : 0;
+    const int r = chunk_base[(size_t)c * N + e] + rank;
+    if (r < 0 || r >= T * K) {  // only when counts[] disagree with idx (flagged)
+      sslot[p] = -1;
+      continue;
+    }
+    sslot[p] = r;
+    slot[(size_t)t0 * K + p] = r;
+    perm_tok[r] = t0 + tl;
+  }
+  __syncthreads();
+  // gather: warp per token, 16-byte vectors
+  constexpr int kElems = 16 / sizeof(XT);
+  const int nvec = d / kElems;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int tl = warp; tl < nt; tl += 8) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t0 + tl) * d);
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 val = __ldg(src + v);
+      for (int k = 0; k < K; ++k) {
+        const int r = sslot[tl * K + k];
+        if (r >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)r * d)[v] = val;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* idx,
+                            const int32_t* counts, int32_t* offsets, int32_t* perm_tok,
+                            int32_t* slot, void* x_perm, float* x_perm_scales, void* ws,
+                            cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
+  int32_t* chunk_hist = reinterpret_cast<int32_t*>(w + L.chunk_hist);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(w + L.chunk_base);
+  const int nch = chunks_of(s.T);
+  chunk_hist_kernel<<<nch, 256, 0, st>>>(idx, s.T, s.K, s.N, chunk_hist, status);
+  expert_scan_kernel<<<s.N, 256, 0, st>>>(counts, chunk_hist, nch, s.N, offsets, chunk_base,
+                                          status);
+  if (s.dtype == MOE_DTYPE_FP32)
+    scatter_gather_kernel<float><<<nch, 256, 0, st>>>(
+        static_cast<const float*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok, slot,
+        static_cast<float*>(x_perm));
+  else if (s.dtype == MOE_DTYPE_BF16)
+    scatter_gather_kernel<__nv_bfloat16><<<nch, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
+        slot, static_cast<__nv_bfloat16*>(x_perm));
+  else
+    return cudaErrorNotSupported;
+  (void)x_perm_scales;
+  return cudaGetLastError();
+}
+
+}  // namespace moe

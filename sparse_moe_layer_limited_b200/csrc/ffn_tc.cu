@@ -1,0 +1,404 @@
+// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores (bf16).
+//
+// The experts are FFNs (mhpq.cn article §1.1; wenxiaobai §二(一)4) in the
+// SwiGLU form y = (silu(a W1^T) * (a W3^T)) W2^T; the routed experts run on
+// their dispatched rows and the shared expert on every token, all in one
+// persistent launch per GEMM:
+//   GEMM1  [rows_g, d] x [d, 2f] -> SwiGLU epilogue -> H [rows_g, f] (bf16)
+//   GEMM2  [rows_g, f] x [f, d]  -> Y [rows_g, d] (bf16)
+// Group g < N is routed expert g (rows offsets[g]..offsets[g+1]); group N is
+// the shared expert (T rows).
+//
+// Work unit: a 128 x 256 output tile (tcgen05.mma cta_group::1, M=128,
+// N=256, K=16 per instruction), ordered group-major, then n-tile, then
+// m-tile, so CTAs running side by side share the same weight tile through
+// L2 and each expert's weights stream from HBM about once.  Each CTA (one
+// per SM) walks tiles blockIdx.x, +gridDim.x, ... with three roles:
+//   warp 0    one thread issues TMA loads of 64-wide K slices of A and B
+//             (128-byte swizzle) into a 4-stage shared-memory ring;
+//   warp 1    allocates 512 TMEM columns (two 256-column accumulators) and
+//             one thread issues the MMAs, committing each ring slot back to
+//             the producer and each finished accumulator to the epilogue;
+//   warps 2-5 drain an accumulator with tcgen05.ld (one TMEM lane = one
+//             output row per thread) while the next tile accumulates in the
+//             other buffer, apply SwiGLU (GEMM1), round to bf16 and store
+//             the rows that belong to the group.
+// In GEMM1 the packed weight rows hold, per 128-row block j, W1 rows then
+// W3 rows, so one accumulator tile holds matching gate and up columns.
+// Every mbarrier wait is bounded (~2 s); a wait that gives up sets the
+// device status word and the CTA unwinds, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;  // BK bf16 = 128 bytes = one swizzle row
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;
+constexpr int kBBytes = BN * BK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+enum Epi { kEpiSwiGLU = 0, kEpiStore = 1 };
+
+struct alignas(64) GemmArgs {
+  CUtensorMap tmA_routed;
+  CUtensorMap tmA_shared;
+  CUtensorMap tmB;
+  const int32_t* offsets;
+  __nv_bfloat16* out_routed;
+  __nv_bfloat16* out_shared;
+  uint32_t* status;
+  int N, T;
+  int rows_routed;  // T*K
+  int a_shared_row0;
+  int n_acc;   // accumulator columns per expert (2f for GEMM1, d for GEMM2)
+  int k_dim;   // contraction length
+  int out_ld;  // output row stride in elements
+};
+
+__host__ __device__ constexpr size_t smem_bytes_for(int groups) {
+  return 1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(groups + 1) * 4;
+}
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) {
+  uint4 w[4];
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = w[i];
+}
+
+template <int kEpi>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
+    const __grid_constant__ GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)kStages * kStageBytes);
+  uint64_t* full = bars;                 // [kStages]
+  uint64_t* empty = bars + kStages;      // [kStages]
+  uint64_t* tfull = bars + 2 * kStages;  // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* drain = tempty + 2;          // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  int* tile_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + 256);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int G1 = args.N + 1;
+  const int NT = args.n_acc / BN;
+  const int KB = args.k_dim / BK;
+
+  // ---- set-up: barriers, TMEM, tile schedule --------------------------------
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int g = tid; g < G1; g += kThreads) {
+    const int rows = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+    tile_start[g] = rows > 0 ? (rows + BM - 1) / BM : 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {  // exclusive scan of m-tiles per group, times NT
+    const int per = (G1 + 31) / 32;
+    const int g0 = min(G1, lane * per), g1 = min(G1, g0 + per);
+    int sum = 0;
+    for (int g = g0; g < g1; ++g) sum += tile_start[g];
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    int run = inc - sum;
+    for (int g = g0; g < g1; ++g) {
+      const int mt = tile_start[g];
+      tile_start[g] = run * NT;
+      run += mt;
+    }
+    if (lane == 31) tile_start[G1] = inc * NT;
+  }
+  __syncthreads();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = tile_start[G1];
+
+  auto decode = [&](int tile, int& g, int& n, int& m, int& mt) {
+    int lo = 0, hi = G1;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_start[mid] <= tile) lo = mid; else hi = mid;
+    }
+    g = lo;
+    mt = (tile_start[g + 1] - tile_start[g]) / NT;
+    const int local = tile - tile_start[g];
+    n = local / mt;
+    m = local - n * mt;
+  };
+
+  if (warp == 0) {
+    // ---- TMA producer ---------------------------------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&args.tmA_routed);
+      tma_prefetch_desc(&args.tmA_shared);
+      tma_prefetch_desc(&args.tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, n, m, mt;
+        decode(tile, g, n, m, mt);
+        const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
+        const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * BM;
+        const int brow = g * args.n_acc + n * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = base + (size_t)stage * kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          tma_load_2d(sa, am, kb * BK, arow, &full[stage]);
+          tma_load_2d(sa + kABytes, &args.tmB, kb * BK, brow, &full[stage]);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {  // let the copies already issued land before the CTA exits
+        for (int s = 0; s < kStages; ++s)
+          if ((issued >> s) & 1u)
+            mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.status, kTimeoutNs / 8);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer -----------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t aphase = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], aphase ^ 1u, args.status, kTimeoutNs)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, args.status, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(base + (size_t)stage * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
+                     (kb | k) != 0);
+          mma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit(&tfull[acc]);
+      }
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0, args.status, kTimeoutNs / 8);
+    }
+  } else {
+    // ---- epilogue: warps 2..5 --------------------------------------------------
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      int g, n, m, mt;
+      decode(tile, g, n, m, mt);
+      const int acc = local & 1;
+      const uint32_t aphase = (local >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], aphase, args.status, kTimeoutNs)) break;
+      tc_fence_after();
+      const int rows_g = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+      const int r = m * BM + row;
+      // rows past the group's end belong to the next group (or are padding);
+      // the second test keeps a corrupted offsets[] from writing out of range
+      const bool valid = r < rows_g && (g == args.N || args.offsets[g] + r < args.rows_routed);
+      __nv_bfloat16* orow =
+          (g < args.N) ? args.out_routed + (size_t)(args.offsets[g] + r) * args.out_ld
+                       : args.out_shared + (size_t)r * args.out_ld;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if constexpr (kEpi == kEpiSwiGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t ga[32], up[32];
+          tmem_ld32(taddr + c, ga);
+          tmem_ld32(taddr + BN / 2 + c, up);
+          tmem_wait_ld();
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            h[i] = silu_f(__uint_as_float(ga[i])) * __uint_as_float(up[i]);
+          if (valid) store_row32(orow + n * (BN / 2) + c, h);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
+          if (valid) store_row32(orow + n * BN + c, y);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  // ---- teardown ------------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---- host side -----------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, inner] with a (box_inner x box_rows) box and
+// the 128-byte swizzle; out-of-range rows read as zero.
+bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t elem_bytes,
+              uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int kEpi>
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
+  const size_t smem = smem_bytes_for(a.N + 1);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_bf16_kernel<kEpi><<<num_sms(), kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                       const void* x, const void* w13, const void* w2, void* y_perm,
+                       void* y_shared, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(w + L.h);
+  const uint64_t TK = (uint64_t)s.T * s.K;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+
+  GemmArgs g1{};
+  bool ok = make_map(&g1.tmA_routed, x_perm, BF, 2, s.d, TK, BK, BM) &&
+            make_map(&g1.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, BN);
+  if (!ok) return MOE_ERR_CUDA;
+  g1.offsets = offsets;
+  g1.out_routed = H;
+  g1.out_shared = H + TK * s.f;
+  g1.status = reinterpret_cast<uint32_t*>(w + L.status);
+  g1.N = s.N;
+  g1.T = s.T;
+  g1.rows_routed = (int)TK;
+  g1.a_shared_row0 = 0;
+  g1.n_acc = 2 * s.f;
+  g1.k_dim = s.d;
+  g1.out_ld = s.f;
+  if (launch_gemm<kEpiSwiGLU>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  GemmArgs g2{};
+  ok = make_map(&g2.tmA_routed, H, BF, 2, s.f, TK + s.T, BK, BM) &&
+       make_map(&g2.tmA_shared, H, BF, 2, s.f, TK + s.T, BK, BM) &&
+       make_map(&g2.tmB, w2, BF, 2, s.f, (uint64_t)(s.N + 1) * s.d, BK, BN);
+  if (!ok) return MOE_ERR_CUDA;
+  g2.offsets = offsets;
+  g2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
+  g2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
+  g2.status = g1.status;
+  g2.N = s.N;
+  g2.T = s.T;
+  g2.rows_routed = (int)TK;
+  g2.a_shared_row0 = (int)TK;
+  g2.n_acc = s.d;
+  g2.k_dim = s.f;
+  g2.out_ld = s.d;
+  if (launch_gemm<kEpiStore>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,68 @@
+// Internal declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+constexpr int kRouteTokens = 32;   // tokens per routing CTA (4 per warp)
+constexpr int kRouteMaxN = 256;    // experts a routing warp holds (8 per lane)
+constexpr int kChunkTokens = 32;   // tokens per dispatch chunk
+constexpr int kMaxK = 32;
+
+inline int chunks_of(int T) { return (T + kChunkTokens - 1) / kChunkTokens; }
+
+// Byte offsets of the workspace regions (each 256-byte aligned).
+struct WsLayout {
+  size_t status = 0;      // uint32 device status word (+ padding to 256)
+  size_t chunk_hist = 0;  // int32 [chunks, N]
+  size_t chunk_base = 0;  // int32 [chunks, N]
+  size_t h = 0;           // hidden activation [T*K + T, f] (bf16 / fp32 / e4m3)
+  size_t h_scales = 0;    // fp32 [T*K + T, f/128] (E4M3)
+  size_t xq = 0;          // E4M3 codes of x for the shared expert [T, d]
+  size_t xq_scales = 0;   // fp32 [T, d/128]
+  size_t total = 0;
+};
+WsLayout ws_layout(const moe_shape& s);
+
+inline size_t dtype_bytes(int dtype) {
+  return dtype == MOE_DTYPE_FP32 ? 4 : (dtype == MOE_DTYPE_BF16 ? 2 : 1);
+}
+// Bytes per element of the layer input x and output y.
+inline size_t io_bytes(int dtype) { return dtype == MOE_DTYPE_FP32 ? 4 : 2; }
+// Rows of a W1/W3 block in the packed w13 layout.
+inline int pack_block(int f) { return f < 128 ? f : 128; }
+
+// ---- launchers (return cudaError_t of the launch) -----------------------------
+cudaError_t launch_route(const moe_shape& s, const void* x, const float* router,
+                         const float* bias, int32_t* idx, float* gate, int32_t* counts,
+                         uint32_t* status, cudaStream_t st);
+cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* idx,
+                            const int32_t* counts, int32_t* offsets, int32_t* perm_tok,
+                            int32_t* slot, void* x_perm, float* x_perm_scales, void* ws,
+                            cudaStream_t st);
+cudaError_t launch_combine(const moe_shape& s, const void* y_perm, const void* y_shared,
+                           const int32_t* slot, const float* gate, void* y, cudaStream_t st);
+cudaError_t launch_bias_update(const moe_shape& s, const int32_t* counts, float* bias,
+                               float gamma, cudaStream_t st);
+cudaError_t launch_pack_w13(const moe_shape& s, const void* w1, const void* w3, void* w13,
+                            cudaStream_t st);
+cudaError_t launch_ffn_simt(const moe_shape& s, const float* x_perm, const int32_t* offsets,
+                            const float* x, const float* w13, const float* w2, float* y_perm,
+                            float* y_shared, void* ws, cudaStream_t st);
+// Returns MOE_OK or a MOE_ERR_* status (tensor maps can fail to encode).
+int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                       const void* x, const void* w13, const void* w2, void* y_perm,
+                       void* y_shared, void* ws, cudaStream_t st);
+int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_perm_scales,
+                       const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                       const float* w13_scales, const float* w2_scales, void* y_perm,
+                       void* y_shared, void* ws, cudaStream_t st);
+cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const void* w2,
+                                    void* w13_q, float* w13_scales, void* w2_q,
+                                    float* w2_scales, cudaStream_t st);
+
+}  // namespace moe

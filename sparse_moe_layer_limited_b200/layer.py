@@ -1,0 +1,67 @@
+"""MoELayer: owns the device buffers of one layer shape and runs the forward
+through the C-ABI calls (route -> dispatch -> experts -> combine -> bias update)."""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+class MoELayer:
+    """DeepSeekMoE layer on one GPU.
+
+    router_w [N, d] fp32, bias [N] fp32 (updated in place by forward), w13
+    [N+1, 2f, d] packed (see moe_pack_w13), w2 [N+1, d, f]; for E4M3 the
+    quantised weights and their 128x128-block scales.  All tensors must be on
+    the same CUDA device.  Intermediate buffers are allocated once here."""
+
+    def __init__(self, shape: L.MoEShape, router_w, bias, w13, w2, w13_scales=None,
+                 w2_scales=None, gamma: float = 0.001):
+        rc = L.check_shape(shape)
+        if rc != L.OK:
+            raise L.MoEError("moe_check_shape", rc)
+        self.shape = s = shape
+        self.router_w, self.bias, self.w13, self.w2 = router_w, bias, w13, w2
+        self.w13_scales, self.w2_scales = w13_scales, w2_scales
+        self.gamma = float(gamma)
+        dev = router_w.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        xdt = L.x_torch_dtype(s)
+        self.topk_idx = torch.empty(s.T, s.K, **i32)
+        self.topk_gate = torch.empty(s.T, s.K, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(s.N, **i32)
+        self.offsets = torch.empty(s.N + 1, **i32)
+        self.perm_tok = torch.empty(s.T * s.K, **i32)
+        self.slot = torch.empty(s.T, s.K, **i32)
+        pdt = torch.float8_e4m3fn if s.dtype == L.DTYPE_E4M3 else xdt
+        self.x_perm = torch.empty(s.T * s.K, s.d, dtype=pdt, device=dev)
+        self.x_perm_scales = (torch.empty(s.T * s.K, s.d // 128, dtype=torch.float32, device=dev)
+                              if s.dtype == L.DTYPE_E4M3 else None)
+        self.y_perm = torch.empty(s.T * s.K, s.d, dtype=xdt, device=dev)
+        self.y_shared = torch.empty(s.T, s.d, dtype=xdt, device=dev)
+        self.y = torch.empty(s.T, s.d, dtype=xdt, device=dev)
+        self.ws = torch.zeros(L.workspace_size(s), dtype=torch.uint8, device=dev)
+
+    def route(self, x, stream=None):
+        s = self.shape
+        L.moe_route(s, x, self.router_w, self.bias, self.topk_idx, self.topk_gate, self.counts,
+                    self.ws, stream)
+
+    def forward(self, x, update_bias: bool = True, stream=None):
+        """y = shared(x) + sum_k gate_k expert_k(x); then (optionally) the bias
+        update from this batch's counts.  Returns self.y (overwritten next call)."""
+        s = self.shape
+        L.moe_route(s, x, self.router_w, self.bias, self.topk_idx, self.topk_gate, self.counts,
+                    self.ws, stream)
+        L.moe_dispatch(s, x, self.topk_idx, self.counts, self.offsets, self.perm_tok, self.slot,
+                       self.x_perm, self.x_perm_scales, self.ws, stream)
+        L.moe_expert_ffn(s, self.x_perm, self.x_perm_scales, self.offsets, x, self.w13, self.w2,
+                         self.w13_scales, self.w2_scales, self.y_perm, self.y_shared, self.ws,
+                         stream)
+        L.moe_combine(s, self.y_perm, self.y_shared, self.slot, self.topk_gate, self.y, stream)
+        if update_bias:
+            L.moe_bias_update(s, self.counts, self.bias, self.gamma, stream)
+        return self.y
+
+    def device_status(self, clear: bool = False) -> int:
+        return L.moe_read_device_status(self.ws, None, clear)

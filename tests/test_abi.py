@@ -1,0 +1,94 @@
+"""The C ABI without a GPU: the library loads, exports every declared
+symbol, and rejects bad shapes and pointers before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_moe_layer_limited_b200 import build
+    if not os.path.exists(build.LIB_PATH):
+        build.build()
+    from sparse_moe_layer_limited_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_bias_update",
+              "moe_workspace_size", "moe_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    raw = ctypes.CDLL(L.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+    assert set(declared_functions()) <= set(L._SIGS), "binding misses a declared entry point"
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5, 7):
+        assert isinstance(L.status_string(code), str) and L.status_string(code)
+
+
+def test_shape_checks(L):
+    from synth import CONFIGS
+    from tests.support import moe_shape
+    for cfg in CONFIGS.values():
+        s = moe_shape(cfg)
+        if cfg.dtype == "e4m3":
+            continue
+        assert L.check_shape(s) == L.OK, cfg.name
+        assert L.workspace_size(s) > 0
+    ok = L.shape(128, 64, 16, 4, 1, 1, 32, L.DTYPE_FP32)
+    assert L.check_shape(ok) == L.OK
+    bad = [
+        (L.shape(0, 64, 16, 4, 1, 1, 32, 0), L.ERR_ARG),        # T = 0
+        (L.shape(128, 64, 16, 4, 3, 1, 32, 0), L.ERR_UNSUPPORTED),  # G does not divide N
+        (L.shape(128, 64, 16, 4, 4, 5, 32, 0), L.ERR_UNSUPPORTED),  # topG > G
+        (L.shape(128, 64, 16, 17, 1, 1, 32, 0), L.ERR_UNSUPPORTED),  # K > N
+        (L.shape(128, 64, 16, 5, 4, 1, 32, 0), L.ERR_UNSUPPORTED),  # K > topG * N/G
+        (L.shape(128, 64, 512, 4, 1, 1, 32, 0), L.ERR_UNSUPPORTED),  # N > 256
+        (L.shape(128, 100, 16, 4, 1, 1, 32, 0), L.ERR_UNSUPPORTED),  # d % 32
+        (L.shape(128, 128, 16, 4, 1, 1, 256, 1), L.ERR_UNSUPPORTED),  # bf16 needs d % 256
+        (L.shape(128, 256, 16, 4, 1, 1, 200, 1), L.ERR_UNSUPPORTED),  # bf16 needs f % 128
+        (L.shape(128, 256, 16, 4, 1, 1, 256, 9), L.ERR_UNSUPPORTED),  # dtype
+    ]
+    for s, want in bad:
+        assert L.check_shape(s) == want, s
+        assert L.workspace_size(s) == 0
+
+
+def test_null_pointers_rejected_before_any_launch(L):
+    s = L.shape(128, 64, 16, 4, 1, 1, 32, L.DTYPE_FP32)
+    f = L.lib()
+    p = ctypes.byref(s)
+    assert f.moe_route(p, None, None, None, None, None, None, None, None) == L.ERR_ARG
+    assert f.moe_dispatch(p, *([None] * 10)) == L.ERR_ARG
+    assert f.moe_expert_ffn(p, *([None] * 12)) == L.ERR_ARG
+    assert f.moe_combine(p, *([None] * 6)) == L.ERR_ARG
+    assert f.moe_bias_update(p, None, None, ctypes.c_float(0.001), None) == L.ERR_ARG
+    assert f.moe_route(None, *([None] * 8)) == L.ERR_ARG
+    # misaligned (not 16-byte aligned) pointers are rejected too
+    mis = ctypes.c_void_p(0x1001)
+    assert f.moe_combine(p, mis, mis, mis, mis, mis, None) == L.ERR_ARG
+
+
+def test_workspace_layout_grows_with_shape(L):
+    a = L.workspace_size(L.shape(1024, 256, 8, 2, 2, 1, 256, L.DTYPE_BF16))
+    b = L.workspace_size(L.shape(2048, 256, 8, 2, 2, 1, 256, L.DTYPE_BF16))
+    assert 0 < a < b
+    assert a % 256 == 0

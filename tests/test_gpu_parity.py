@@ -1,0 +1,178 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Routing indices, counts, offsets, the permutation and slots must match bit
+for bit; gates within 1e-6; layer outputs within rel-Frobenius 1e-5 (fp32
+layer) and 1e-2 (bf16 layer, oracle on bf16-rounded operands with the hidden
+activation rounded to bf16).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from synth import CONFIGS, gen
+from tests import support as S
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-5, "bf16": 1e-2, "e4m3": 2e-2}
+
+
+@pytest.fixture(scope="module")
+def M():
+    import sparse_moe_layer_limited_b200 as M
+    return M
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _run_route(M, cfg, x, R, b, T=None):
+    torch = _torch()
+    s = S.moe_shape(cfg, T)
+    xd = S.to_dev_x(x, cfg)
+    Rd = torch.from_numpy(R).cuda()
+    bd = torch.from_numpy(np.asarray(b, np.float32)).cuda()
+    idx = torch.empty(s.T, s.K, dtype=torch.int32, device="cuda")
+    gate = torch.empty(s.T, s.K, dtype=torch.float32, device="cuda")
+    counts = torch.empty(s.N, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(M.workspace_size(s), dtype=torch.uint8, device="cuda")
+    M.moe_route(s, xd, Rd, bd, idx, gate, counts, ws)
+    assert M.moe_read_device_status(ws) == 0
+    return idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy()
+
+
+def _check_route(cfg, r, idx, gate, counts):
+    np.testing.assert_array_equal(idx, r["idx"])
+    np.testing.assert_array_equal(counts, r["counts"])
+    np.testing.assert_allclose(gate, r["gate"], rtol=0, atol=1e-6)
+
+
+def test_device_generator_matches_host():
+    torch = _torch()
+    from synth import device as sdev
+    cfg = CONFIGS[1]
+    w = sdev.expert_weights_bf16(cfg, 0, "w2")
+    for e in (0, 17, cfg.N):
+        host = gen.make_expert_weight(cfg, 0, "w2", e)
+        dev = w[e].float().cpu().numpy()
+        np.testing.assert_array_equal(dev, host)
+
+
+@pytest.mark.parametrize("cfg_id", [0, 1])
+def test_route_bitexact(M, cfg_id):
+    cfg = CONFIGS[cfg_id]
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
+    _check_route(cfg, r, *_run_route(M, cfg, x, R, b))
+
+
+def test_route_ragged_and_hot_expert(M):
+    """T not a multiple of the 32-token tile; a +10 bias forces one expert."""
+    cfg = CONFIGS[1].with_(T=1000)
+    R = gen.make_router(cfg)
+    b = gen.make_bias(cfg).copy()
+    b[13] = 10.0
+    x, _ = S.tie_free_x(cfg, R, b)
+    r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
+    assert r["counts"][13] == cfg.T
+    _check_route(cfg, r, *_run_route(M, cfg, x, R, b))
+
+
+def _layer(M, cfg, x, R, b, W):
+    torch = _torch()
+    s = S.moe_shape(cfg)
+    layer = M.MoELayer(s, torch.from_numpy(R).cuda(),
+                       torch.from_numpy(np.asarray(b, np.float32)).cuda(), W["w13"], W["w2"],
+                       W["w13_scales"], W["w2_scales"], gamma=cfg.gamma)
+    xd = S.to_dev_x(x, cfg)
+    return layer, xd
+
+
+def _check_dispatch(layer, r):
+    d = oracle.dispatch(r["idx"], layer.shape.N)
+    np.testing.assert_array_equal(layer.offsets.cpu().numpy(), d["offsets"])
+    np.testing.assert_array_equal(layer.perm_tok.cpu().numpy(), d["perm_tok"])
+    np.testing.assert_array_equal(layer.slot.cpu().numpy(), d["slot"])
+    return d
+
+
+def test_tiny_fp32_layer_full(M):
+    """The tiny fp32 layer end to end, every output element."""
+    cfg = CONFIGS[0]
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K)
+    r = ref["route"]
+    _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
+                 layer.counts.cpu().numpy())
+    _check_dispatch(layer, r)
+    err = S.rel_fro(y, ref["y"])
+    assert err <= TOL["fp32"], err
+    nb = oracle.bias_update(b, r["counts"], cfg.T, cfg.K, cfg.gamma)
+    np.testing.assert_array_equal(layer.bias.cpu().numpy(), nb)
+    assert layer.device_status() == 0
+
+
+def _small_bf16(T=1000):
+    # several m-tiles per expert with a ragged tail, 2 n-tiles in GEMM1
+    return CONFIGS[1].with_(T=T, d=256, N=8, K=2, G=2, topG=1, f=256)
+
+
+@pytest.mark.parametrize("T", [1000, 129, 1])
+def test_small_bf16_layer_full(M, T):
+    cfg = _small_bf16(T)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).float().cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             h_round="bf16")
+    r = ref["route"]
+    _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
+                 layer.counts.cpu().numpy())
+    d = _check_dispatch(layer, r)
+    # per-expert rows of the grouped GEMM output
+    get = S.host_weights(cfg)
+    yp = layer.y_perm.float().cpu().numpy()
+    for e in range(cfg.N):
+        a, z = d["offsets"][e], d["offsets"][e + 1]
+        if z == a:
+            continue
+        want = oracle.swiglu_expert(x[d["perm_tok"][a:z]], *get(e), h_round="bf16")
+        assert S.rel_fro(yp[a:z], want) <= TOL["bf16"], e
+    ysh = layer.y_shared.float().cpu().numpy()
+    assert S.rel_fro(ysh, oracle.swiglu_expert(x, *get(cfg.N), h_round="bf16")) <= TOL["bf16"]
+    err = S.rel_fro(y, ref["y"])
+    assert err <= TOL["bf16"], err
+    assert layer.device_status() == 0
+
+
+def test_mid_bf16_layer_sampled(M):
+    """The mid-size bf16 layer: full routing/dispatch, outputs on 256 tokens."""
+    torch = _torch()
+    cfg = CONFIGS[1]
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).float().cpu().numpy()
+    r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
+    _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
+                 layer.counts.cpu().numpy())
+    d = _check_dispatch(layer, r)
+    # tokens that sit in the last (ragged) m-tile of their expert are included
+    tail = [int(d["perm_tok"][d["offsets"][e + 1] - 1]) for e in range(0, cfg.N, 8)]
+    tokens = np.unique(np.concatenate([np.random.default_rng(0).choice(cfg.T, 256, False), tail]))
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             tokens=tokens, h_round="bf16")
+    err = S.rel_fro(y[tokens], ref["y"])
+    assert err <= TOL["bf16"], err
+    assert layer.device_status() == 0
+    del torch
