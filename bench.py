@@ -36,12 +36,14 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--cpu-sample", type=int, default=4, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
+    p.add_argument("--N", type=int, default=None, help="override routed experts (profiling)")
     return p.parse_args()
 
 
@@ -97,6 +99,7 @@ class ClockSampler:
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)  # let nvidia-smi start sampling before the timed region
         except Exception:
             self.proc = None
         return self
@@ -207,6 +210,10 @@ def run_reference(args, cfg):
 def main():
     args = parse()
     cfg = BY_NAME[args.config]
+    if args.T:
+        cfg = cfg.with_(T=args.T)
+    if args.N:
+        cfg = cfg.with_(N=args.N)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -318,7 +325,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
             "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
-                       "l2": "inputs larger than L2: the 22.6 GB of expert weights stream "
+                       "l2": "inputs larger than L2: the expert weights "
+                             f"({(cfg.N + 1) * 3 * cfg.d * cfg.f * 2 / 1e9:.1f} GB) stream "
                              "through it every step",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, "
