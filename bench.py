@@ -40,7 +40,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="v3_bf16")
-    p.add_argument("--cpu-sample", type=int, default=4, help="tokens per oracle sample")
+    p.add_argument("--cpu-sample", type=int, default=2, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
     p.add_argument("--N", type=int, default=None, help="override routed experts (profiling)")
@@ -135,33 +135,33 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def cpu_oracle_baseline(cfg, n_tokens, seed=0, rounds=1):
+def cpu_oracle_baseline(cfg, n_tokens, seed=0, batch=1000):
     """The float64 oracle as it stands on this host's cores: routing plus the
-    expert and combine work of `n_tokens` sampled tokens per round (weight
-    generation is excluded from the time).  Returns (tokens/s, cores, note)."""
+    expert and combine work of `n_tokens` tokens of a fresh batch.  Weight
+    generation (into reused buffers) is excluded from the time.
+    Returns (tokens/s, cores, note)."""
     import oracle
     R, b = gen.make_router(cfg), gen.make_bias(cfg)
     cores = len(os.sched_getaffinity(0))
-    total_t, total_tok = 0.0, 0
-    for r in range(rounds):
-        x = gen.make_x(cfg, seed, batch=1000 + r)[:max(n_tokens, 1)]
-        gen_time = [0.0]
+    x = gen.make_x(cfg, seed, batch=batch)[:max(n_tokens, 1)]
+    bufs = {w: np.empty(gen.weight_shape(cfg, w), np.float64) for w in ("w1", "w3", "w2")}
+    gen_time = [0.0]
 
-        def get(e):
-            t0 = time.perf_counter()
-            w = tuple(gen.make_expert_weight(cfg, seed, w, e).astype(np.float64)
-                      for w in ("w1", "w3", "w2"))
-            gen_time[0] += time.perf_counter() - t0
-            return w
-
+    def get(e):
         t0 = time.perf_counter()
-        oracle.moe_forward(x, R, b, get, cfg.G, cfg.topG, cfg.K,
-                           h_round="none" if cfg.dtype == "fp32" else "bf16")
-        total_t += time.perf_counter() - t0 - gen_time[0]
-        total_tok += x.shape[0]
-    note = (f"{total_tok} tokens of the {cfg.name} workload (full routing and expert math per "
-            f"token, weight generation excluded), numpy float64 on {cores} cores")
-    return total_tok / total_t, cores, note
+        out = tuple(gen.make_expert_weight(cfg, seed, w, e, out=bufs[w])
+                    for w in ("w1", "w3", "w2"))
+        gen_time[0] += time.perf_counter() - t0
+        return out
+
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, R, b, get, cfg.G, cfg.topG, cfg.K,
+                       h_round="none" if cfg.dtype == "fp32" else "bf16")
+    dt = time.perf_counter() - t0 - gen_time[0]
+    note = (f"{x.shape[0]} token(s) of the {cfg.name} workload per sample (full routing, the "
+            f"K+1 expert FFNs and the combine; weight generation excluded), numpy float64 "
+            f"on {cores} cores")
+    return x.shape[0] / dt, cores, note
 
 
 def dist_setup(args):
@@ -185,12 +185,12 @@ def run_reference(args, cfg):
         return
     times = []
     n = max(1, args.cpu_sample)
-    for _ in range(args.warmup):
-        cpu_oracle_baseline(cfg, 1)
+    for w in range(args.warmup):
+        cpu_oracle_baseline(cfg, 1, batch=2000 + w)
     cores = len(os.sched_getaffinity(0))
     note = ""
-    for _ in range(args.steps):
-        v, cores, note = cpu_oracle_baseline(cfg, n)
+    for k in range(args.steps):
+        v, cores, note = cpu_oracle_baseline(cfg, n, batch=3000 + k)
         times.append(n / v)
     value = n * len(times) / sum(times)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",

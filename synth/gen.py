@@ -298,8 +298,23 @@ def weight_dtype(cfg: MoEConfig) -> str:
     return "fp32" if cfg.dtype == "fp32" else "bf16"
 
 
-def make_expert_weight(cfg: MoEConfig, seed: int, which: str, expert: int) -> np.ndarray:
+def make_expert_weight(cfg: MoEConfig, seed: int, which: str, expert: int,
+                       out: np.ndarray | None = None) -> np.ndarray:
     """W1[e], W3[e] ([f, d]) or W2[e] ([d, f]) of expert e (e == N is the
-    shared expert); entries ~ N(0, 1/fan_in), float32 array of stored values."""
-    return normal(weight_key(cfg, seed, which, expert), weight_shape(cfg, which),
-                  weight_sigma(cfg, which), weight_dtype(cfg))
+    shared expert); entries ~ N(0, 1/fan_in), as a float32 array of stored
+    values, or written into ``out`` (float32 or float64, right shape)."""
+    key = weight_key(cfg, seed, which, expert)
+    shape = weight_shape(cfg, which)
+    table = normal_table(weight_sigma(cfg, which), weight_dtype(cfg))
+    if out is None:
+        return normal(key, shape, weight_sigma(cfg, which), weight_dtype(cfg))
+    assert out.shape == shape and out.flags.c_contiguous
+    lib = _host_lib()
+    flat = out.reshape(-1)
+    if lib is not None and out.dtype in (np.float32, np.float64):
+        t = np.ascontiguousarray(table, dtype=out.dtype)
+        fn = lib.synth_host_fill_f32 if out.dtype == np.float32 else lib.synth_host_fill_f64
+        fn(flat.ctypes.data, key, 0, flat.size, t.ctypes.data)
+    else:
+        flat[:] = _table_draw_numpy(key, flat.size, table)
+    return out
