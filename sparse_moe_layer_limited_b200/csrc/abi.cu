@@ -17,6 +17,12 @@ WsLayout ws_layout(const moe_shape& s) {
   off = align256(off + nch * s.N * 4);
   L.chunk_base = off;
   off = align256(off + nch * s.N * 4);
+  if (s.dtype != MOE_DTYPE_FP32) {
+    L.router_split = off;
+    off = align256(off + (size_t)s.N * 3 * s.d * 2);
+    L.scores = off;
+    off = align256(off + (size_t)s.T * s.N * 4);
+  }
   const size_t rows = (size_t)s.T * s.K + s.T;
   L.h = off;
   off = align256(off + rows * s.f * dtype_bytes(s.dtype));
@@ -68,7 +74,6 @@ int ws_check(const moe_shape* s, void* ws) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-uint32_t* status_word(void* ws) { return static_cast<uint32_t*>(ws); }
 
 }  // namespace
 
@@ -122,8 +127,8 @@ int moe_route(const moe_shape* shape, const void* x, const float* router_w, cons
       !ptr_ok(topk_gate) || !ptr_ok(counts))
     return MOE_ERR_ARG;
   if ((rc = ws_check(shape, ws))) return rc;
-  return cuda_status(launch_route(*shape, x, router_w, bias, topk_idx, topk_gate, counts,
-                                  status_word(ws), static_cast<cudaStream_t>(stream)));
+  return launch_route(*shape, x, router_w, bias, topk_idx, topk_gate, counts, ws,
+                      static_cast<cudaStream_t>(stream));
 }
 
 int moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx,

@@ -1,4 +1,5 @@
-// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores (bf16).
+// Grouped bf16 GEMMs on the 5th-generation tensor cores: the SwiGLU expert
+// GEMMs and the router score GEMM.
 //
 // The experts are FFNs (mhpq.cn article §1.1; wenxiaobai §二(一)4) in the
 // SwiGLU form y = (silu(a W1^T) * (a W3^T)) W2^T; the routed experts run on
@@ -27,6 +28,15 @@
 // W3 rows, so one accumulator tile holds matching gate and up columns.
 // Every mbarrier wait is bounded (~2 s); a wait that gives up sets the
 // device status word and the CTA unwinds, frees its TMEM and returns.
+//
+// The same kernel computes the router scores z = x . e_i (one group of T
+// rows, tile width N): the fp32 router matrix is split exactly into three
+// bf16 parts R = R0 + R1 + R2 (R0 = bf16(R), R1 = bf16(R - R0), R2 =
+// bf16(R - R0 - R1), residual below 2^-27 |R|), stored as one [N, 3d]
+// operand whose 64-column blocks run (R0, R1, R2) per 64 columns of d; each
+// A tile of x is used for three consecutive K blocks (a_rep = 3), so the
+// fp32 accumulator receives x.R0 + x.R1 + x.R2 = x.R.  The sigmoid epilogue
+// writes s = sigmoid(z) as fp32 for the selection kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -39,16 +49,23 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64;  // BK bf16 = 128 bytes = one swizzle row
+constexpr int BM = 128, BK = 64;  // BK bf16 = 128 bytes = one swizzle row
 constexpr int kStages = 4;
 constexpr int kABytes = BM * BK * 2;
-constexpr int kBBytes = BN * BK * 2;
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum Epi { kEpiSwiGLU = 0, kEpiStore = 1 };
+enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiSigmoid = 2 };
+
+template <int kBN>
+struct TileCfg {
+  static constexpr int kBBytes = kBN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * kBN;  // two accumulators
+  static constexpr size_t smem_bytes(int groups) {
+    return 1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(groups + 1) * 4;
+  }
+};
 
 struct alignas(64) GemmArgs {
   CUtensorMap tmA_routed;
@@ -57,6 +74,7 @@ struct alignas(64) GemmArgs {
   const int32_t* offsets;
   __nv_bfloat16* out_routed;
   __nv_bfloat16* out_shared;
+  float* out_f32;   // sigmoid epilogue: [T, n_valid]
   uint32_t* status;
   int N, T;
   int rows_routed;  // T*K
@@ -64,11 +82,9 @@ struct alignas(64) GemmArgs {
   int n_acc;   // accumulator columns per expert (2f for GEMM1, d for GEMM2)
   int k_dim;   // contraction length
   int out_ld;  // output row stride in elements
+  int a_rep;   // K blocks that reuse one A tile (3 for the split router, else 1)
+  int n_valid; // columns to store (sigmoid epilogue)
 };
-
-__host__ __device__ constexpr size_t smem_bytes_for(int groups) {
-  return 1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(groups + 1) * 4;
-}
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
@@ -82,9 +98,15 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) 
   for (int i = 0; i < 4; ++i) d4[i] = w[i];
 }
 
-template <int kEpi>
+template <int kEpi, int kBN>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     const __grid_constant__ GemmArgs args) {
+  constexpr int BN = kBN;
+  constexpr int kBBytes = TileCfg<kBN>::kBBytes;
+  constexpr int kStageBytes = TileCfg<kBN>::kStageBytes;
+  constexpr int kTmemCols = TileCfg<kBN>::kTmemCols;
+  static_assert(kEpi != kEpiSwiGLU || kBN == 256, "SwiGLU tiles pair 128 gate + 128 up columns");
+  (void)kBBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -186,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           }
           uint8_t* sa = base + (size_t)stage * kStageBytes;
           mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          tma_load_2d(sa, am, kb * BK, arow, &full[stage]);
+          tma_load_2d(sa, am, (kb / args.a_rep) * BK, arow, &full[stage]);
           tma_load_2d(sa + kABytes, &args.tmB, kb * BK, brow, &full[stage]);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -205,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   } else if (warp == 1) {
     // ---- MMA issuer -----------------------------------------------------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN);
+      const uint32_t idesc = idesc_bf16_f32(BM, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -273,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
             h[i] = silu_f(__uint_as_float(ga[i])) * __uint_as_float(up[i]);
           if (valid) store_row32(orow + n * (BN / 2) + c, h);
         }
-      } else {
+      } else if constexpr (kEpi == kEpiStore) {
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
@@ -283,6 +305,29 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
           if (valid) store_row32(orow + n * BN + c, y);
+        }
+      } else {  // sigmoid scores, fp32, columns < n_valid
+        float* srow = args.out_f32 + (size_t)r * args.n_valid;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (valid && c < args.n_valid) {
+            float sg[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sg[i] = 1.f / (1.f + expf(-__uint_as_float(v[i])));
+            if (c + 32 <= args.n_valid) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(srow + c + i) =
+                    make_float4(sg[i], sg[i + 1], sg[i + 2], sg[i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c + i < args.n_valid) srow[c + i] = sg[i];
+            }
+          }
         }
       }
       tc_fence_before();
@@ -342,14 +387,37 @@ int num_sms() {
   return n;
 }
 
-template <int kEpi>
+template <int kEpi, int kBN>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
-  const size_t smem = smem_bytes_for(a.N + 1);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi>,
+  const size_t smem = TileCfg<kBN>::smem_bytes(a.N + 1);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_bf16_kernel<kEpi><<<num_sms(), kThreads, smem, st>>>(a);
+  grouped_gemm_bf16_kernel<kEpi, kBN><<<num_sms(), kThreads, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+// R fp32 [N, d] -> three exact bf16 parts laid out [N, 3d] as described at
+// the top of this file.
+__global__ void router_split_kernel(const float* __restrict__ R, int N, int d,
+                                    __nv_bfloat16* __restrict__ Rs) {
+  const long long total = (long long)N * d;
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < total;
+       q += (long long)gridDim.x * blockDim.x) {
+    const long long n = q / d;
+    const int c = (int)(q - n * d);
+    const float v = R[q];
+    const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
+    const float r1 = __fsub_rn(v, __bfloat162float(p0));
+    const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+    const float r2 = __fsub_rn(r1, __bfloat162float(p1));
+    const __nv_bfloat16 p2 = __float2bfloat16_rn(r2);
+    const int cb = c / BK, i = c % BK;
+    __nv_bfloat16* row = Rs + n * 3LL * d + (long long)(3 * cb) * BK + i;
+    row[0] = p0;
+    row[BK] = p1;
+    row[2 * BK] = p2;
+  }
 }
 
 }  // namespace
@@ -366,7 +434,7 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   GemmArgs g1{};
   bool ok = make_map(&g1.tmA_routed, x_perm, BF, 2, s.d, TK, BK, BM) &&
             make_map(&g1.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
-            make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, BN);
+            make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, 256);
   if (!ok) return MOE_ERR_CUDA;
   g1.offsets = offsets;
   g1.out_routed = H;
@@ -379,12 +447,13 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g1.n_acc = 2 * s.f;
   g1.k_dim = s.d;
   g1.out_ld = s.f;
-  if (launch_gemm<kEpiSwiGLU>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+  g1.a_rep = 1;
+  if (launch_gemm<kEpiSwiGLU, 256>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   GemmArgs g2{};
   ok = make_map(&g2.tmA_routed, H, BF, 2, s.f, TK + s.T, BK, BM) &&
        make_map(&g2.tmA_shared, H, BF, 2, s.f, TK + s.T, BK, BM) &&
-       make_map(&g2.tmB, w2, BF, 2, s.f, (uint64_t)(s.N + 1) * s.d, BK, BN);
+       make_map(&g2.tmB, w2, BF, 2, s.f, (uint64_t)(s.N + 1) * s.d, BK, 256);
   if (!ok) return MOE_ERR_CUDA;
   g2.offsets = offsets;
   g2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
@@ -397,8 +466,45 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g2.n_acc = s.d;
   g2.k_dim = s.f;
   g2.out_ld = s.d;
-  if (launch_gemm<kEpiStore>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+  g2.a_rep = 1;
+  if (launch_gemm<kEpiStore, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* S,
+                            void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(w + L.router_split);
+  const long long total = (long long)s.N * s.d;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  router_split_kernel<<<(int)blocks, 256, 0, st>>>(router, s.N, s.d, Rs);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+  const int bn = s.N <= 64 ? 64 : (s.N <= 128 ? 128 : 256);
+  GemmArgs a{};
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = make_map(&a.tmA_routed, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&a.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&a.tmB, Rs, BF, 2, 3ull * s.d, s.N, BK, bn);
+  if (!ok) return MOE_ERR_CUDA;
+  a.offsets = nullptr;
+  a.out_f32 = S;
+  a.status = reinterpret_cast<uint32_t*>(w + L.status);
+  a.N = 0;  // a single group: all T rows of x
+  a.T = s.T;
+  a.rows_routed = 0;
+  a.a_shared_row0 = 0;
+  a.n_acc = bn;
+  a.k_dim = 3 * s.d;
+  a.out_ld = s.N;
+  a.a_rep = 3;
+  a.n_valid = s.N;
+  cudaError_t e = bn == 64    ? launch_gemm<kEpiSigmoid, 64>(a, st)
+                  : bn == 128 ? launch_gemm<kEpiSigmoid, 128>(a, st)
+                              : launch_gemm<kEpiSigmoid, 256>(a, st);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

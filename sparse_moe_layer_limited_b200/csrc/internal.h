@@ -20,6 +20,8 @@ struct WsLayout {
   size_t status = 0;      // uint32 device status word (+ padding to 256)
   size_t chunk_hist = 0;  // int32 [chunks, N]
   size_t chunk_base = 0;  // int32 [chunks, N]
+  size_t router_split = 0;  // bf16 [N, 3d] exact three-part split of the router (bf16 x)
+  size_t scores = 0;        // fp32 [T, N] sigmoid affinities (bf16 x)
   size_t h = 0;           // hidden activation [T*K + T, f] (bf16 / fp32 / e4m3)
   size_t h_scales = 0;    // fp32 [T*K + T, f/128] (E4M3)
   size_t xq = 0;          // E4M3 codes of x for the shared expert [T, d]
@@ -37,9 +39,8 @@ inline size_t io_bytes(int dtype) { return dtype == MOE_DTYPE_FP32 ? 4 : 2; }
 inline int pack_block(int f) { return f < 128 ? f : 128; }
 
 // ---- launchers (return cudaError_t of the launch) -----------------------------
-cudaError_t launch_route(const moe_shape& s, const void* x, const float* router,
-                         const float* bias, int32_t* idx, float* gate, int32_t* counts,
-                         uint32_t* status, cudaStream_t st);
+int launch_route(const moe_shape& s, const void* x, const float* router, const float* bias,
+                 int32_t* idx, float* gate, int32_t* counts, void* ws, cudaStream_t st);
 cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* idx,
                             const int32_t* counts, int32_t* offsets, int32_t* perm_tok,
                             int32_t* slot, void* x_perm, float* x_perm_scales, void* ws,
@@ -53,6 +54,9 @@ cudaError_t launch_pack_w13(const moe_shape& s, const void* w1, const void* w3, 
 cudaError_t launch_ffn_simt(const moe_shape& s, const float* x_perm, const int32_t* offsets,
                             const float* x, const float* w13, const float* w2, float* y_perm,
                             float* y_shared, void* ws, cudaStream_t st);
+// Router scores on the tensor cores (bf16 x): S[t, i] = sigmoid(x_t . e_i).
+int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* S,
+                            void* ws, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* status (tensor maps can fail to encode).
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                        const void* x, const void* w13, const void* w2, void* y_perm,

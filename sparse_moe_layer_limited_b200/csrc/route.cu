@@ -7,8 +7,12 @@
 // (mhpq.cn article §3.1, "at most 4 nodes").  Group score = sum of the two
 // largest biased scores in the group (the reading this library takes).
 //
-// One CTA handles 32 tokens against all N (<= 256) experts.  Phase 1 is a
-// SIMT fp32 GEMM tile: x and the router are staged through shared memory in
+// bf16 inputs: the scores come from the tensor cores (an exact three-part
+// bf16 split of the fp32 router, see gemm_tc.cu) into a [T, N] fp32 buffer,
+// and select_kernel does the per-token selection below.
+//
+// fp32 inputs: one CTA handles 32 tokens against all N (<= 256) experts.
+// Phase 1 is a SIMT fp32 GEMM tile: x and the router are staged through shared memory in
 // 32-wide slices of d; warp w accumulates tokens 4w..4w+3 and lane l holds
 // experts l, l+32, ..., so after the K loop a warp owns every score of its
 // four tokens in registers.  Phase 2 (per token, inside the warp, no shared
@@ -29,7 +33,6 @@ constexpr int kKC = 32;            // d slice
 constexpr int kEPL = kRouteMaxN / 32;  // experts per lane
 
 __device__ __forceinline__ float load_f(const float* p) { return *p; }
-__device__ __forceinline__ float load_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 // (v, i) beats (w, j) if v > w, or v == w and i < j.
 __device__ __forceinline__ bool better(float v, int i, float w, int j) {
@@ -55,6 +58,98 @@ __device__ __forceinline__ void top2_merge(float& a1, float& a2, float b1, float
   }
 }
 
+// Selection for one token by one warp.  Lane l holds experts l + 32 j in
+// s[j] (un-biased sigmoid scores) and bj[j] (their biases).  Writes the K
+// chosen experts in ascending id order with their gates, and counts them in
+// the shared-memory histogram.
+__device__ __forceinline__ void select_token(const float (&s)[kEPL], const float (&bj)[kEPL],
+                                             int lane, int t, int N, int K, int G, int topG,
+                                             int32_t* __restrict__ topk_idx,
+                                             float* __restrict__ topk_gate, int* hist,
+                                             uint32_t* status) {
+  const int gs = N / G;
+  float sb[kEPL];
+#pragma unroll
+  for (int j = 0; j < kEPL; ++j) sb[j] = (lane + 32 * j < N) ? s[j] + bj[j] : -INFINITY;
+  // group scores: lane g ends up holding group g's score
+  float my_gscore = -INFINITY;
+  for (int g = 0; g < G; ++g) {
+    float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kEPL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < N && e / gs == g) top2_merge(m1, m2, sb[j], -INFINITY);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float b1 = __shfl_xor_sync(0xffffffffu, m1, o);
+      const float b2 = __shfl_xor_sync(0xffffffffu, m2, o);
+      top2_merge(m1, m2, b1, b2);
+    }
+    const float score = (gs >= 2) ? m1 + m2 : m1;
+    if (lane == g) my_gscore = score;
+  }
+  // keep the topG best groups
+  uint32_t kept = 0;
+  for (int r = 0; r < topG; ++r) {
+    float v = (lane < G && !((kept >> lane) & 1u)) ? my_gscore : -INFINITY;
+    int gi = (lane < G && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+    warp_argmax(v, gi);
+    kept |= 1u << (gi & 31);
+  }
+  // top-K among experts of kept groups
+  uint32_t taken = 0;  // bit j: this lane's expert lane+32j already chosen
+  int my_e = 0x7fffffff;
+  float my_s = 0.f;
+  for (int r = 0; r < K; ++r) {
+    float v = -INFINITY;
+    int ei = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < kEPL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < N && ((kept >> (e / gs)) & 1u) && !((taken >> j) & 1u) &&
+          better(sb[j], e, v, ei)) {
+        v = sb[j];
+        ei = e;
+      }
+    }
+    warp_argmax(v, ei);
+    // the owner marks it and broadcasts its un-biased score
+    float sv = 0.f;
+#pragma unroll
+    for (int j = 0; j < kEPL; ++j) {
+      if (lane + 32 * j == ei) {
+        taken |= 1u << j;
+        sv = s[j];
+      }
+    }
+    sv = __shfl_sync(0xffffffffu, sv, ei & 31);
+    if (lane == r) {
+      my_e = ei;
+      my_s = sv;
+    }
+  }
+  // ascending expert order and gates
+  int rank = 0;
+  for (int q = 0; q < K; ++q) {
+    const int eq = __shfl_sync(0xffffffffu, my_e, q);
+    rank += (eq < my_e) ? 1 : 0;
+  }
+  float sum = (lane < K) ? my_s : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < K) {
+    if (my_e < 0 || my_e >= N) {
+      atomicOr(status, kErrBadIndex);
+    } else {
+      topk_idx[(size_t)t * K + rank] = my_e;
+      topk_gate[(size_t)t * K + rank] = my_s / sum;
+      atomicAdd(&hist[my_e], 1);
+    }
+  }
+}
+
+// fp32 inputs: SIMT score tile + selection (see the top of this file).
 template <typename XT>
 __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
                                                     const float* __restrict__ router,
@@ -108,103 +203,48 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
   }
 
   // ---- phase 2: selection, one token at a time per warp ----
-  const int gs = N / G;
   float bj[kEPL];
 #pragma unroll
-  for (int j = 0; j < kEPL; ++j) {
-    const int e = lane + 32 * j;
-    bj[j] = (e < N) ? bias[e] : 0.f;
-  }
-
+  for (int j = 0; j < kEPL; ++j) bj[j] = (lane + 32 * j < N) ? bias[lane + 32 * j] : 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int t = t0 + warp * 4 + i;
     if (t >= T) break;  // warp-uniform
-    float s[kEPL], sb[kEPL];
+    float s[kEPL];
 #pragma unroll
-    for (int j = 0; j < kEPL; ++j) {
-      const int e = lane + 32 * j;
-      s[j] = 1.f / (1.f + expf(-acc[i][j]));
-      sb[j] = (e < N) ? s[j] + bj[j] : -INFINITY;
-    }
-    // group scores: lane g ends up holding group g's score
-    float my_gscore = -INFINITY;
-    for (int g = 0; g < G; ++g) {
-      float m1 = -INFINITY, m2 = -INFINITY;
+    for (int j = 0; j < kEPL; ++j) s[j] = 1.f / (1.f + expf(-acc[i][j]));
+    select_token(s, bj, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
+  }
+  __syncthreads();
+  for (int e = tid; e < N; e += blockDim.x)
+    if (hist[e]) atomicAdd(&counts[e], hist[e]);
+}
+
+// Selection from precomputed sigmoid scores S [T, N] (tensor-core path):
+// warp per token, 32 tokens per CTA.
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ S,
+                                                     const float* __restrict__ bias, int T, int N,
+                                                     int K, int G, int topG,
+                                                     int32_t* __restrict__ topk_idx,
+                                                     float* __restrict__ topk_gate,
+                                                     int32_t* __restrict__ counts,
+                                                     uint32_t* __restrict__ status) {
+  __shared__ int hist[kRouteMaxN];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < N; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  float bj[kEPL];
 #pragma unroll
-      for (int j = 0; j < kEPL; ++j) {
-        const int e = lane + 32 * j;
-        if (e < N && e / gs == g) top2_merge(m1, m2, sb[j], -INFINITY);
-      }
+  for (int j = 0; j < kEPL; ++j) bj[j] = (lane + 32 * j < N) ? bias[lane + 32 * j] : 0.f;
+  for (int i = 0; i < 4; ++i) {
+    const int t = blockIdx.x * kBT + warp * 4 + i;
+    if (t >= T) break;
+    float s[kEPL];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float b1 = __shfl_xor_sync(0xffffffffu, m1, o);
-        const float b2 = __shfl_xor_sync(0xffffffffu, m2, o);
-        top2_merge(m1, m2, b1, b2);
-      }
-      const float score = (gs >= 2) ? m1 + m2 : m1;
-      if (lane == g) my_gscore = score;
-    }
-    // keep the topG best groups
-    uint32_t kept = 0;
-    for (int r = 0; r < topG; ++r) {
-      float v = ((kept >> lane) & 1u) ? -INFINITY : my_gscore;
-      int gi = (lane < G && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
-      if (lane >= G) v = -INFINITY;
-      warp_argmax(v, gi);
-      kept |= 1u << gi;
-    }
-    // top-K among experts of kept groups
-    uint32_t taken = 0;  // bit j: this lane's expert lane+32j already chosen
-    int my_e = 0x7fffffff;
-    float my_s = 0.f;
-    for (int r = 0; r < K; ++r) {
-      float v = -INFINITY;
-      int ei = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < kEPL; ++j) {
-        const int e = lane + 32 * j;
-        if (e < N && ((kept >> (e / gs)) & 1u) && !((taken >> j) & 1u) &&
-            better(sb[j], e, v, ei)) {
-          v = sb[j];
-          ei = e;
-        }
-      }
-      warp_argmax(v, ei);
-      // the owner marks it and broadcasts its un-biased score
-      float sv = 0.f;
-#pragma unroll
-      for (int j = 0; j < kEPL; ++j) {
-        if (lane + 32 * j == ei) {
-          taken |= 1u << j;
-          sv = s[j];
-        }
-      }
-      const int owner = ei & 31;
-      sv = __shfl_sync(0xffffffffu, sv, owner);
-      if (lane == r) {
-        my_e = ei;
-        my_s = sv;
-      }
-    }
-    // ascending expert order and gates
-    int rank = 0;
-    for (int q = 0; q < K; ++q) {
-      const int eq = __shfl_sync(0xffffffffu, my_e, q);
-      rank += (eq < my_e) ? 1 : 0;
-    }
-    float sum = (lane < K) ? my_s : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane < K) {
-      if (my_e < 0 || my_e >= N) {
-        atomicOr(status, kErrBadIndex);
-      } else {
-        topk_idx[(size_t)t * K + rank] = my_e;
-        topk_gate[(size_t)t * K + rank] = my_s / sum;
-        atomicAdd(&hist[my_e], 1);
-      }
-    }
+    for (int j = 0; j < kEPL; ++j)
+      s[j] = (lane + 32 * j < N) ? __ldg(S + (size_t)t * N + lane + 32 * j) : 0.f;
+    select_token(s, bj, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
   }
   __syncthreads();
   for (int e = tid; e < N; e += blockDim.x)
@@ -213,21 +253,25 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
 
 }  // namespace
 
-cudaError_t launch_route(const moe_shape& s, const void* x, const float* router,
-                         const float* bias, int32_t* idx, float* gate, int32_t* counts,
-                         uint32_t* status, cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * s.N, st);
-  if (e != cudaSuccess) return e;
+int launch_route(const moe_shape& s, const void* x, const float* router, const float* bias,
+                 int32_t* idx, float* gate, int32_t* counts, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * s.N, st) != cudaSuccess) return MOE_ERR_CUDA;
   const int grid = (s.T + kBT - 1) / kBT;
-  if (s.dtype == MOE_DTYPE_FP32)
+  if (s.dtype == MOE_DTYPE_FP32) {
     route_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), router, bias, s.T,
                                               s.d, s.N, s.K, s.G, s.topG, idx, gate, counts,
                                               status);
-  else
-    route_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), router, bias, s.T, s.d, s.N, s.K, s.G, s.topG,
-        idx, gate, counts, status);
-  return cudaGetLastError();
+  } else {
+    float* S = reinterpret_cast<float*>(w + L.scores);
+    const int rc = launch_router_scores_tc(s, x, router, S, ws, st);
+    if (rc != MOE_OK) return rc;
+    select_kernel<<<grid, 256, 0, st>>>(S, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate, counts,
+                                        status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

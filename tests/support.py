@@ -49,6 +49,18 @@ def host_weights(cfg: MoEConfig, seed: int = 0):
     return get
 
 
+def streaming_weights(cfg: MoEConfig, seed: int = 0):
+    """Oracle-side accessor e -> (W1, W3, W2) float64 that regenerates each
+    expert into the same three buffers (the oracle uses one expert at a time),
+    for full-size layers whose weights do not fit in host memory at once."""
+    bufs = {w: np.empty(gen.weight_shape(cfg, w), np.float64) for w in ("w1", "w3", "w2")}
+
+    def get(e):
+        return tuple(gen.make_expert_weight(cfg, seed, w, e, out=bufs[w])
+                     for w in ("w1", "w3", "w2"))
+    return get
+
+
 def rel_fro(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
