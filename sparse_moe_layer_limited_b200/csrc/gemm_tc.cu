@@ -5,48 +5,38 @@
 // SwiGLU form y = (silu(a W1^T) * (a W3^T)) W2^T; the routed experts run on
 // their dispatched rows and the shared expert on every token, all in one
 // persistent launch per GEMM:
-//   GEMM1  H[rows_g, f] = SwiGLU of [rows_g, d] x [d, 2f]   (bf16 out)
-//   GEMM2  Y[rows_g, d] = [rows_g, f] x [f, d]             (bf16 out)
+//   GEMM1  [rows_g, d] x [d, 2f] -> SwiGLU epilogue -> H [rows_g, f] (bf16)
+//   GEMM2  [rows_g, f] x [f, d]  -> Y [rows_g, d] (bf16)
 // Group g < N is routed expert g (rows offsets[g]..offsets[g+1]); group N is
 // the shared expert (T rows).
 //
-// Orientation: the weights are the MMA's M side and the tokens its N side
-// (D^T = W . A^T).  A tile is 256 weight rows (two tcgen05.mma M=128 halves
-// into two TMEM column ranges) by up to 128 token rows; the token count of a
-// tile is rounded up to a multiple of 16 only, so the ragged last tile of an
-// expert costs MMA work in proportion to its rows (a 128-row M tile over the
-// tokens would waste about a quarter of the routed work at ~256 rows per
-// expert).  In GEMM1 the packed weight rows hold, per 128-row block j, W1
-// rows then W3 rows, so TMEM lane i of the two halves holds the gate and the
-// up projection of the same hidden feature: SwiGLU needs no data exchange.
-//
-// Work units are ordered group-major, then weight tile, then token tile, so
-// CTAs running side by side read the same weight tile (one HBM read, the
-// rest from L2).  Each CTA (one per SM) walks units blockIdx.x, +gridDim.x,
-// ... with three roles:
-//   warp 0    one thread issues TMA loads (128-byte swizzle) of 64-wide K
-//             slices: 256 weight rows + 128 token rows per stage, 4 stages;
+// Work unit: a 128 x 256 output tile (tcgen05.mma cta_group::1, M=128,
+// N=256, K=16 per instruction), ordered group-major, then n-tile, then
+// m-tile, so CTAs running side by side share the same weight tile through
+// L2 and each expert's weights stream from HBM about once.  Each CTA (one
+// per SM) walks tiles blockIdx.x, +gridDim.x, ... with three roles:
+//   warp 0    one thread issues TMA loads of 64-wide K slices of A and B
+//             (128-byte swizzle) into a 4-stage shared-memory ring;
 //   warp 1    allocates 512 TMEM columns (two 256-column accumulators) and
-//             one thread issues the MMAs (K=16 each), committing each ring
-//             slot back to the producer and each accumulator to the epilogue;
-//   warps 2-5 drain an accumulator with tcgen05.ld (thread = weight row,
-//             32 token columns per load) while the next unit accumulates in
-//             the other buffer, apply the epilogue and store: consecutive
-//             lanes write consecutive output features of one token row.
-// The producer also prefetches each weight K block into L2 a few blocks
-// ahead of its shared-memory load, so the first CTA on a weight tile does not
-// stall on HBM latency with only four stages in flight.
+//             one thread issues the MMAs, committing each ring slot back to
+//             the producer and each finished accumulator to the epilogue;
+//   warps 2-5 drain an accumulator with tcgen05.ld (one TMEM lane = one
+//             output row per thread) while the next tile accumulates in the
+//             other buffer, apply SwiGLU (GEMM1), round to bf16 and store
+//             the rows that belong to the group.
+// In GEMM1 the packed weight rows hold, per 128-row block j, W1 rows then
+// W3 rows, so one accumulator tile holds matching gate and up columns.
 // Every mbarrier wait is bounded (~2 s); a wait that gives up sets the
 // device status word and the CTA unwinds, frees its TMEM and returns.
 //
 // The same kernel computes the router scores z = x . e_i (one group of T
-// token rows; the "weights" are the experts): the fp32 router matrix is
-// split exactly into three bf16 parts R = R0 + R1 + R2 (R0 = bf16(R),
-// R1 = bf16(R - R0), R2 = bf16(R - R0 - R1), residual below 2^-27 |R|),
-// stored as one [N, 3d] operand whose 64-column blocks run (R0, R1, R2) per
-// 64 columns of d; each token tile of x serves three consecutive K blocks
-// (x_rep = 3), so the fp32 accumulator receives x.R0 + x.R1 + x.R2 = x.R.
-// The sigmoid epilogue writes s = sigmoid(z) as fp32 [T, N].
+// rows, tile width N): the fp32 router matrix is split exactly into three
+// bf16 parts R = R0 + R1 + R2 (R0 = bf16(R), R1 = bf16(R - R0), R2 =
+// bf16(R - R0 - R1), residual below 2^-27 |R|), stored as one [N, 3d]
+// operand whose 64-column blocks run (R0, R1, R2) per 64 columns of d; each
+// A tile of x is used for three consecutive K blocks (a_rep = 3), so the
+// fp32 accumulator receives x.R0 + x.R1 + x.R2 = x.R.  The sigmoid epilogue
+// writes s = sigmoid(z) as fp32 for the selection kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -59,49 +49,64 @@
 namespace moe {
 namespace {
 
-constexpr int BW = 256;   // weight rows per unit (two M=128 MMAs)
-constexpr int BT = 128;   // token rows per unit (MMA N <= 128)
-constexpr int BK = 64;    // bf16 K slice: 128 bytes = one swizzle row
+constexpr int BM = 128, BK = 64;  // BK bf16 = 128 bytes = one swizzle row
 constexpr int kStages = 4;
-constexpr int kWBytes = BW * BK * 2;         // 32 KB
-constexpr int kXBytes = BT * BK * 2;         // 16 KB
-constexpr int kStageBytes = kWBytes + kXBytes;
-constexpr int kAccCols = 256;                // per accumulator: 2 halves x 128 token columns
-constexpr int kTmemCols = 2 * kAccCols;
+constexpr int kABytes = BM * BK * 2;
 constexpr int kThreads = 192;
-constexpr int kPrefetchAhead = 8;  // weight K blocks brought into L2 ahead of their load
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiSigmoid = 2 };
 
-struct alignas(64) GemmArgs {
-  CUtensorMap tmW;          // weights [(groups) * n_feat rows, k_dim], box {64, 256}
-  CUtensorMap tmX_routed;   // token rows of routed groups, box {64, 128}
-  CUtensorMap tmX_shared;   // token rows of the shared group
-  const int32_t* offsets;
-  __nv_bfloat16* out_routed;  // row (offsets[g] + r)
-  __nv_bfloat16* out_shared;  // row r
-  float* out_f32;             // sigmoid epilogue: [T, n_valid]
-  uint32_t* status;
-  int N, T;
-  int rows_routed;    // T*K
-  int x_shared_row0;  // first token row of the shared group in tmX_shared
-  int n_feat;         // weight rows per group (2f for GEMM1, d for GEMM2)
-  int k_dim;          // contraction length of the weight operand
-  int x_rep;          // K blocks served by one token tile (3 for the split router)
-  int out_ld;         // output row stride (elements)
-  int n_valid;        // sigmoid epilogue: experts to store
+template <int kBN>
+struct TileCfg {
+  static constexpr int kBBytes = kBN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * kBN;  // two accumulators
+  static constexpr size_t smem_bytes(int groups) {
+    return 1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(groups + 1) * 4;
+  }
 };
 
-constexpr size_t smem_bytes_for(int groups) {
-  return 1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(groups + 1) * 4;
-}
+struct alignas(64) GemmArgs {
+  CUtensorMap tmA_routed;
+  CUtensorMap tmA_shared;
+  CUtensorMap tmB;
+  const int32_t* offsets;
+  __nv_bfloat16* out_routed;
+  __nv_bfloat16* out_shared;
+  float* out_f32;   // sigmoid epilogue: [T, n_valid]
+  uint32_t* status;
+  int N, T;
+  int rows_routed;  // T*K
+  int a_shared_row0;
+  int n_acc;   // accumulator columns per expert (2f for GEMM1, d for GEMM2)
+  int k_dim;   // contraction length
+  int out_ld;  // output row stride in elements
+  int a_rep;   // K blocks that reuse one A tile (3 for the split router, else 1)
+  int n_valid; // columns to store (sigmoid epilogue)
+};
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
-template <int kEpi>
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) {
+  uint4 w[4];
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = w[i];
+}
+
+template <int kEpi, int kBN>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     const __grid_constant__ GemmArgs args) {
+  constexpr int BN = kBN;
+  constexpr int kBBytes = TileCfg<kBN>::kBBytes;
+  constexpr int kStageBytes = TileCfg<kBN>::kStageBytes;
+  constexpr int kTmemCols = TileCfg<kBN>::kTmemCols;
+  static_assert(kEpi != kEpiSwiGLU || kBN == 256, "SwiGLU tiles pair 128 gate + 128 up columns");
+  (void)kBBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -112,15 +117,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   uint64_t* tempty = tfull + 2;          // [2]
   uint64_t* drain = tempty + 2;          // [1]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  int* unit_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + 256);
+  int* tile_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + 256);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int G1 = args.N + 1;
-  const int NF = args.n_feat / BW;   // weight tiles per group (router: 1)
+  const int NT = args.n_acc / BN;
   const int KB = args.k_dim / BK;
 
-  // ---- set-up: barriers, TMEM, unit schedule --------------------------------
+  // ---- set-up: barriers, TMEM, tile schedule --------------------------------
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -139,16 +144,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   }
   for (int g = tid; g < G1; g += kThreads) {
     const int rows = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
-    unit_start[g] = rows > 0 ? (rows + BT - 1) / BT : 0;
+    tile_start[g] = rows > 0 ? (rows + BM - 1) / BM : 0;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) {  // exclusive scan of token tiles per group, times NF
+  if (warp == 0) {  // exclusive scan of m-tiles per group, times NT
     const int per = (G1 + 31) / 32;
     const int g0 = min(G1, lane * per), g1 = min(G1, g0 + per);
     int sum = 0;
-    for (int g = g0; g < g1; ++g) sum += unit_start[g];
+    for (int g = g0; g < g1; ++g) sum += tile_start[g];
     int inc = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -157,64 +162,54 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     }
     int run = inc - sum;
     for (int g = g0; g < g1; ++g) {
-      const int mt = unit_start[g];
-      unit_start[g] = run * NF;
+      const int mt = tile_start[g];
+      tile_start[g] = run * NT;
       run += mt;
     }
-    if (lane == 31) unit_start[G1] = inc * NF;
+    if (lane == 31) tile_start[G1] = inc * NT;
   }
   __syncthreads();
   const uint32_t tmem_base = *tmem_holder;
-  const int total = unit_start[G1];
+  const int total = tile_start[G1];
 
-  // unit -> (group g, weight tile nf, token tile mt, token tiles of g)
-  auto decode = [&](int u, int& g, int& nf, int& mt) {
+  auto decode = [&](int tile, int& g, int& n, int& m, int& mt) {
     int lo = 0, hi = G1;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (unit_start[mid] <= u) lo = mid; else hi = mid;
+      if (tile_start[mid] <= tile) lo = mid; else hi = mid;
     }
     g = lo;
-    const int tiles = (unit_start[g + 1] - unit_start[g]) / NF;
-    const int local = u - unit_start[g];
-    nf = local / tiles;
-    mt = local - nf * tiles;
-  };
-  auto group_rows = [&](int g) {
-    return (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+    mt = (tile_start[g + 1] - tile_start[g]) / NT;
+    const int local = tile - tile_start[g];
+    n = local / mt;
+    m = local - n * mt;
   };
 
   if (warp == 0) {
     // ---- TMA producer ---------------------------------------------------------
     if (lane == 0) {
-      tma_prefetch_desc(&args.tmW);
-      tma_prefetch_desc(&args.tmX_routed);
-      tma_prefetch_desc(&args.tmX_shared);
+      tma_prefetch_desc(&args.tmA_routed);
+      tma_prefetch_desc(&args.tmA_shared);
+      tma_prefetch_desc(&args.tmB);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        int g, nf, mt;
-        decode(u, g, nf, mt);
-        const CUtensorMap* xm = (g < args.N) ? &args.tmX_routed : &args.tmX_shared;
-        const int xrow = ((g < args.N) ? args.offsets[g] : args.x_shared_row0) + mt * BT;
-        const int wrow = g * args.n_feat + nf * BW;
-        // the first CTA to reach a weight tile misses L2 on every K block; an
-        // L2 prefetch a few blocks ahead turns those misses into hits
-        for (int kb = 0; kb < min(kPrefetchAhead, KB); ++kb)
-          tma_prefetch_l2_2d(&args.tmW, kb * BK, wrow);
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, n, m, mt;
+        decode(tile, g, n, m, mt);
+        const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
+        const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * BM;
+        const int brow = g * args.n_acc + n * BN;
         for (int kb = 0; kb < KB; ++kb) {
-          if (kb + kPrefetchAhead < KB)
-            tma_prefetch_l2_2d(&args.tmW, (kb + kPrefetchAhead) * BK, wrow);
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs)) {
             ok = false;
             break;
           }
-          uint8_t* sw = base + (size_t)stage * kStageBytes;
+          uint8_t* sa = base + (size_t)stage * kStageBytes;
           mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          tma_load_2d(sw, &args.tmW, kb * BK, wrow, &full[stage]);
-          tma_load_2d(sw + kWBytes, xm, (kb / args.x_rep) * BK, xrow, &full[stage]);
+          tma_load_2d(sa, am, (kb / args.a_rep) * BK, arow, &full[stage]);
+          tma_load_2d(sa + kABytes, &args.tmB, kb * BK, brow, &full[stage]);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -232,36 +227,29 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   } else if (warp == 1) {
     // ---- MMA issuer -----------------------------------------------------------
     if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++local) {
-        int g, nf, mt;
-        decode(u, g, nf, mt);
-        const int ntok = min(BT, group_rows(g) - mt * BT);
-        const int n_mma = (ntok + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aphase ^ 1u, args.status, kTimeoutNs)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + acc * kAccCols;
+        const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, args.status, kTimeoutNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t w0 = smem_u32(base + (size_t)stage * kStageBytes);
-          const uint32_t x0 = w0 + kWBytes;
+          const uint32_t a0 = smem_u32(base + (size_t)stage * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t xd = smem_desc_sw128(x0 + k * 32);
-            mma_bf16(d0, smem_desc_sw128(w0 + k * 32), xd, idesc, (kb | k) != 0);
-            mma_bf16(d0 + 128, smem_desc_sw128(w0 + kWBytes / 2 + k * 32), xd, idesc,
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
                      (kb | k) != 0);
-          }
           mma_commit(&empty[stage]);
           if (++stage == kStages) {
             stage = 0;
@@ -275,59 +263,71 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     }
   } else {
     // ---- epilogue: warps 2..5 --------------------------------------------------
-    const int q = warp & 3;      // TMEM lane quadrant this warp may access
-    const int j = q * 32 + lane; // weight row within each 128-row half
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
     int local = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
-      int g, nf, mt;
-      decode(u, g, nf, mt);
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      int g, n, m, mt;
+      decode(tile, g, n, m, mt);
       const int acc = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
       if (!mbar_wait_bounded(&tfull[acc], aphase, args.status, kTimeoutNs)) break;
       tc_fence_after();
-      const int ntok = min(BT, group_rows(g) - mt * BT);
-      // output row of the unit's first token
-      const long long row0 =
-          (g < args.N) ? (long long)args.offsets[g] + mt * BT : (long long)mt * BT;
-      const bool in_range =
-          (g == args.N) || (args.offsets[g] >= 0 && row0 + ntok <= args.rows_routed);
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kAccCols;
+      const int rows_g = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+      const int r = m * BM + row;
+      // rows past the group's end belong to the next group (or are padding);
+      // the second test keeps a corrupted offsets[] from writing out of range
+      const bool valid = r < rows_g && (g == args.N || args.offsets[g] + r < args.rows_routed);
+      __nv_bfloat16* orow =
+          (g < args.N) ? args.out_routed + (size_t)(args.offsets[g] + r) * args.out_ld
+                       : args.out_shared + (size_t)r * args.out_ld;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if constexpr (kEpi == kEpiSwiGLU) {
 #pragma unroll 1
-      for (int c = 0; c < ntok; c += 32) {
-        uint32_t v0[32], v1[32];
-        tmem_ld32(taddr + c, v0);
-        tmem_ld32(taddr + 128 + c, v1);
-        tmem_wait_ld();
-        if (!in_range) continue;
-        if constexpr (kEpi == kEpiSwiGLU) {
-          __nv_bfloat16* o = ((g < args.N) ? args.out_routed : args.out_shared) +
-                             (row0 + c) * args.out_ld + nf * 128 + j;
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t ga[32], up[32];
+          tmem_ld32(taddr + c, ga);
+          tmem_ld32(taddr + BN / 2 + c, up);
+          tmem_wait_ld();
+          float h[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c + i < ntok)
-              o[(long long)i * args.out_ld] = __float2bfloat16_rn(
-                  silu_f(__uint_as_float(v0[i])) * __uint_as_float(v1[i]));
-        } else if constexpr (kEpi == kEpiStore) {
-          __nv_bfloat16* o = ((g < args.N) ? args.out_routed : args.out_shared) +
-                             (row0 + c) * args.out_ld + nf * BW + j;
+            h[i] = silu_f(__uint_as_float(ga[i])) * __uint_as_float(up[i]);
+          if (valid) store_row32(orow + n * (BN / 2) + c, h);
+        }
+      } else if constexpr (kEpi == kEpiStore) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          float y[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c + i < ntok) {
-              o[(long long)i * args.out_ld] = __float2bfloat16_rn(__uint_as_float(v0[i]));
-              o[(long long)i * args.out_ld + 128] = __float2bfloat16_rn(__uint_as_float(v1[i]));
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
+          if (valid) store_row32(orow + n * BN + c, y);
+        }
+      } else {  // sigmoid scores, fp32, columns < n_valid
+        float* srow = args.out_f32 + (size_t)r * args.n_valid;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (valid && c < args.n_valid) {
+            float sg[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sg[i] = 1.f / (1.f + expf(-__uint_as_float(v[i])));
+            if (c + 32 <= args.n_valid) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(srow + c + i) =
+                    make_float4(sg[i], sg[i + 1], sg[i + 2], sg[i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c + i < args.n_valid) srow[c + i] = sg[i];
             }
-        } else {  // sigmoid scores, fp32, experts < n_valid
-          float* o = args.out_f32 + (row0 + c) * args.n_valid;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c + i < ntok) {
-              if (j < args.n_valid)
-                o[(long long)i * args.n_valid + j] =
-                    1.f / (1.f + expf(-__uint_as_float(v0[i])));
-              if (128 + j < args.n_valid)
-                o[(long long)i * args.n_valid + 128 + j] =
-                    1.f / (1.f + expf(-__uint_as_float(v1[i])));
-            }
+          }
         }
       }
       tc_fence_before();
@@ -387,13 +387,13 @@ int num_sms() {
   return n;
 }
 
-template <int kEpi>
+template <int kEpi, int kBN>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
-  const size_t smem = smem_bytes_for(a.N + 1);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi>,
+  const size_t smem = TileCfg<kBN>::smem_bytes(a.N + 1);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_bf16_kernel<kEpi><<<num_sms(), kThreads, smem, st>>>(a);
+  grouped_gemm_bf16_kernel<kEpi, kBN><<<num_sms(), kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -430,47 +430,44 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(w + L.h);
   const uint64_t TK = (uint64_t)s.T * s.K;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
 
-  // GEMM1: weights W13 [(N+1)*2f, d], tokens x_perm (routed) / x (shared)
   GemmArgs g1{};
-  bool ok = make_map(&g1.tmW, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, BW) &&
-            make_map(&g1.tmX_routed, x_perm, BF, 2, s.d, TK, BK, BT) &&
-            make_map(&g1.tmX_shared, x, BF, 2, s.d, s.T, BK, BT);
+  bool ok = make_map(&g1.tmA_routed, x_perm, BF, 2, s.d, TK, BK, BM) &&
+            make_map(&g1.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, 256);
   if (!ok) return MOE_ERR_CUDA;
   g1.offsets = offsets;
   g1.out_routed = H;
   g1.out_shared = H + TK * s.f;
-  g1.status = status;
+  g1.status = reinterpret_cast<uint32_t*>(w + L.status);
   g1.N = s.N;
   g1.T = s.T;
   g1.rows_routed = (int)TK;
-  g1.x_shared_row0 = 0;
-  g1.n_feat = 2 * s.f;
+  g1.a_shared_row0 = 0;
+  g1.n_acc = 2 * s.f;
   g1.k_dim = s.d;
-  g1.x_rep = 1;
   g1.out_ld = s.f;
-  if (launch_gemm<kEpiSwiGLU>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+  g1.a_rep = 1;
+  if (launch_gemm<kEpiSwiGLU, 256>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
 
-  // GEMM2: weights W2 [(N+1)*d, f], tokens H (routed rows, then the shared rows)
   GemmArgs g2{};
-  ok = make_map(&g2.tmW, w2, BF, 2, s.f, (uint64_t)(s.N + 1) * s.d, BK, BW) &&
-       make_map(&g2.tmX_routed, H, BF, 2, s.f, TK + s.T, BK, BT) &&
-       make_map(&g2.tmX_shared, H, BF, 2, s.f, TK + s.T, BK, BT);
+  ok = make_map(&g2.tmA_routed, H, BF, 2, s.f, TK + s.T, BK, BM) &&
+       make_map(&g2.tmA_shared, H, BF, 2, s.f, TK + s.T, BK, BM) &&
+       make_map(&g2.tmB, w2, BF, 2, s.f, (uint64_t)(s.N + 1) * s.d, BK, 256);
   if (!ok) return MOE_ERR_CUDA;
   g2.offsets = offsets;
   g2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   g2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
-  g2.status = status;
+  g2.status = g1.status;
   g2.N = s.N;
   g2.T = s.T;
   g2.rows_routed = (int)TK;
-  g2.x_shared_row0 = (int)TK;
-  g2.n_feat = s.d;
+  g2.a_shared_row0 = (int)TK;
+  g2.n_acc = s.d;
   g2.k_dim = s.f;
-  g2.x_rep = 1;
   g2.out_ld = s.d;
-  if (launch_gemm<kEpiStore>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+  g2.a_rep = 1;
+  if (launch_gemm<kEpiStore, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -485,25 +482,29 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
   router_split_kernel<<<(int)blocks, 256, 0, st>>>(router, s.N, s.d, Rs);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
+  const int bn = s.N <= 64 ? 64 : (s.N <= 128 ? 128 : 256);
   GemmArgs a{};
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  bool ok = make_map(&a.tmW, Rs, BF, 2, 3ull * s.d, s.N, BK, BW) &&
-            make_map(&a.tmX_routed, x, BF, 2, s.d, s.T, BK, BT) &&
-            make_map(&a.tmX_shared, x, BF, 2, s.d, s.T, BK, BT);
+  bool ok = make_map(&a.tmA_routed, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&a.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&a.tmB, Rs, BF, 2, 3ull * s.d, s.N, BK, bn);
   if (!ok) return MOE_ERR_CUDA;
   a.offsets = nullptr;
   a.out_f32 = S;
   a.status = reinterpret_cast<uint32_t*>(w + L.status);
-  a.N = 0;  // a single group: all T token rows of x
+  a.N = 0;  // a single group: all T rows of x
   a.T = s.T;
   a.rows_routed = 0;
-  a.x_shared_row0 = 0;
-  a.n_feat = BW;  // one weight tile: experts 0..255 (rows >= N read as zero)
+  a.a_shared_row0 = 0;
+  a.n_acc = bn;
   a.k_dim = 3 * s.d;
-  a.x_rep = 3;
   a.out_ld = s.N;
+  a.a_rep = 3;
   a.n_valid = s.N;
-  return launch_gemm<kEpiSigmoid>(a, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  cudaError_t e = bn == 64    ? launch_gemm<kEpiSigmoid, 64>(a, st)
+                  : bn == 128 ? launch_gemm<kEpiSigmoid, 128>(a, st)
+                              : launch_gemm<kEpiSigmoid, 256>(a, st);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe
