@@ -21,7 +21,7 @@ WsLayout ws_layout(const moe_shape& s) {
     L.router_split = off;
     off = align256(off + (size_t)s.N * 3 * s.d * 2);
     L.scores = off;
-    off = align256(off + (size_t)s.T * s.N * 4);
+    off = align256(off + (size_t)8 * s.T * s.N * 4);
   }
   const size_t rows = (size_t)s.T * s.K + s.T;
   L.h = off;

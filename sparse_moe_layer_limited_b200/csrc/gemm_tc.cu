@@ -35,8 +35,11 @@
 // bf16(R - R0 - R1), residual below 2^-27 |R|), stored as one [N, 3d]
 // operand whose 64-column blocks run (R0, R1, R2) per 64 columns of d; each
 // A tile of x is used for three consecutive K blocks (a_rep = 3), so the
-// fp32 accumulator receives x.R0 + x.R1 + x.R2 = x.R.  The sigmoid epilogue
-// writes s = sigmoid(z) as fp32 for the selection kernel.
+// fp32 accumulator receives x.R0 + x.R1 + x.R2 = x.R.  With only T/128 token
+// tiles, the 3d-long K loop is split into k_splits ranges run by separate
+// units (the n-tile index carries the split); each writes its fp32 partial
+// z to its own [T, N] slab, and the selection kernel adds the slabs in split
+// order (deterministic) before the sigmoid.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -55,7 +58,7 @@ constexpr int kABytes = BM * BK * 2;
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiSigmoid = 2 };
+enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiScores = 2 };
 
 template <int kBN>
 struct TileCfg {
@@ -74,7 +77,7 @@ struct alignas(64) GemmArgs {
   const int32_t* offsets;
   __nv_bfloat16* out_routed;
   __nv_bfloat16* out_shared;
-  float* out_f32;   // sigmoid epilogue: [T, n_valid]
+  float* out_f32;   // score epilogue: fp32 partial sums [k_splits, T, n_valid]
   uint32_t* status;
   int N, T;
   int rows_routed;  // T*K
@@ -83,7 +86,8 @@ struct alignas(64) GemmArgs {
   int k_dim;   // contraction length
   int out_ld;  // output row stride in elements
   int a_rep;   // K blocks that reuse one A tile (3 for the split router, else 1)
-  int n_valid; // columns to store (sigmoid epilogue)
+  int n_valid; // columns to store (score epilogue)
+  int k_splits; // K ranges computed by separate units (score epilogue; else 1)
 };
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
@@ -122,8 +126,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int G1 = args.N + 1;
-  const int NT = args.n_acc / BN;
+  const int NT = (args.n_acc / BN) * args.k_splits;  // n-tiles x K splits
   const int KB = args.k_dim / BK;
+  const int KBs = (KB + args.k_splits - 1) / args.k_splits;  // K blocks per split
 
   // ---- set-up: barriers, TMEM, tile schedule --------------------------------
   if (tid == 0) {
@@ -200,8 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
         decode(tile, g, n, m, mt);
         const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
         const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * BM;
-        const int brow = g * args.n_acc + n * BN;
-        for (int kb = 0; kb < KB; ++kb) {
+        const int brow = g * args.n_acc + (n / args.k_splits) * BN;
+        const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs)) {
             ok = false;
             break;
@@ -233,12 +239,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
       int local = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        int g, n, m, mt;
+        decode(tile, g, n, m, mt);
+        const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
         const int acc = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aphase ^ 1u, args.status, kTimeoutNs)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, args.status, kTimeoutNs)) {
             ok = false;
             break;
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_bf16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
-                     (kb | k) != 0);
+                     ((kb - kb0) | k) != 0);
           mma_commit(&empty[stage]);
           if (++stage == kStages) {
             stage = 0;
@@ -306,26 +315,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
           if (valid) store_row32(orow + n * BN + c, y);
         }
-      } else {  // sigmoid scores, fp32, columns < n_valid
-        float* srow = args.out_f32 + (size_t)r * args.n_valid;
+      } else {  // raw fp32 scores of this K split, columns < n_valid
+        float* srow = args.out_f32 +
+                      ((size_t)(n % args.k_splits) * args.T + r) * args.n_valid;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
           tmem_ld32(taddr + c, v);
           tmem_wait_ld();
           if (valid && c < args.n_valid) {
-            float sg[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sg[i] = 1.f / (1.f + expf(-__uint_as_float(v[i])));
             if (c + 32 <= args.n_valid) {
 #pragma unroll
               for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4*>(srow + c + i) =
-                    make_float4(sg[i], sg[i + 1], sg[i + 2], sg[i + 3]);
+                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c + i < args.n_valid) srow[c + i] = sg[i];
+                if (c + i < args.n_valid) srow[c + i] = __uint_as_float(v[i]);
             }
           }
         }
@@ -448,6 +456,7 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g1.k_dim = s.d;
   g1.out_ld = s.f;
   g1.a_rep = 1;
+  g1.k_splits = 1;
   if (launch_gemm<kEpiSwiGLU, 256>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   GemmArgs g2{};
@@ -467,12 +476,22 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g2.k_dim = s.f;
   g2.out_ld = s.d;
   g2.a_rep = 1;
+  g2.k_splits = 1;
   if (launch_gemm<kEpiStore, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
-int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* S,
-                            void* ws, cudaStream_t st) {
+int router_k_splits(const moe_shape& s) {
+  const int m_tiles = (s.T + BM - 1) / BM;
+  const int KB = 3 * s.d / BK;
+  int want = num_sms() / m_tiles;  // fill the SMs with token tiles x K splits
+  want = want < 1 ? 1 : (want > 8 ? 8 : want);
+  while (want > 1 && KB % want != 0) --want;
+  return want;
+}
+
+int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* Z,
+                            int k_splits, void* ws, cudaStream_t st) {
   const WsLayout L = ws_layout(s);
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(w + L.router_split);
@@ -490,7 +509,7 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
             make_map(&a.tmB, Rs, BF, 2, 3ull * s.d, s.N, BK, bn);
   if (!ok) return MOE_ERR_CUDA;
   a.offsets = nullptr;
-  a.out_f32 = S;
+  a.out_f32 = Z;
   a.status = reinterpret_cast<uint32_t*>(w + L.status);
   a.N = 0;  // a single group: all T rows of x
   a.T = s.T;
@@ -501,9 +520,10 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
   a.out_ld = s.N;
   a.a_rep = 3;
   a.n_valid = s.N;
-  cudaError_t e = bn == 64    ? launch_gemm<kEpiSigmoid, 64>(a, st)
-                  : bn == 128 ? launch_gemm<kEpiSigmoid, 128>(a, st)
-                              : launch_gemm<kEpiSigmoid, 256>(a, st);
+  a.k_splits = k_splits;
+  cudaError_t e = bn == 64    ? launch_gemm<kEpiScores, 64>(a, st)
+                  : bn == 128 ? launch_gemm<kEpiScores, 128>(a, st)
+                              : launch_gemm<kEpiScores, 256>(a, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

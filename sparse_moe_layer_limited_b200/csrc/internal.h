@@ -21,7 +21,7 @@ struct WsLayout {
   size_t chunk_hist = 0;  // int32 [chunks, N]
   size_t chunk_base = 0;  // int32 [chunks, N]
   size_t router_split = 0;  // bf16 [N, 3d] exact three-part split of the router (bf16 x)
-  size_t scores = 0;        // fp32 [T, N] sigmoid affinities (bf16 x)
+  size_t scores = 0;        // fp32 [splits <= 8, T, N] partial router logits (bf16 x)
   size_t h = 0;           // hidden activation [T*K + T, f] (bf16 / fp32 / e4m3)
   size_t h_scales = 0;    // fp32 [T*K + T, f/128] (E4M3)
   size_t xq = 0;          // E4M3 codes of x for the shared expert [T, d]
@@ -54,9 +54,11 @@ cudaError_t launch_pack_w13(const moe_shape& s, const void* w1, const void* w3, 
 cudaError_t launch_ffn_simt(const moe_shape& s, const float* x_perm, const int32_t* offsets,
                             const float* x, const float* w13, const float* w2, float* y_perm,
                             float* y_shared, void* ws, cudaStream_t st);
-// Router scores on the tensor cores (bf16 x): S[t, i] = sigmoid(x_t . e_i).
-int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* S,
-                            void* ws, cudaStream_t st);
+// Router logits on the tensor cores (bf16 x): Z[split, t, i] = partial sums
+// of x_t . e_i over K split `split`; sum the splits in order for z.
+int router_k_splits(const moe_shape& s);
+int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* Z,
+                            int k_splits, void* ws, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* status (tensor maps can fail to encode).
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                        const void* x, const void* w13, const void* w2, void* y_perm,

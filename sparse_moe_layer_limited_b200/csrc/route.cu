@@ -7,9 +7,9 @@
 // (mhpq.cn article §3.1, "at most 4 nodes").  Group score = sum of the two
 // largest biased scores in the group (the reading this library takes).
 //
-// bf16 inputs: the scores come from the tensor cores (an exact three-part
-// bf16 split of the fp32 router, see gemm_tc.cu) into a [T, N] fp32 buffer,
-// and select_kernel does the per-token selection below.
+// bf16 inputs: the logits come from the tensor cores (an exact three-part
+// bf16 split of the fp32 router, see gemm_tc.cu) as fp32 K-split partials,
+// and select_kernel sums them, applies the sigmoid and selects (below).
 //
 // fp32 inputs: one CTA handles 32 tokens against all N (<= 256) experts.
 // Phase 1 is a SIMT fp32 GEMM tile: x and the router are staged through shared memory in
@@ -220,9 +220,10 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
     if (hist[e]) atomicAdd(&counts[e], hist[e]);
 }
 
-// Selection from precomputed sigmoid scores S [T, N] (tensor-core path):
-// warp per token, 32 tokens per CTA.
-__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ S,
+// Selection from the tensor-core logits Z [splits, T, N]: z is the sum of
+// the split partials in split order, s = sigmoid(z); warp per token, 32
+// tokens per CTA.
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z, int splits,
                                                      const float* __restrict__ bias, int T, int N,
                                                      int K, int G, int topG,
                                                      int32_t* __restrict__ topk_idx,
@@ -242,8 +243,15 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ S
     if (t >= T) break;
     float s[kEPL];
 #pragma unroll
-    for (int j = 0; j < kEPL; ++j)
-      s[j] = (lane + 32 * j < N) ? __ldg(S + (size_t)t * N + lane + 32 * j) : 0.f;
+    for (int j = 0; j < kEPL; ++j) {
+      float z = 0.f;
+      if (lane + 32 * j < N) {
+        z = __ldg(Z + (size_t)t * N + lane + 32 * j);
+        for (int p = 1; p < splits; ++p)
+          z = __fadd_rn(z, __ldg(Z + ((size_t)p * T + t) * N + lane + 32 * j));
+      }
+      s[j] = 1.f / (1.f + expf(-z));
+    }
     select_token(s, bj, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
   }
   __syncthreads();
@@ -265,11 +273,12 @@ int launch_route(const moe_shape& s, const void* x, const float* router, const f
                                               s.d, s.N, s.K, s.G, s.topG, idx, gate, counts,
                                               status);
   } else {
-    float* S = reinterpret_cast<float*>(w + L.scores);
-    const int rc = launch_router_scores_tc(s, x, router, S, ws, st);
+    float* Z = reinterpret_cast<float*>(w + L.scores);
+    const int splits = router_k_splits(s);
+    const int rc = launch_router_scores_tc(s, x, router, Z, splits, ws, st);
     if (rc != MOE_OK) return rc;
-    select_kernel<<<grid, 256, 0, st>>>(S, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate, counts,
-                                        status);
+    select_kernel<<<grid, 256, 0, st>>>(Z, splits, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate,
+                                        counts, status);
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
