@@ -1,8 +1,8 @@
 """DeepSeekMoE layer forward for one NVIDIA B200 (sm_100a).
 
 The compute runs in ``libmoe_b200.so`` (hand-written CUDA, C ABI declared in
-``include/moe_b200.h``); this package only marshals arguments.  Import fails
-loudly when the library has not been built.
+``include/moe_b200.h``); this package only marshals arguments.  The library is
+loaded on first use, and any call fails loudly when it has not been built.
 """
 from ._lib import (  # noqa: F401
     DTYPE_BF16, DTYPE_E4M3, DTYPE_FP32, MoEError, MoEShape, check_shape, lib, moe_bias_update,
@@ -11,5 +11,3 @@ from ._lib import (  # noqa: F401
     workspace_size, x_torch_dtype, w_torch_dtype,
 )
 from .layer import MoELayer  # noqa: F401
-
-lib()
