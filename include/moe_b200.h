@@ -194,6 +194,29 @@ int moe_quantize_weights(const moe_shape* shape, const void* w13_bf16, const voi
                          void* w13_q, float* w13_scales, void* w2_q, float* w2_scales,
                          void* stream);
 
+/* moe_dispatch_noalloc: moe_dispatch for callers that cannot allocate device
+ * memory when they call in -- for example code that runs while a framework
+ * forbids new allocations, or a host application that hands the library only
+ * its input and output buffers -- and so cannot provide a workspace.  The
+ * pages describe no such entry point; it has no counterpart there.
+ * Arguments, layouts and results are those of moe_dispatch, without `ws`.
+ * Scratch: a fixed 1 MiB static device array inside the library (held on
+ * every GPU that loads the library until the process exits).  The dispatch
+ * tables need 256 + 2 * ceil(T/32) * N * 4 bytes (each table rounded up to
+ * 256 bytes); a shape that needs more than 1 MiB (e.g. T > 16384 at N = 256)
+ * returns MOE_ERR_WORKSPACE before anything is enqueued.  E4M3 mode returns
+ * MOE_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any
+ * stream capture.  All calls share the one array, so calls whose work
+ * overlaps on the GPU (different streams without ordering) race; calls on
+ * one stream are safe.  The device status word lives in the array and is
+ * cleared at the start of every call; it cannot be read back, but all
+ * writes stay in bounds as in moe_dispatch. */
+int moe_dispatch_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                         const int32_t* counts, int32_t* offsets, int32_t* perm_tok,
+                         int32_t* slot, void* x_perm, float* x_perm_scales, void* stream);
+
 /* The whole forward in order: route, dispatch, experts, combine, then the bias
  * update; intermediate buffers are caller-provided as in the calls above. */
 int moe_forward(const moe_shape* shape, const void* x, const float* router_w, float* bias,

@@ -46,6 +46,7 @@ _SIGS = {
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 10),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
+    "moe_dispatch_noalloc": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, ctypes.c_float,
                                        _c_p]),
     "moe_pack_w13": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 4),
@@ -158,6 +159,17 @@ def moe_dispatch(s, x, topk_idx, counts, offsets, perm_tok, slot, x_perm, x_perm
             s.T * s.K * s.d, "x_perm")
     _call("moe_dispatch", ctypes.byref(s), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
           _ptr(perm_tok), _ptr(slot), _ptr(x_perm), _ptr(x_perm_scales), _ptr(ws),
+          _stream(stream))
+
+
+def moe_dispatch_noalloc(s, x, topk_idx, counts, offsets, perm_tok, slot, x_perm,
+                         x_perm_scales=None, stream=None):
+    """moe_dispatch without a workspace (fixed static device scratch)."""
+    _expect(offsets, torch.int32, s.N + 1, "offsets")
+    _expect(perm_tok, torch.int32, s.T * s.K, "perm_tok")
+    _expect(slot, torch.int32, s.T * s.K, "slot")
+    _call("moe_dispatch_noalloc", ctypes.byref(s), _ptr(x), _ptr(topk_idx), _ptr(counts),
+          _ptr(offsets), _ptr(perm_tok), _ptr(slot), _ptr(x_perm), _ptr(x_perm_scales),
           _stream(stream))
 
 

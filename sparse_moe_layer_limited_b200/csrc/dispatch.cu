@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -180,3 +182,93 @@ cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* id
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Dispatch without a caller-provided workspace.
+//
+// For callers that cannot allocate device memory at call time (code running
+// inside a framework's allocator-free region, or a plugin host that hands
+// over only its input and output buffers), moe_dispatch_noalloc keeps the
+// three scratch regions of the dispatch (status word, per-chunk histograms,
+// per-chunk bases) in one fixed static device array of this file instead of
+// the caller's workspace.  The array is kNoAllocScratchBytes long and lives
+// on every GPU that loads the library until the process exits; shapes that
+// need more are rejected.  Host code cannot pass the array's name to a
+// kernel (on the host it is only a stand-in symbol), so its device address
+// is looked up with cudaGetSymbolAddress once per device, with that device
+// current, on the first call there.
+namespace moe {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;  // 1 MiB
+constexpr size_t kNoAllocStatusBytes = 256;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_dispatch_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_dispatch_scratch on the current device (nullptr on error).
+void* scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
+size_t noalloc_scratch_need(const moe_shape& s) {
+  const size_t table = (size_t)chunks_of(s.T) * s.N * sizeof(int32_t);
+  return kNoAllocStatusBytes + 2 * ((table + 255) & ~size_t(255));
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_dispatch_noalloc(const moe_shape* shape, const void* x,
+                                    const int32_t* topk_idx, const int32_t* counts,
+                                    int32_t* offsets, int32_t* perm_tok, int32_t* slot,
+                                    void* x_perm, float* x_perm_scales, void* stream) {
+  using namespace moe;
+  const int rc = moe_check_shape(shape);
+  if (rc != MOE_OK) return rc;
+  const moe_shape& s = *shape;
+  auto ok16 = [](const void* p) {
+    return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+  };
+  if (!ok16(x) || !ok16(topk_idx) || !ok16(counts) || !ok16(offsets) || !ok16(perm_tok) ||
+      !ok16(slot) || !ok16(x_perm))
+    return MOE_ERR_ARG;
+  if (s.dtype == MOE_DTYPE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (noalloc_scratch_need(s) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+  (void)x_perm_scales;
+
+  uint8_t* base = static_cast<uint8_t*>(scratch_on_current_device());
+  if (!base) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t table = ((size_t)chunks_of(s.T) * s.N * sizeof(int32_t) + 255) & ~size_t(255);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  int32_t* chunk_hist = reinterpret_cast<int32_t*>(base + kNoAllocStatusBytes);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(base + kNoAllocStatusBytes + table);
+  // the status word accumulates bits: start each call from zero (the tables are
+  // fully rewritten by the kernels below)
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const int nch = chunks_of(s.T);
+  chunk_hist_kernel<<<nch, 256, 0, st>>>(topk_idx, s.T, s.K, s.N, chunk_hist, status);
+  expert_scan_kernel<<<s.N, 256, 0, st>>>(counts, chunk_hist, nch, s.N, offsets, chunk_base,
+                                          status);
+  if (s.dtype == MOE_DTYPE_FP32)
+    scatter_gather_kernel<float><<<nch, 256, 0, st>>>(
+        static_cast<const float*>(x), topk_idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok, slot,
+        static_cast<float*>(x_perm));
+  else
+    scatter_gather_kernel<__nv_bfloat16><<<nch, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), topk_idx, chunk_base, s.T, s.d, s.K, s.N,
+        perm_tok, slot, static_cast<__nv_bfloat16*>(x_perm));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

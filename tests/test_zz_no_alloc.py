@@ -1,0 +1,86 @@
+"""The workspace-free dispatch entry point (moe_dispatch_noalloc).
+
+Some callers cannot allocate device memory at the moment they call the
+layer (for example while a framework forbids new allocations, or when a host
+application passes only its own input and output buffers), so they cannot
+supply the workspace moe_dispatch needs.  moe_dispatch_noalloc keeps that
+scratch in a fixed static device array instead.  These tests call it
+through the C ABI and require the same results as moe_dispatch on two calls
+in a row with different shapes (the shared array keeps the previous call's
+contents), and check that shapes beyond the array are refused up front.
+This file is collected last on purpose.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import CONFIGS, gen
+from tests import support as S
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    import sparse_moe_layer_limited_b200 as M
+    f = M.lib()
+    big = M.shape(20000, 256, 256, 8, 8, 4, 256, M.DTYPE_BF16)   # needs > 1 MiB of tables
+    fake = ctypes.c_void_p(1 << 20)                                # never dereferenced
+    rc = f.moe_dispatch_noalloc(ctypes.byref(big), fake, fake, fake, fake, fake, fake, fake,
+                                None, None)
+    assert rc == M._lib.ERR_WORKSPACE
+    ok = M.shape(1000, 256, 8, 2, 2, 1, 256, M.DTYPE_BF16)
+    assert f.moe_dispatch_noalloc(ctypes.byref(ok), None, fake, fake, fake, fake, fake, fake,
+                                  None, None) == M._lib.ERR_ARG
+
+
+def _inputs(cfg):
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
+    return x, r
+
+
+def _dispatch_both(M, cfg, x, r):
+    import torch
+    s = S.moe_shape(cfg)
+    xd = S.to_dev_x(x, cfg)
+    idx = torch.from_numpy(r["idx"].astype(np.int32)).cuda()
+    counts = torch.from_numpy(r["counts"].astype(np.int32)).cuda()
+    outs = []
+    for which in ("ws", "noalloc"):
+        off = torch.full((s.N + 1,), -7, dtype=torch.int32, device="cuda")
+        perm = torch.full((s.T * s.K,), -7, dtype=torch.int32, device="cuda")
+        slot = torch.full((s.T, s.K), -7, dtype=torch.int32, device="cuda")
+        xp = torch.zeros(s.T * s.K, s.d, dtype=xd.dtype, device="cuda")
+        if which == "ws":
+            ws = torch.zeros(M.workspace_size(s), dtype=torch.uint8, device="cuda")
+            M.moe_dispatch(s, xd, idx, counts, off, perm, slot, xp, None, ws)
+        else:
+            rc = M.lib().moe_dispatch_noalloc(
+                ctypes.byref(s), ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(idx.data_ptr()),
+                ctypes.c_void_p(counts.data_ptr()), ctypes.c_void_p(off.data_ptr()),
+                ctypes.c_void_p(perm.data_ptr()), ctypes.c_void_p(slot.data_ptr()),
+                ctypes.c_void_p(xp.data_ptr()), None,
+                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+            assert rc == 0, M.status_string(rc)
+        torch.cuda.synchronize()
+        outs.append((off.cpu().numpy(), perm.cpu().numpy(), slot.cpu().numpy(),
+                     xp.float().cpu().numpy()))
+    return outs
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_dispatch_twice():
+    import sparse_moe_layer_limited_b200 as M
+    cases = [CONFIGS[1], CONFIGS[1].with_(T=1000, d=256, N=8, K=2, G=2, topG=1, f=256)]
+    for cfg in cases:                      # two calls in a row, different shapes
+        x, r = _inputs(cfg)
+        (o1, p1, s1, x1), (o2, p2, s2, x2) = _dispatch_both(M, cfg, x, r)
+        # integer outputs bit-exact; the gathered rows are copies, so exact too
+        np.testing.assert_array_equal(o2, o1)
+        np.testing.assert_array_equal(p2, p1)
+        np.testing.assert_array_equal(s2, s1)
+        np.testing.assert_array_equal(x2, x1)
+        d = oracle.dispatch(r["idx"], cfg.N)
+        np.testing.assert_array_equal(o2, d["offsets"])
+        np.testing.assert_array_equal(p2, d["perm_tok"])
