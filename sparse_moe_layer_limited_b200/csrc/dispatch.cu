@@ -17,6 +17,7 @@
 
 #include <mutex>
 
+#include "fp8_util.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -104,6 +105,39 @@ __global__ void __launch_bounds__(256) expert_scan_kernel(const int32_t* __restr
   }
 }
 
+// Rows of this chunk's (token, expert) pairs: rank among the chunk's earlier
+// tokens that chose the same expert, plus the chunk's base row for that
+// expert.  Writes slot[] and perm_tok[] and leaves the rows in sslot (-1 for
+// a pair that cannot be placed, which only happens when counts[] disagree
+// with idx; that is flagged by the histogram and scan kernels).
+__device__ __forceinline__ void chunk_slots(const int32_t* __restrict__ idx,
+                                            const int32_t* __restrict__ chunk_base, int c,
+                                            int t0, int nt, int T, int K, int N,
+                                            int32_t* __restrict__ perm_tok,
+                                            int32_t* __restrict__ slot, int* sidx, int* sslot) {
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) sidx[p] = idx[(size_t)t0 * K + p];
+  __syncthreads();
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) {
+    const int tl = p / K;
+    const int e = sidx[p];
+    if (e < 0 || e >= N) {
+      sslot[p] = -1;
+      continue;
+    }
+    int rank = 0;
+    for (int q = 0; q < tl * K; ++q) rank += (sidx[q] == e) ? 1 : 0;
+    const int r = chunk_base[(size_t)c * N + e] + rank;
+    if (r < 0 || r >= T * K) {
+      sslot[p] = -1;
+      continue;
+    }
+    sslot[p] = r;
+    slot[(size_t)t0 * K + p] = r;
+    perm_tok[r] = t0 + tl;
+  }
+  __syncthreads();
+}
+
 // Slots for one chunk, then the row gather (bf16 / fp32 rows copied verbatim).
 template <typename XT>
 __global__ void __launch_bounds__(256) scatter_gather_kernel(
@@ -115,27 +149,7 @@ __global__ void __launch_bounds__(256) scatter_gather_kernel(
   const int c = blockIdx.x;
   const int t0 = c * kChunkTokens;
   const int nt = min(kChunkTokens, T - t0);
-  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) sidx[p] = idx[(size_t)t0 * K + p];
-  __syncthreads();
-  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) {
-    const int tl = p / K;
-    const int e = sidx[p];
-    if (e < 0 || e >= N) {  // flagged by the histogram kernel; keep writes in bounds
-      sslot[p] = -1;
-      continue;
-    }
-    int rank = 0;
-    for (int q = 0; q < tl * K; ++q) rank += (sidx[q] == e) ? 1 : 0;
-    const int r = chunk_base[(size_t)c * N + e] + rank;
-    if (r < 0 || r >= T * K) {  // only when counts[] disagree with idx (flagged)
-      sslot[p] = -1;
-      continue;
-    }
-    sslot[p] = r;
-    slot[(size_t)t0 * K + p] = r;
-    perm_tok[r] = t0 + tl;
-  }
-  __syncthreads();
+  chunk_slots(idx, chunk_base, c, t0, nt, T, K, N, perm_tok, slot, sidx, sslot);
   // gather: warp per token, 16-byte vectors
   constexpr int kElems = 16 / sizeof(XT);
   const int nvec = d / kElems;
@@ -147,6 +161,43 @@ __global__ void __launch_bounds__(256) scatter_gather_kernel(
       for (int k = 0; k < K; ++k) {
         const int r = sslot[tl * K + k];
         if (r >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)r * d)[v] = val;
+      }
+    }
+  }
+}
+
+// E4M3 layer: slots as above, then each x row is quantised once per 1x128
+// tile (a half-warp per tile) and its codes and scales are written to the
+// token's K destination rows.
+__global__ void __launch_bounds__(256) scatter_gather_fp8_kernel(
+    const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ chunk_base, int T, int d, int K, int N,
+    int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot, uint8_t* __restrict__ x_perm,
+    float* __restrict__ x_perm_scales) {
+  __shared__ int sidx[kChunkTokens * kMaxK];
+  __shared__ int sslot[kChunkTokens * kMaxK];
+  const int c = blockIdx.x;
+  const int t0 = c * kChunkTokens;
+  const int nt = min(kChunkTokens, T - t0);
+  chunk_slots(idx, chunk_base, c, t0, nt, T, K, N, perm_tok, slot, sidx, sslot);
+  const int tiles = d / QB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, l16 = lane & 15;
+  for (int tl = warp; tl < nt; tl += 8) {
+    const __nv_bfloat16* src = x + (size_t)(t0 + tl) * d;
+    for (int tc0 = 0; tc0 < tiles; tc0 += 2) {  // two tiles per warp pass
+      const int tc = tc0 + half;
+      const bool live = tc < tiles;
+      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (live) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(src + tc * QB) + l16), v);
+      uint2 codes;
+      const float sc = quant_tile_16lanes(v, codes);
+      if (!live) continue;
+      for (int k = 0; k < K; ++k) {
+        const int r = sslot[tl * K + k];
+        if (r < 0) continue;
+        *reinterpret_cast<uint2*>(x_perm + (size_t)r * d + tc * QB + 8 * l16) = codes;
+        if (l16 == 0) x_perm_scales[(size_t)r * tiles + tc] = sc;
       }
     }
   }
@@ -176,8 +227,9 @@ cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* id
         static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
         slot, static_cast<__nv_bfloat16*>(x_perm));
   else
-    return cudaErrorNotSupported;
-  (void)x_perm_scales;
+    scatter_gather_fp8_kernel<<<nch, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
+        slot, static_cast<uint8_t*>(x_perm), x_perm_scales);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,563 @@
+// FP8-E4M3 expert GEMMs with fine-grained fp32 block scales.
+//
+// The FP8 recipe follows the mhpq.cn article §4.1 (精细量化策略 / 在线量化 /
+// 高精度累加): activations are scaled per 1x128 tile and weights per
+// 128x128 block, each scale taken online from the current max-abs; products
+// accumulate in fp32.  Reading taken: scale = amax/448 and inverse
+// 448/amax in fp32 (IEEE division), code = E4M3_RNE_satfinite(v * inverse),
+// a tile with amax = 0 gets scale 1 and all-zero codes.
+//
+// GEMM (one persistent launch per expert GEMM, all groups):
+//   C[row, col] = sum over 128-wide K slices kb of
+//                 sa[row, kb] * sw[col/128, kb] * sum_{k in kb} qa[row,k] qw[col,k]
+// The per-slice products come from tcgen05.mma kind::f8f6f4 (E4M3 x E4M3,
+// fp32 accumulate, M=128 tokens, N=256 weight columns, K=32 each); every
+// 128-wide slice lands in its own TMEM buffer (two 256-column buffers, so
+// the tensor core fills one while the other is drained).  Eight epilogue
+// warps -- two per TMEM lane quadrant, each owning 128 of the 256 columns --
+// fold each slice into fp32 register sums with the product of the two
+// scales.  This per-slice promotion is the tcgen05 counterpart of the
+// article's "accumulate at an interval in fp32 on the CUDA cores" (the
+// kaiyunto.com walk-through describes the same H800 step); on sm_100 the
+// partial sums already sit in TMEM in fp32, so only the scale product is
+// applied per slice.
+//
+// GEMM1 epilogue: h = silu(gate) * up for the 128 hidden features of the
+// tile (gate and up columns of one feature lie in the same tile and thread
+// row), then h is quantised per 1x128 tile along f; the two warps that share
+// a row exchange their half-tile max-abs through shared memory under an
+// mbarrier.  GEMM2 epilogue: bf16 output rows.
+// Roles: warp 0 TMA producer (4-stage ring: 128 token rows + 256 weight rows
+// of 128 bytes), warp 1 TMEM owner and MMA issuer, warps 2-9 epilogue.
+// All waits are bounded (~2 s) and set the device status word on expiry.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "fp8_util.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int FBM = 128, FBN = 256, FBK = 128;
+constexpr int FStages = 4;
+constexpr int FABytes = FBM * FBK;      // 16 KB
+constexpr int FBBytes = FBN * FBK;      // 32 KB
+constexpr int FStageBytes = FABytes + FBBytes;
+constexpr int FThreads = 320;
+constexpr int FEpiWarps = 8;
+constexpr uint64_t FTimeoutNs = 2000000000ull;
+
+enum FEpi { kFEpiSwiGLUQuant = 0, kFEpiStore = 1 };
+
+// x [rows, d] bf16 -> codes [rows, d], scales [rows, d/128]; one half-warp per tile.
+__global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ x, long long rows, int d,
+                                  uint8_t* __restrict__ q, float* __restrict__ sc) {
+  const int tiles_per_row = d / QB;
+  const long long tiles = rows * tiles_per_row;
+  const int half = (threadIdx.x >> 4) & 1, l16 = threadIdx.x & 15;
+  const long long hw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const long long hw_stride = ((long long)gridDim.x * blockDim.x) >> 4;
+  (void)half;
+  // every half-warp walks the same number of iterations so shuffles stay converged
+  const long long iters = (tiles + hw_stride - 1) / hw_stride;
+  for (long long it = 0; it < iters; ++it) {
+    const long long tile = hw + it * hw_stride;
+    const bool live = tile < tiles;
+    const long long r = live ? tile / tiles_per_row : 0;
+    const int tc = live ? (int)(tile - r * tiles_per_row) : 0;
+    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (live)
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(x + r * d + tc * QB + 8 * l16), v);
+    uint2 codes;
+    const float s = quant_tile_16lanes(v, codes);
+    if (live) {
+      *reinterpret_cast<uint2*>(q + r * d + tc * QB + 8 * l16) = codes;
+      if (l16 == 0) sc[r * tiles_per_row + tc] = s;
+    }
+  }
+}
+
+// ---- 128x128 weight quantisation ---------------------------------------------------
+// One CTA (128 threads) per block; thread t handles row t of the block.
+__global__ void __launch_bounds__(128) quant_blocks_kernel(const __nv_bfloat16* __restrict__ w,
+                                                           int cols, long long blocks_r,
+                                                           int blocks_c,
+                                                           uint8_t* __restrict__ q,
+                                                           float* __restrict__ sc) {
+  __shared__ float red[4];
+  const long long b = blockIdx.x;
+  const long long br = b / blocks_c;
+  const int bc = (int)(b - br * blocks_c);
+  const int t = threadIdx.x;
+  const __nv_bfloat16* row = w + (br * QB + t) * (long long)cols + (long long)bc * QB;
+  float amax = 0.f;
+  uint4 raw[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    raw[i] = reinterpret_cast<const uint4*>(row)[i];
+    float f[8];
+    bf16x8_to_f32(raw[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((t & 31) == 0) red[t >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const bool zero = amax == 0.f;
+  const float scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
+  const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
+  uint8_t* qrow = q + (br * QB + t) * (long long)cols + (long long)bc * QB;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float f[8];
+    bf16x8_to_f32(raw[i], f);
+    uint32_t w2[2] = {0u, 0u};
+    if (!zero) {
+#pragma unroll
+      for (int p = 0; p < 2; ++p)
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const int k = 4 * p + 2 * qq;
+          const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(
+              make_float2(__fmul_rn(f[k], inv), __fmul_rn(f[k + 1], inv)), __NV_SATFINITE,
+              __NV_E4M3);
+          w2[p] |= (uint32_t)c2 << (16 * qq);
+        }
+    }
+    reinterpret_cast<uint2*>(qrow)[i] = make_uint2(w2[0], w2[1]);
+  }
+  if (t == 0) sc[br * blocks_c + bc] = scale;
+}
+
+// ---- block-scaled FP8 grouped GEMM -------------------------------------------------
+struct alignas(64) Fp8Args {
+  CUtensorMap tmA_routed;
+  CUtensorMap tmA_shared;
+  CUtensorMap tmB;
+  const int32_t* offsets;
+  const float* sa_routed;  // [rows, KB] activation scales (row index as in tmA_routed)
+  const float* sa_shared;  // [rows, KB] (row index as in tmA_shared)
+  const float* sw;         // [(N+1) * n_acc / 128, KB] weight block scales
+  uint8_t* q_routed;       // GEMM1: h codes, row (offsets[g] + r)
+  uint8_t* q_shared;       // GEMM1: h codes, row r
+  float* qs_routed;        // GEMM1: h scales [row, out_ld/128]
+  float* qs_shared;
+  __nv_bfloat16* y_routed;  // GEMM2 outputs
+  __nv_bfloat16* y_shared;
+  uint32_t* status;
+  int N, T;
+  int rows_routed;
+  int a_shared_row0;
+  int n_acc;   // weight rows per group (2f or d)
+  int k_dim;   // contraction length
+  int out_ld;  // f (GEMM1 codes) or d (GEMM2)
+};
+
+constexpr size_t fp8_smem_bytes(int groups) {
+  return 1024 + (size_t)FStages * FStageBytes + 512 + 2 * 2 * FBM * 4 + (size_t)(groups + 1) * 4;
+}
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
+
+template <int kEpi>
+__global__ void __maxnreg__(200) grouped_gemm_fp8_kernel(
+    const __grid_constant__ Fp8Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)FStages * FStageBytes);
+  uint64_t* full = bars;                  // [FStages]
+  uint64_t* empty = bars + FStages;       // [FStages]
+  uint64_t* sfull = bars + 2 * FStages;   // [2] slice buffer written
+  uint64_t* sempty = sfull + 2;           // [2] slice buffer drained (8 warps)
+  uint64_t* xbar = sempty + 2;            // [2] amax exchange (8 warps)
+  uint64_t* drain = xbar + 2;             // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  float* xchg = reinterpret_cast<float*>(base + (size_t)FStages * FStageBytes + 512);  // [2][2][128]
+  int* tile_start = reinterpret_cast<int*>(xchg + 2 * 2 * FBM);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int G1 = args.N + 1;
+  const int NT = args.n_acc / FBN;
+  const int KB = args.k_dim / FBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < FStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sfull[a], 1);
+      mbar_init(&sempty[a], FEpiWarps);
+      mbar_init(&xbar[a], FEpiWarps);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  for (int g = tid; g < G1; g += FThreads) {
+    const int rows = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+    tile_start[g] = rows > 0 ? (rows + FBM - 1) / FBM : 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    const int per = (G1 + 31) / 32;
+    const int g0 = min(G1, lane * per), g1 = min(G1, g0 + per);
+    int sum = 0;
+    for (int g = g0; g < g1; ++g) sum += tile_start[g];
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    int run = inc - sum;
+    for (int g = g0; g < g1; ++g) {
+      const int mt = tile_start[g];
+      tile_start[g] = run * NT;
+      run += mt;
+    }
+    if (lane == 31) tile_start[G1] = inc * NT;
+  }
+  __syncthreads();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = tile_start[G1];
+
+  auto decode = [&](int tile, int& g, int& n, int& m) {
+    int lo = 0, hi = G1;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_start[mid] <= tile) lo = mid; else hi = mid;
+    }
+    g = lo;
+    const int mt = (tile_start[g + 1] - tile_start[g]) / NT;
+    const int local = tile - tile_start[g];
+    n = local / mt;
+    m = local - n * mt;
+  };
+
+  if (warp == 0) {
+    // ---- TMA producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&args.tmA_routed);
+      tma_prefetch_desc(&args.tmA_shared);
+      tma_prefetch_desc(&args.tmB);
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, n, m;
+        decode(tile, g, n, m);
+        const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
+        const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * FBM;
+        const int brow = g * args.n_acc + n * FBN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, FTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = base + (size_t)stage * FStageBytes;
+          mbar_arrive_expect_tx(&full[stage], FStageBytes);
+          tma_load_2d(sa, am, kb * FBK, arow, &full[stage]);
+          tma_load_2d(sa + FABytes, &args.tmB, kb * FBK, brow, &full[stage]);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == FStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < FStages; ++s)
+          if ((issued >> s) & 1u)
+            mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.status, FTimeoutNs / 8);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer: one TMEM slice buffer per 128-wide K slice ----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_e4m3_f32(FBM, FBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t slice = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < KB; ++kb, ++slice) {
+          const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
+          if (!mbar_wait_bounded(&sempty[sb], sph ^ 1u, args.status, FTimeoutNs) ||
+              !mbar_wait_bounded(&full[stage], phase, args.status, FTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(base + (size_t)stage * FStageBytes);
+          const uint32_t b0 = a0 + FABytes;
+#pragma unroll
+          for (int k = 0; k < FBK / 32; ++k)
+            mma_e4m3(tmem_base + sb * FBN, smem_desc_sw128(a0 + k * 32),
+                     smem_desc_sw128(b0 + k * 32), idesc, k != 0);
+          mma_commit(&empty[stage]);
+          mma_commit(&sfull[sb]);
+          if (++stage == FStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0, args.status, FTimeoutNs / 8);
+    }
+  } else {
+    // ---- epilogue: warps 2..9 ----
+    const int q = warp & 3;             // TMEM lane quadrant
+    const int half = (warp - 2) >> 2;   // which 128 of the 256 columns
+    const int row = q * 32 + lane;      // token row within the tile
+    const int ewarp = warp - 2;
+    uint32_t slice = 0;
+    int local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+      int g, n, m;
+      decode(tile, g, n, m);
+      const int rows_g = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+      const int r = m * FBM + row;
+      const bool valid =
+          r < rows_g && (g == args.N || args.offsets[g] + r < args.rows_routed);
+      const long long arow_idx =
+          (g < args.N) ? (long long)args.offsets[g] + r : (long long)args.a_shared_row0 + r;
+      const float* sa_row = ((g < args.N) ? args.sa_routed : args.sa_shared) +
+                            (valid ? arow_idx : 0) * KB;
+      const long long wblk0 = ((long long)g * args.n_acc + (long long)n * FBN) / QB;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int kb = 0; kb < KB; ++kb, ++slice) {
+        const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
+        const float sa = valid ? __ldg(sa_row + kb) : 0.f;
+        const float sw0 = __ldg(args.sw + wblk0 * KB + kb);
+        const float sw1 = __ldg(args.sw + (wblk0 + 1) * KB + kb);
+        if (!mbar_wait_bounded(&sfull[sb], sph, args.status, FTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * FBN;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          int col;
+          float s;
+          if constexpr (kEpi == kFEpiSwiGLUQuant) {
+            // gate columns (W1 block) then up columns (W3 block) of features 64*half..
+            col = (c < 2) ? 64 * half + 32 * c : 128 + 64 * half + 32 * (c - 2);
+            s = sa * ((c < 2) ? sw0 : sw1);
+          } else {
+            col = 128 * half + 32 * c;
+            s = sa * (half ? sw1 : sw0);
+          }
+          uint32_t p[32];
+          tmem_ld32(taddr + col, p);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(__uint_as_float(p[i]), s, acc[c * 32 + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[sb]);
+      }
+      if (!ok) break;
+
+      if constexpr (kEpi == kFEpiSwiGLUQuant) {
+        // h for hidden features n*128 + 64*half + i, i < 64
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          acc[i] = silu_f(acc[i]) * acc[64 + i];
+          amax = fmaxf(amax, fabsf(acc[i]));
+        }
+        // exchange the half-tile max-abs with the warp holding the other 64 features
+        float* xb = xchg + (local & 1) * 2 * FBM;
+        xb[half * FBM + row] = amax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[local & 1]);
+        if (!mbar_wait_bounded(&xbar[local & 1], (local >> 1) & 1, args.status, FTimeoutNs)) break;
+        amax = fmaxf(xb[row], xb[FBM + row]);
+        const bool zero = amax == 0.f;
+        const float scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
+        const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
+        if (valid) {
+          uint8_t* qrow = ((g < args.N) ? args.q_routed + (long long)args.offsets[g] * args.out_ld
+                                        : args.q_shared) +
+                          (long long)r * args.out_ld + n * QB + 64 * half;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              uint32_t word = 0;
+#pragma unroll
+              for (int qq = 0; qq < 2; ++qq) {
+                const int i = 16 * v + 4 * wd + 2 * qq;
+                const __nv_fp8x2_storage_t c2 =
+                    zero ? (__nv_fp8x2_storage_t)0
+                         : __nv_cvt_float2_to_fp8x2(
+                               make_float2(__fmul_rn(acc[i], inv), __fmul_rn(acc[i + 1], inv)),
+                               __NV_SATFINITE, __NV_E4M3);
+                word |= (uint32_t)c2 << (16 * qq);
+              }
+              w4[wd] = word;
+            }
+            reinterpret_cast<uint4*>(qrow)[v] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+          if (half == 0) {
+            float* srow = (g < args.N) ? args.qs_routed + ((long long)args.offsets[g] + r) *
+                                                            (args.out_ld / QB)
+                                       : args.qs_shared + (long long)r * (args.out_ld / QB);
+            srow[n] = scale;
+          }
+        }
+      } else {
+        if (valid) {
+          __nv_bfloat16* yrow =
+              ((g < args.N) ? args.y_routed + ((long long)args.offsets[g] + r) * args.out_ld
+                            : args.y_shared + (long long)r * args.out_ld) +
+              n * FBN + 128 * half;
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            uint4 w;
+            __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              hb[i] = __floats2bfloat162_rn(acc[8 * v + 2 * i], acc[8 * v + 2 * i + 1]);
+            reinterpret_cast<uint4*>(yrow)[v] = w;
+          }
+        }
+      }
+      (void)ewarp;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int kEpi>
+cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
+  const size_t smem = fp8_smem_bytes(a.N + 1);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kEpi>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_fp8_kernel<kEpi><<<num_sms(), FThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
+                              cudaStream_t st) {
+  const long long tiles = rows * (d / QB);
+  long long blocks = (tiles * 16 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  quant_rows_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rows, d,
+                                                 q, sc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const void* w2,
+                                    void* w13_q, float* w13_scales, void* w2_q,
+                                    float* w2_scales, cudaStream_t st) {
+  const long long E = s.N + 1;
+  // w13 [E * 2f, d]: blocks of 128 rows x 128 columns
+  const long long br13 = E * 2 * s.f / QB;
+  const int bc13 = s.d / QB;
+  quant_blocks_kernel<<<(unsigned)(br13 * bc13), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w13), s.d, br13, bc13, static_cast<uint8_t*>(w13_q),
+      w13_scales);
+  const long long br2 = E * s.d / QB;
+  const int bc2 = s.f / QB;
+  quant_blocks_kernel<<<(unsigned)(br2 * bc2), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w2), s.f, br2, bc2, static_cast<uint8_t*>(w2_q),
+      w2_scales);
+  return cudaGetLastError();
+}
+
+int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_perm_scales,
+                       const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                       const float* w13_scales, const float* w2_scales, void* y_perm,
+                       void* y_shared, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint8_t* Hq = w + L.h;
+  float* Hs = reinterpret_cast<float*>(w + L.h_scales);
+  uint8_t* xq = w + L.xq;
+  float* xs = reinterpret_cast<float*>(w + L.xq_scales);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
+  const uint64_t TK = (uint64_t)s.T * s.K;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+
+  // the shared expert reads x: quantise it per 1x128 tile first
+  if (launch_quant_rows(x, s.T, s.d, xq, xs, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  Fp8Args g1{};
+  bool ok = make_map(&g1.tmA_routed, x_perm, U8, 1, s.d, TK, FBK, FBM) &&
+            make_map(&g1.tmA_shared, xq, U8, 1, s.d, s.T, FBK, FBM) &&
+            make_map(&g1.tmB, w13, U8, 1, s.d, (uint64_t)(s.N + 1) * 2 * s.f, FBK, FBN);
+  if (!ok) return MOE_ERR_CUDA;
+  g1.offsets = offsets;
+  g1.sa_routed = x_perm_scales;
+  g1.sa_shared = xs;
+  g1.sw = w13_scales;
+  g1.q_routed = Hq;
+  g1.q_shared = Hq + TK * s.f;
+  g1.qs_routed = Hs;
+  g1.qs_shared = Hs + TK * (s.f / QB);
+  g1.status = status;
+  g1.N = s.N;
+  g1.T = s.T;
+  g1.rows_routed = (int)TK;
+  g1.a_shared_row0 = 0;
+  g1.n_acc = 2 * s.f;
+  g1.k_dim = s.d;
+  g1.out_ld = s.f;
+  if (launch_fp8_gemm<kFEpiSwiGLUQuant>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  Fp8Args g2{};
+  ok = make_map(&g2.tmA_routed, Hq, U8, 1, s.f, TK + s.T, FBK, FBM) &&
+       make_map(&g2.tmA_shared, Hq, U8, 1, s.f, TK + s.T, FBK, FBM) &&
+       make_map(&g2.tmB, w2, U8, 1, s.f, (uint64_t)(s.N + 1) * s.d, FBK, FBN);
+  if (!ok) return MOE_ERR_CUDA;
+  g2.offsets = offsets;
+  g2.sa_routed = Hs;
+  g2.sa_shared = Hs;
+  g2.sw = w2_scales;
+  g2.y_routed = static_cast<__nv_bfloat16*>(y_perm);
+  g2.y_shared = static_cast<__nv_bfloat16*>(y_shared);
+  g2.status = status;
+  g2.N = s.N;
+  g2.T = s.T;
+  g2.rows_routed = (int)TK;
+  g2.a_shared_row0 = (int)TK;
+  g2.n_acc = s.d;
+  g2.k_dim = s.f;
+  g2.out_ld = s.d;
+  if (launch_fp8_gemm<kFEpiStore>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/moe_b200.h"
@@ -38,6 +39,13 @@ inline size_t io_bytes(int dtype) { return dtype == MOE_DTYPE_FP32 ? 4 : 2; }
 // Rows of a W1/W3 block in the packed w13 layout.
 inline int pack_block(int f) { return f < 128 ? f : 128; }
 
+// ---- host helpers (tma_host.cu) ------------------------------------------------
+// 2-D row-major tensor [rows, inner] with a (box_inner x box_rows) box and the
+// 128-byte swizzle; out-of-range rows read as zero.
+bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t elem_bytes,
+              uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows);
+int num_sms();
+
 // ---- launchers (return cudaError_t of the launch) -----------------------------
 int launch_route(const moe_shape& s, const void* x, const float* router, const float* bias,
                  int32_t* idx, float* gate, int32_t* counts, void* ws, cudaStream_t st);
@@ -67,6 +75,9 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
                        const int32_t* offsets, const void* x, const void* w13, const void* w2,
                        const float* w13_scales, const float* w2_scales, void* y_perm,
                        void* y_shared, void* ws, cudaStream_t st);
+// x [rows, d] bf16 -> E4M3 codes [rows, d] and fp32 scales [rows, d/128].
+cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
+                              cudaStream_t st);
 cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const void* w2,
                                     void* w13_q, float* w13_scales, void* w2_q,
                                     float* w2_scales, cudaStream_t st);

@@ -62,24 +62,30 @@ __device__ __forceinline__ void top2_merge(float& a1, float& a2, float b1, float
 // s[j] (un-biased sigmoid scores) and bj[j] (their biases).  Writes the K
 // chosen experts in ascending id order with their gates, and counts them in
 // the shared-memory histogram.
+// Group of each expert a lane holds (expert lane + 32 j; -1 past N).
+__device__ __forceinline__ void lane_groups(int lane, int N, int G, int (&grp)[kEPL]) {
+  const int gs = N / G;
+#pragma unroll
+  for (int j = 0; j < kEPL; ++j) grp[j] = (lane + 32 * j < N) ? (lane + 32 * j) / gs : -1;
+}
+
 __device__ __forceinline__ void select_token(const float (&s)[kEPL], const float (&bj)[kEPL],
-                                             int lane, int t, int N, int K, int G, int topG,
+                                             const int (&grp)[kEPL], int lane, int t, int N,
+                                             int K, int G, int topG,
                                              int32_t* __restrict__ topk_idx,
                                              float* __restrict__ topk_gate, int* hist,
                                              uint32_t* status) {
   const int gs = N / G;
   float sb[kEPL];
 #pragma unroll
-  for (int j = 0; j < kEPL; ++j) sb[j] = (lane + 32 * j < N) ? s[j] + bj[j] : -INFINITY;
+  for (int j = 0; j < kEPL; ++j) sb[j] = (grp[j] >= 0) ? s[j] + bj[j] : -INFINITY;
   // group scores: lane g ends up holding group g's score
   float my_gscore = -INFINITY;
   for (int g = 0; g < G; ++g) {
     float m1 = -INFINITY, m2 = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kEPL; ++j) {
-      const int e = lane + 32 * j;
-      if (e < N && e / gs == g) top2_merge(m1, m2, sb[j], -INFINITY);
-    }
+    for (int j = 0; j < kEPL; ++j)
+      if (grp[j] == g) top2_merge(m1, m2, sb[j], -INFINITY);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float b1 = __shfl_xor_sync(0xffffffffu, m1, o);
@@ -107,7 +113,7 @@ __device__ __forceinline__ void select_token(const float (&s)[kEPL], const float
 #pragma unroll
     for (int j = 0; j < kEPL; ++j) {
       const int e = lane + 32 * j;
-      if (e < N && ((kept >> (e / gs)) & 1u) && !((taken >> j) & 1u) &&
+      if (grp[j] >= 0 && ((kept >> grp[j]) & 1u) && !((taken >> j) & 1u) &&
           better(sb[j], e, v, ei)) {
         v = sb[j];
         ei = e;
@@ -204,6 +210,8 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
 
   // ---- phase 2: selection, one token at a time per warp ----
   float bj[kEPL];
+  int grp[kEPL];
+  lane_groups(lane, N, G, grp);
 #pragma unroll
   for (int j = 0; j < kEPL; ++j) bj[j] = (lane + 32 * j < N) ? bias[lane + 32 * j] : 0.f;
 #pragma unroll
@@ -213,7 +221,7 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
     float s[kEPL];
 #pragma unroll
     for (int j = 0; j < kEPL; ++j) s[j] = 1.f / (1.f + expf(-acc[i][j]));
-    select_token(s, bj, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
+    select_token(s, bj, grp, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
   }
   __syncthreads();
   for (int e = tid; e < N; e += blockDim.x)
@@ -221,8 +229,10 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
 }
 
 // Selection from the tensor-core logits Z [splits, T, N]: z is the sum of
-// the split partials in split order, s = sigmoid(z); warp per token, 32
-// tokens per CTA.
+// the split partials in split order, s = sigmoid(z); one warp per token,
+// 8 tokens per CTA.
+constexpr int kSelTokens = 8;
+
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z, int splits,
                                                      const float* __restrict__ bias, int T, int N,
                                                      int K, int G, int topG,
@@ -235,24 +245,24 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z
   const int warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < N; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  float bj[kEPL];
-#pragma unroll
-  for (int j = 0; j < kEPL; ++j) bj[j] = (lane + 32 * j < N) ? bias[lane + 32 * j] : 0.f;
-  for (int i = 0; i < 4; ++i) {
-    const int t = blockIdx.x * kBT + warp * 4 + i;
-    if (t >= T) break;
-    float s[kEPL];
+  const int t = blockIdx.x * kSelTokens + warp;
+  if (t < T) {
+    float bj[kEPL], s[kEPL];
+    int grp[kEPL];
+    lane_groups(lane, N, G, grp);
 #pragma unroll
     for (int j = 0; j < kEPL; ++j) {
       float z = 0.f;
-      if (lane + 32 * j < N) {
+      bj[j] = 0.f;
+      if (grp[j] >= 0) {
+        bj[j] = __ldg(bias + lane + 32 * j);
         z = __ldg(Z + (size_t)t * N + lane + 32 * j);
         for (int p = 1; p < splits; ++p)
           z = __fadd_rn(z, __ldg(Z + ((size_t)p * T + t) * N + lane + 32 * j));
       }
       s[j] = 1.f / (1.f + expf(-z));
     }
-    select_token(s, bj, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
+    select_token(s, bj, grp, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
   }
   __syncthreads();
   for (int e = tid; e < N; e += blockDim.x)
@@ -277,8 +287,8 @@ int launch_route(const moe_shape& s, const void* x, const float* router, const f
     const int splits = router_k_splits(s);
     const int rc = launch_router_scores_tc(s, x, router, Z, splits, ws, st);
     if (rc != MOE_OK) return rc;
-    select_kernel<<<grid, 256, 0, st>>>(Z, splits, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate,
-                                        counts, status);
+    select_kernel<<<(s.T + kSelTokens - 1) / kSelTokens, 256, 0, st>>>(
+        Z, splits, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate, counts, status);
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -104,3 +104,32 @@ def test_decode_zipf_200_steps(M):
     # most 0.2 in score units over 200 steps
     print("max/mean load: first", loads[0], "last", loads[-1])
     del torch
+
+
+def test_v3_fp8_routing_and_sampled_outputs(M):
+    """The V3 layer with E4M3 expert GEMMs at T=16384: routing bit-exact for all
+    tokens, dispatched-row quantisation bit-exact on sampled rows, outputs of
+    sampled tokens within rel-Frobenius 2e-2 of the oracle's FP8 emulation."""
+    import torch
+    cfg = CONFIGS[3]
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    W = S.device_weights(cfg)
+    layer = _layer(M, cfg, R, b, W)
+    x, _ = S.tie_free_x(cfg, R, b)
+    y = layer.forward(S.to_dev_x(x, cfg))
+    r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
+    np.testing.assert_array_equal(layer.topk_idx.cpu().numpy(), r["idx"])
+    np.testing.assert_array_equal(layer.counts.cpu().numpy(), r["counts"])
+    d = oracle.dispatch(r["idx"], cfg.N)
+    np.testing.assert_array_equal(layer.perm_tok.cpu().numpy(), d["perm_tok"])
+    rows = np.random.default_rng(1).choice(cfg.T * cfg.K, 512, replace=False)
+    codes, scales = oracle.quant_rows_1x128(x[d["perm_tok"][rows]])
+    np.testing.assert_array_equal(layer.x_perm.view(torch.uint8)[rows].cpu().numpy(), codes)
+    np.testing.assert_array_equal(layer.x_perm_scales[rows].cpu().numpy(), scales)
+    tail = [int(d["perm_tok"][d["offsets"][e + 1] - 1]) for e in (5, 131)]
+    tokens, _ = S.greedy_token_sample(r["idx"], 6, must=tail + [cfg.T - 1])
+    ref = oracle.moe_forward(x, R, b, S.streaming_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             tokens=tokens, expert_fn=oracle.fp8_swiglu_expert)
+    err = S.rel_fro(y.float().cpu().numpy()[tokens], ref["y"])
+    assert err <= 2e-2, err
+    assert layer.device_status() == 0

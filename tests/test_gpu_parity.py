@@ -176,3 +176,68 @@ def test_mid_bf16_layer_sampled(M):
     assert err <= TOL["bf16"], err
     assert layer.device_status() == 0
     del torch
+
+
+# ---------------------------------------------------------------------------
+# FP8-E4M3 layer
+# ---------------------------------------------------------------------------
+
+def _small_fp8(T=1000):
+    return CONFIGS[3].with_(T=T, d=256, N=8, K=2, G=2, topG=1, f=256)
+
+
+def test_fp8_weight_quantisation_bitexact(M):
+    """Per-128x128-block E4M3 codes and fp32 scales of the packed W1/W3 and W2
+    equal the oracle's quantisation of the same bf16 weights."""
+    cfg = CONFIGS[3].with_(N=16)
+    W = S.device_weights(cfg)
+    q13 = W["w13"].view(__import__("torch").uint8).cpu().numpy()
+    s13 = W["w13_scales"].cpu().numpy()
+    q2 = W["w2"].view(__import__("torch").uint8).cpu().numpy()
+    s2 = W["w2_scales"].cpu().numpy()
+    get = S.host_weights(cfg)
+    for e in (0, cfg.N):
+        w1, w3, w2 = get(e)
+        c1, sc1 = oracle.quant_blocks_128(w1)
+        c3, sc3 = oracle.quant_blocks_128(w3)
+        c2, sc2 = oracle.quant_blocks_128(w2)
+        for j in range(cfg.f // 128):          # packed: W1 block j, then W3 block j
+            np.testing.assert_array_equal(q13[e, 256 * j:256 * j + 128], c1[128 * j:128 * j + 128])
+            np.testing.assert_array_equal(q13[e, 256 * j + 128:256 * j + 256],
+                                          c3[128 * j:128 * j + 128])
+            np.testing.assert_array_equal(s13[e, 2 * j], sc1[j])
+            np.testing.assert_array_equal(s13[e, 2 * j + 1], sc3[j])
+        np.testing.assert_array_equal(q2[e], c2)
+        np.testing.assert_array_equal(s2[e], sc2)
+
+
+@pytest.mark.parametrize("T", [1000, 1])
+def test_small_fp8_layer_full(M, T):
+    torch = _torch()
+    cfg = _small_fp8(T)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).float().cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             expert_fn=oracle.fp8_swiglu_expert)
+    r = ref["route"]
+    _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
+                 layer.counts.cpu().numpy())
+    d = _check_dispatch(layer, r)
+    # dispatched rows are quantised per 1x128 tile exactly as the oracle does
+    codes, scales = oracle.quant_rows_1x128(x[d["perm_tok"]])
+    np.testing.assert_array_equal(layer.x_perm.view(torch.uint8).cpu().numpy(), codes)
+    np.testing.assert_array_equal(layer.x_perm_scales.cpu().numpy(), scales)
+    get = S.host_weights(cfg)
+    yp = layer.y_perm.float().cpu().numpy()
+    for e in range(cfg.N):
+        a, z = d["offsets"][e], d["offsets"][e + 1]
+        if z == a:
+            continue
+        want = oracle.fp8_swiglu_expert(x[d["perm_tok"][a:z]], *get(e))
+        assert S.rel_fro(yp[a:z], want) <= TOL["e4m3"], e
+    err = S.rel_fro(y, ref["y"])
+    assert err <= TOL["e4m3"], err
+    assert layer.device_status() == 0
