@@ -94,6 +94,11 @@ enum {
 /* Human-readable text for a MOE_* status.  Never NULL; static storage. */
 const char* moe_status_string(int status);
 
+/* Text of the last CUDA failure recorded on this thread (the failing call and
+ * CUDA's message), "" if none; explains a MOE_ERR_CUDA status.  Static,
+ * thread-local storage, overwritten by the next failure. */
+const char* moe_last_error(void);
+
 /* Check a shape: MOE_OK, MOE_ERR_ARG or MOE_ERR_UNSUPPORTED.
  * Supported: T >= 1; 1 <= K <= min(32, topG*N/G); N <= 256; G divides N;
  * 1 <= topG <= G; for BF16 and E4M3 also d % 256 == 0 and f % 128 == 0;

@@ -31,13 +31,16 @@ class MoEShape(ctypes.Structure):
 
 class MoEError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        detail = lib().moe_last_error().decode() if status == ERR_CUDA else ""
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})"
+                         + (f": {detail}" if detail else ""))
         self.status = status
 
 
 _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_check_shape": (ctypes.c_int, [ctypes.POINTER(MoEShape)]),
+    "moe_last_error": (ctypes.c_char_p, []),
     "moe_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
     "moe_workspace_init": (ctypes.c_int, [_c_p, _c_p]),
     "moe_read_device_status": (ctypes.c_int, [_c_p, _c_p, ctypes.POINTER(ctypes.c_uint32),

@@ -72,7 +72,10 @@ int ws_check(const moe_shape* s, void* ws) {
   return MOE_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+int cuda_status(cudaError_t e) {
+  note_cuda(e, "kernel launch");
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
 
 }  // namespace

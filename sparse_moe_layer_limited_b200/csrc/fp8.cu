@@ -165,7 +165,7 @@ constexpr size_t fp8_smem_bytes(int groups) {
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
 template <int kEpi>
-__global__ void __maxnreg__(200) grouped_gemm_fp8_kernel(
+__global__ void __maxnreg__(192) grouped_gemm_fp8_kernel(
     const __grid_constant__ Fp8Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -459,11 +459,13 @@ __global__ void __maxnreg__(200) grouped_gemm_fp8_kernel(
 template <int kEpi>
 cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
   const size_t smem = fp8_smem_bytes(a.N + 1);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kEpi>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kEpi>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem),
+                            "fp8 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
   grouped_gemm_fp8_kernel<kEpi><<<num_sms(), FThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return note_cuda(cudaGetLastError(), "fp8 GEMM launch");
 }
 
 }  // namespace
@@ -476,7 +478,7 @@ cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, 
   if (blocks < 1) blocks = 1;
   quant_rows_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rows, d,
                                                  q, sc);
-  return cudaGetLastError();
+  return note_cuda(cudaGetLastError(), "1x128 quantisation launch");
 }
 
 cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const void* w2,
@@ -518,7 +520,10 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
   bool ok = make_map(&g1.tmA_routed, x_perm, U8, 1, s.d, TK, FBK, FBM) &&
             make_map(&g1.tmA_shared, xq, U8, 1, s.d, s.T, FBK, FBM) &&
             make_map(&g1.tmB, w13, U8, 1, s.d, (uint64_t)(s.N + 1) * 2 * s.f, FBK, FBN);
-  if (!ok) return MOE_ERR_CUDA;
+  if (!ok) {
+    note_text("fp8 GEMM1: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
   g1.offsets = offsets;
   g1.sa_routed = x_perm_scales;
   g1.sa_shared = xs;
@@ -541,7 +546,10 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
   ok = make_map(&g2.tmA_routed, Hq, U8, 1, s.f, TK + s.T, FBK, FBM) &&
        make_map(&g2.tmA_shared, Hq, U8, 1, s.f, TK + s.T, FBK, FBM) &&
        make_map(&g2.tmB, w2, U8, 1, s.f, (uint64_t)(s.N + 1) * s.d, FBK, FBN);
-  if (!ok) return MOE_ERR_CUDA;
+  if (!ok) {
+    note_text("fp8 GEMM2: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
   g2.offsets = offsets;
   g2.sa_routed = Hs;
   g2.sa_shared = Hs;

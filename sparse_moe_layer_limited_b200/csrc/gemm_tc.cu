@@ -356,11 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
 template <int kEpi, int kBN>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
   const size_t smem = TileCfg<kBN>::smem_bytes(a.N + 1);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem),
+                            "bf16 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
   grouped_gemm_bf16_kernel<kEpi, kBN><<<num_sms(), kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return note_cuda(cudaGetLastError(), "bf16 GEMM launch");
 }
 
 // R fp32 [N, d] -> three exact bf16 parts laid out [N, 3d] as described at
@@ -401,7 +403,10 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   bool ok = make_map(&g1.tmA_routed, x_perm, BF, 2, s.d, TK, BK, BM) &&
             make_map(&g1.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
             make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, 256);
-  if (!ok) return MOE_ERR_CUDA;
+  if (!ok) {
+    note_text("bf16 GEMM: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
   g1.offsets = offsets;
   g1.out_routed = H;
   g1.out_shared = H + TK * s.f;
@@ -421,7 +426,10 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   ok = make_map(&g2.tmA_routed, H, BF, 2, s.f, TK + s.T, BK, BM) &&
        make_map(&g2.tmA_shared, H, BF, 2, s.f, TK + s.T, BK, BM) &&
        make_map(&g2.tmB, w2, BF, 2, s.f, (uint64_t)(s.N + 1) * s.d, BK, 256);
-  if (!ok) return MOE_ERR_CUDA;
+  if (!ok) {
+    note_text("bf16 GEMM: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
   g2.offsets = offsets;
   g2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   g2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
@@ -465,7 +473,10 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
   bool ok = make_map(&a.tmA_routed, x, BF, 2, s.d, s.T, BK, BM) &&
             make_map(&a.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
             make_map(&a.tmB, Rs, BF, 2, 3ull * s.d, s.N, BK, bn);
-  if (!ok) return MOE_ERR_CUDA;
+  if (!ok) {
+    note_text("bf16 GEMM: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
   a.offsets = nullptr;
   a.out_f32 = Z;
   a.status = reinterpret_cast<uint32_t*>(w + L.status);

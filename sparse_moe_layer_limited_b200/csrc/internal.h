@@ -39,6 +39,11 @@ inline size_t io_bytes(int dtype) { return dtype == MOE_DTYPE_FP32 ? 4 : 2; }
 // Rows of a W1/W3 block in the packed w13 layout.
 inline int pack_block(int f) { return f < 128 ? f : 128; }
 
+// ---- error text (errors.cu) ------------------------------------------------------
+// Record `e` (if not cudaSuccess) with the failing call's name; returns e.
+cudaError_t note_cuda(cudaError_t e, const char* where);
+void note_text(const char* what);
+
 // ---- host helpers (tma_host.cu) ------------------------------------------------
 // 2-D row-major tensor [rows, inner] with a (box_inner x box_rows) box and the
 // 128-byte swizzle; out-of-range rows read as zero.
