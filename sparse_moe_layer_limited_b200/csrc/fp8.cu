@@ -29,6 +29,9 @@
 // mbarrier.  GEMM2 epilogue: bf16 output rows.
 // Roles: warp 0 TMA producer (4-stage ring: 128 token rows + 256 weight rows
 // of 128 bytes), warp 1 TMEM owner and MMA issuer, warps 2-9 epilogue.
+// Ten warps put three on some of the SM's four 16K-register banks, which caps
+// a thread at 168 registers: the epilogue keeps its 128 running sums and
+// drains TMEM 16 columns at a time.
 // All waits are bounded (~2 s) and set the device status word on expiry.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -165,7 +168,7 @@ constexpr size_t fp8_smem_bytes(int groups) {
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
 template <int kEpi>
-__global__ void __maxnreg__(192) grouped_gemm_fp8_kernel(
+__global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
     const __grid_constant__ Fp8Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -354,23 +357,26 @@ __global__ void __maxnreg__(192) grouped_gemm_fp8_kernel(
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * FBN;
+        // 16 columns per TMEM load keeps 128 sums + 16 loads within the
+        // register budget of a 10-warp CTA (3 warps share a 16K-register bank)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           int col;
           float s;
           if constexpr (kEpi == kFEpiSwiGLUQuant) {
             // gate columns (W1 block) then up columns (W3 block) of features 64*half..
-            col = (c < 2) ? 64 * half + 32 * c : 128 + 64 * half + 32 * (c - 2);
-            s = sa * ((c < 2) ? sw0 : sw1);
+            col = (c < 4) ? 64 * half + 16 * c : 128 + 64 * half + 16 * (c - 4);
+            s = sa * ((c < 4) ? sw0 : sw1);
           } else {
-            col = 128 * half + 32 * c;
+            col = 128 * half + 16 * c;
             s = sa * (half ? sw1 : sw0);
           }
-          uint32_t p[32];
-          tmem_ld32(taddr + col, p);
+          uint32_t p[16];
+          tmem_ld16(taddr + col, p);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(__uint_as_float(p[i]), s, acc[c * 32 + i]);
+          for (int i = 0; i < 16; ++i)
+            acc[c * 16 + i] = fmaf(__uint_as_float(p[i]), s, acc[c * 16 + i]);
         }
         tc_fence_before();
         __syncwarp();
