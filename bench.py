@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--cpu-sample", type=int, default=2, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the FP8 and decode workloads reported beside the headline")
     p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
     p.add_argument("--N", type=int, default=None, help="override routed experts (profiling)")
     return p.parse_args()
@@ -172,7 +174,9 @@ def dist_setup(args):
     if world > 1:
         import torch.distributed as dist
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        import torch
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
         pg = dist
     return world, rank, local, pg
 
@@ -218,26 +222,96 @@ def main():
         return run_reference(args, cfg)
 
     import torch
-    import sparse_moe_layer_limited_b200 as M
-    from synth import device as sdev
 
     world, rank, local, pg = dist_setup(args)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    s = M.shape(cfg.T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f,
-                {"fp32": M.DTYPE_FP32, "bf16": M.DTYPE_BF16, "e4m3": M.DTYPE_E4M3}[cfg.dtype])
 
-    # ---- inputs resident in HBM (weights generated on the device) ----
+    main_res = run_layer(cfg, dev, args.steps, max(3, args.warmup), pg, local, e2e=True)
+    extra = {}
+    if not args.no_extra and not (args.T or args.N):
+        # the FP8 layer and the decode workload, reported beside the bf16 headline
+        extra["fp8"] = run_layer(BY_NAME["v3_fp8"], dev, max(5, args.steps // 5), 3, pg, local)
+        extra["decode"] = run_layer(BY_NAME["decode_zipf"], dev, max(20, args.steps), 3, pg,
+                                    local)
+
+    if rank == 0:
+        P = peaks()
+        r = main_res
+        ms_step = r["total_ms"] / args.steps
+        value = world * cfg.T * args.steps / (r["total_ms"] / 1e3)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
+            "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
+                       "l2": "inputs larger than L2: the expert weights "
+                             f"({(cfg.N + 1) * 3 * cfg.d * cfg.f * 2 / 1e9:.1f} GB) stream "
+                             "through it every step",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": r["roofline"],
+            "layer_roofline": r["layer_roofline"],
+            "phases_ms": r["phases_ms"],
+            "e2e": {"value": world * cfg.T * args.steps / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": cfg.T * cfg.d * 2,
+                    "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+            "gpu_launches": r["launches_per_step"] * args.steps,
+            "clocks": r["clocks"],
+            "device_status": r["status"],
+            "load_max_over_mean": r["load_max_over_mean"],
+        }
+        for k, v in extra.items():
+            line[k] = {"workload": workload_name(v["cfg"]),
+                       "value": world * v["cfg"].T * v["steps"] / (v["total_ms"] / 1e3),
+                       "unit": "tokens/s", "ms_per_step": v["total_ms"] / v["steps"],
+                       "steps": v["steps"], "roofline": v["roofline"],
+                       "layer_roofline": v["layer_roofline"], "phases_ms": v["phases_ms"],
+                       "clocks": v["clocks"], "device_status": v["status"],
+                       "load_max_over_mean": v["load_max_over_mean"]}
+        if world == 1 and not args.no_cpu_baseline:
+            v, cores, note = cpu_oracle_baseline(cfg, args.cpu_sample)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
+                                    "kind": "oracle", "sample": note}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
+    """Build one layer of `cfg` on `dev` (weights generated on the device), run
+    `warmup` untimed steps and `steps` timed steps, each a full forward plus
+    the bias update, with CUDA events around every entry point."""
+    import torch
+    import sparse_moe_layer_limited_b200 as M
+    from synth import device as sdev
+
+    dt = {"fp32": M.DTYPE_FP32, "bf16": M.DTYPE_BF16, "e4m3": M.DTYPE_E4M3}[cfg.dtype]
+    s = M.shape(cfg.T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f, dt)
     w1 = sdev.expert_weights_bf16(cfg, 0, "w1", dev)
     w3 = sdev.expert_weights_bf16(cfg, 0, "w3", dev)
     w13 = torch.empty(cfg.N + 1, 2 * cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
     M.moe_pack_w13(s, w1, w3, w13)
     del w1, w3
     w2 = sdev.expert_weights_bf16(cfg, 0, "w2", dev)
+    s13 = s2 = None
+    if cfg.dtype == "e4m3":
+        w13q = torch.empty(w13.shape, dtype=torch.float8_e4m3fn, device=dev)
+        w2q = torch.empty(w2.shape, dtype=torch.float8_e4m3fn, device=dev)
+        s13 = torch.empty(cfg.N + 1, 2 * cfg.f // 128, cfg.d // 128, dtype=torch.float32,
+                          device=dev)
+        s2 = torch.empty(cfg.N + 1, cfg.d // 128, cfg.f // 128, dtype=torch.float32, device=dev)
+        M.moe_quantize_weights(s, w13, w2, w13q, s13, w2q, s2)
+        torch.cuda.synchronize()
+        del w13, w2
+        w13, w2 = w13q, w2q
     router = torch.from_numpy(gen.make_router(cfg)).to(dev)
     bias = torch.from_numpy(gen.make_bias(cfg)).to(dev)
-    x = sdev.x_bf16(cfg, 0, 0, dev)
-    layer = M.MoELayer(s, router, bias, w13, w2, gamma=cfg.gamma)
+    if cfg.zipf_s is None:
+        x = sdev.x_bf16(cfg, 0, 0, dev)
+    else:
+        x = torch.from_numpy(gen.make_x(cfg)).to(torch.bfloat16).to(dev)
+    layer = M.MoELayer(s, router, bias, w13, w2, s13, s2, gamma=cfg.gamma)
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream(dev)
@@ -255,7 +329,7 @@ def main():
         if ev is not None:
             ev[2].record(stream)
         M.moe_expert_ffn(s, layer.x_perm, layer.x_perm_scales, layer.offsets, x, w13, w2,
-                         None, None, layer.y_perm, layer.y_shared, layer.ws, stream)
+                         s13, s2, layer.y_perm, layer.y_shared, layer.ws, stream)
         if ev is not None:
             ev[3].record(stream)
         M.moe_combine(s, layer.y_perm, layer.y_shared, layer.slot, layer.topk_gate, layer.y,
@@ -266,91 +340,86 @@ def main():
         if ev is not None:
             ev[5].record(stream)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
     if pg is not None:
         pg.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for k in range(args.steps):
+        for k in range(steps):
             step(evs[k])
         torch.cuda.synchronize()
     if pg is not None:
         pg.barrier()
-    per_phase = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]
+    per_phase = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps)]
                  for i, p in enumerate(phases)}
     total_ms = evs[0][0].elapsed_time(evs[-1][5])
     counts = layer.counts.cpu().numpy()
     status = layer.device_status()
 
-    # ---- end to end through the public API with host buffers ----
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
-    x_dev2 = torch.empty_like(x)
-    for _ in range(2):
-        x_dev2.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev2, stream=stream)
-        y_host.copy_(layer.y, non_blocking=True)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        x_dev2.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev2, stream=stream)
-        y_host.copy_(layer.y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = None
+    if e2e:
+        # end to end through the public API with host buffers
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+        x_dev2 = torch.empty_like(x)
+        for _ in range(2):
+            x_dev2.copy_(x_host, non_blocking=True)
+            layer.forward(x_dev2, stream=stream)
+            y_host.copy_(layer.y, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            x_dev2.copy_(x_host, non_blocking=True)
+            layer.forward(x_dev2, stream=stream)
+            y_host.copy_(layer.y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
 
     if pg is not None:
-        t = torch.tensor([total_ms, e2e_ms], device=dev)
+        t = torch.tensor([total_ms, e2e_ms or 0.0], device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         total_ms, e2e_ms = t.tolist()
 
-    if rank == 0:
-        P = peaks()
-        ms_step = total_ms / args.steps
-        value = world * cfg.T * args.steps / (total_ms / 1e3)
-        ffn_ms = statistics.mean(per_phase["experts"])
+    P = peaks()
+    fp8 = cfg.dtype == "e4m3"
+    # FP8 peak = the measured bf16 peak x the nominal dense ratio (4.5 / 2.25 PFLOP/s)
+    peak = P["bf16"] * (2.0 if fp8 else 1.0)
+    peak_src = P["source"] + (" bf16 burst x nominal fp8/bf16 ratio 2" if fp8 else " burst")
+    ffn_ms = statistics.mean(per_phase["experts"])
+    wbytes = 1 if fp8 else 2
+    fl = flops_per_forward(cfg)
+    used = int(np.count_nonzero(counts)) + 1
+    by = used * 3 * cfg.d * cfg.f * wbytes + 2 * cfg.T * cfg.d * 2 + cfg.N * cfg.d * 4
+    roof_ms = max(fl / (peak * 1e12), by / (P["hbm"] * 1e9)) * 1e3
+    ms_step = total_ms / steps
+    if cfg.zipf_s is None:
         achieved = ffn_flops(cfg) / (ffn_ms / 1e3) / 1e12
-        fl = flops_per_forward(cfg)
-        by = bytes_per_forward(cfg, counts)
-        roof_ms = max(fl / (P["bf16"] * 1e12), by / (P["hbm"] * 1e9)) * 1e3
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded; random-init weights of the DeepSeek-V3 MoE layer shape)",
-            "config": {"workload": workload_name(cfg), "global_batch": world * cfg.T,
-                       "l2": "inputs larger than L2: the expert weights "
-                             f"({(cfg.N + 1) * 3 * cfg.d * cfg.f * 2 / 1e9:.1f} GB) stream "
-                             "through it every step",
-                       "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, "
-                         "GEMM2)", "achieved": achieved, "peak": P["bf16"], "unit": "TFLOP/s",
-                         "frac": achieved / P["bf16"], "peak_source": P["source"] + " burst",
-                         "traffic": None},
-            "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step,
-                               "flops": fl, "bytes": by},
+        roof = {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, GEMM2)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": peak_src, "traffic": None}
+    else:
+        # decode: the experts stream the weights of the experts that received rows
+        wb = used * 3 * cfg.d * cfg.f * wbytes
+        achieved = wb / (ffn_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": "moe_expert_ffn (weights of the experts hit)",
+                "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
+                "frac": achieved / P["hbm"], "peak_source": P["source"] + " copy",
+                "traffic": None, "experts_hit": used - 1}
+    return {"cfg": cfg, "steps": steps, "total_ms": total_ms, "e2e_ms": e2e_ms,
             "phases_ms": {p: statistics.mean(v) for p, v in per_phase.items()},
-            "e2e": {"value": world * cfg.T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": cfg.T * cfg.d * 2,
-                    "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-            "gpu_launches": 8 * args.steps,
-            "clocks": clk.summary(),
-            "device_status": status,
+            "roofline": roof,
+            "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step, "flops": fl, "bytes": by},
+            "clocks": clk.summary(), "status": status,
             "load_max_over_mean": float(counts.max() / counts.mean()),
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            v, cores, note = cpu_oracle_baseline(cfg, args.cpu_sample)
-            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
-                                    "kind": "oracle", "sample": note}
-        print(json.dumps(line), flush=True)
-    if pg is not None:
-        pg.destroy_process_group()
+            # route 3 (split, score GEMM, select), dispatch 3, experts 2 (+1 quantiser
+            # for FP8), combine 1, bias 1
+            "launches_per_step": 10 if not fp8 else 11}
 
 
 if __name__ == "__main__":
