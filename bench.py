@@ -181,6 +181,16 @@ def dist_setup(args):
     return world, rank, local, pg
 
 
+def reduce_max(values, pg, device):
+    """Element-wise max of a list of floats over all ranks (identity on one rank)."""
+    if pg is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_reference(args, cfg):
     world, rank, local, pg = dist_setup(args)
     if rank != 0:
@@ -381,10 +391,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
 
-    if pg is not None:
-        t = torch.tensor([total_ms, e2e_ms or 0.0], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms, e2e_ms = t.tolist()
+    total_ms, e2e_ms = reduce_max([total_ms, e2e_ms or 0.0], pg, dev)
 
     P = peaks()
     fp8 = cfg.dtype == "e4m3"
