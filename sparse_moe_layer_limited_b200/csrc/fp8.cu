@@ -346,11 +346,28 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      // scales are read two slices ahead so their latency hides behind the
+      // previous slices' work
+      const float* sw0p = args.sw + wblk0 * KB;
+      const float* sw1p = args.sw + (wblk0 + 1) * KB;
+      float sa_n0 = valid ? __ldg(sa_row) : 0.f, sw0_n0 = __ldg(sw0p), sw1_n0 = __ldg(sw1p);
+      float sa_n1 = 0.f, sw0_n1 = 0.f, sw1_n1 = 0.f;
+      if (KB > 1) {
+        sa_n1 = valid ? __ldg(sa_row + 1) : 0.f;
+        sw0_n1 = __ldg(sw0p + 1);
+        sw1_n1 = __ldg(sw1p + 1);
+      }
       for (int kb = 0; kb < KB; ++kb, ++slice) {
         const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
-        const float sa = valid ? __ldg(sa_row + kb) : 0.f;
-        const float sw0 = __ldg(args.sw + wblk0 * KB + kb);
-        const float sw1 = __ldg(args.sw + (wblk0 + 1) * KB + kb);
+        const float sa = sa_n0, sw0 = sw0_n0, sw1 = sw1_n0;
+        sa_n0 = sa_n1;
+        sw0_n0 = sw0_n1;
+        sw1_n0 = sw1_n1;
+        if (kb + 2 < KB) {
+          sa_n1 = valid ? __ldg(sa_row + kb + 2) : 0.f;
+          sw0_n1 = __ldg(sw0p + kb + 2);
+          sw1_n1 = __ldg(sw1p + kb + 2);
+        }
         if (!mbar_wait_bounded(&sfull[sb], sph, args.status, FTimeoutNs)) {
           ok = false;
           break;

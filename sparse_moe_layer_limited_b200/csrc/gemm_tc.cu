@@ -44,6 +44,8 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "internal.h"
@@ -393,6 +395,11 @@ __global__ void router_split_kernel(const float* __restrict__ R, int N, int d,
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                        const void* x, const void* w13, const void* w2, void* y_perm,
                        void* y_shared, void* ws, cudaStream_t st) {
+  static const bool pair = [] {
+    const char* v = std::getenv("MOE_BF16_GEMM");
+    return v != nullptr && std::strcmp(v, "pair") == 0;
+  }();
+  if (pair) return launch_ffn_tc_bf16_pair(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
   const WsLayout L = ws_layout(s);
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(w + L.h);
