@@ -159,7 +159,6 @@ struct alignas(64) Fp8Args {
   int n_acc;   // weight rows per group (2f or d)
   int k_dim;   // contraction length
   int out_ld;  // f (GEMM1 codes) or d (GEMM2)
-  int w_prefetch;  // weight K blocks prefetched into L2 ahead (first token tile only)
 };
 
 constexpr size_t fp8_smem_bytes(int groups) {
@@ -266,14 +265,7 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
         const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
         const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * FBM;
         const int brow = g * args.n_acc + n * FBN;
-        // the first token tile of a weight tile prefetches it into L2 far ahead
-        const bool first = (m == 0) && args.w_prefetch > 0;
-        if (first)
-          for (int kb = 0; kb < min(KB, args.w_prefetch); ++kb)
-            tma_prefetch_l2_2d(&args.tmB, kb * FBK, brow);
         for (int kb = 0; kb < KB; ++kb) {
-          if (first && kb + args.w_prefetch < KB)
-            tma_prefetch_l2_2d(&args.tmB, (kb + args.w_prefetch) * FBK, brow);
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, FTimeoutNs)) {
             ok = false;
             break;
@@ -571,7 +563,6 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
   g1.n_acc = 2 * s.f;
   g1.k_dim = s.d;
   g1.out_ld = s.f;
-  g1.w_prefetch = prefetch_blocks();
   if (launch_fp8_gemm<kFEpiSwiGLUQuant>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   Fp8Args g2{};
@@ -596,7 +587,6 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
   g2.n_acc = s.d;
   g2.k_dim = s.f;
   g2.out_ld = s.d;
-  g2.w_prefetch = prefetch_blocks();
   if (launch_fp8_gemm<kFEpiStore>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

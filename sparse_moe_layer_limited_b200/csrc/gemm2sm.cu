@@ -62,7 +62,6 @@ struct alignas(64) PairArgs {
   int n_feat;   // weight rows per group (2f for GEMM1, d for GEMM2)
   int k_dim;
   int out_ld;
-  int w_prefetch;  // weight K blocks prefetched into L2 ahead (first token tile only)
 };
 
 constexpr size_t pair_smem_bytes(int groups) {
@@ -182,21 +181,7 @@ __global__ void __launch_bounds__(PThreads, 1) pair_gemm_bf16_kernel(
         const int xrow = ((g < args.N) ? args.offsets[g] : args.x_shared_row0) + mt * PT +
                          (int)rank * half;
         const int wtile = g * args.n_feat + nf * 2 * PW;
-        // first token tile of a weight tile: prefetch this CTA's weight rows into
-        // L2 far ahead (the other tiles of the expert then hit L2)
-        const bool first = (mt == 0) && args.w_prefetch > 0;
-        auto prefetch_w = [&](int kb) {
-          if constexpr (kEpi == kPSwiGLU) {
-            tma_prefetch_l2_2d(&args.tmW, kb * PK, wtile + 64 * (int)rank);
-            tma_prefetch_l2_2d(&args.tmW, kb * PK, wtile + PW + 64 * (int)rank);
-          } else {
-            tma_prefetch_l2_2d(&args.tmW, kb * PK, wtile + PW * (int)rank);
-          }
-        };
-        if (first)
-          for (int kb = 0; kb < min(KB, args.w_prefetch); ++kb) prefetch_w(kb);
         for (int kb = 0; kb < KB; ++kb) {
-          if (first && kb + args.w_prefetch < KB) prefetch_w(kb + args.w_prefetch);
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, PTimeoutNs)) {
             ok = false;
             break;
@@ -417,7 +402,6 @@ int launch_ffn_tc_bf16_pair(const moe_shape& s, const void* x_perm, const int32_
   g1.n_feat = 2 * s.f;
   g1.k_dim = s.d;
   g1.out_ld = s.f;
-  g1.w_prefetch = prefetch_blocks();
   if (launch_pair<kPSwiGLU>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   PairArgs g2{};
@@ -439,7 +423,6 @@ int launch_ffn_tc_bf16_pair(const moe_shape& s, const void* x_perm, const int32_
   g2.n_feat = s.d;
   g2.k_dim = s.f;
   g2.out_ld = s.d;
-  g2.w_prefetch = prefetch_blocks();
   if (launch_pair<kPStore>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

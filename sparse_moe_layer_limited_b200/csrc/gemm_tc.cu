@@ -90,7 +90,6 @@ struct alignas(64) GemmArgs {
   int a_rep;   // K blocks that reuse one A tile (3 for the split router, else 1)
   int n_valid; // columns to store (score epilogue)
   int k_splits; // K ranges computed by separate units (score epilogue; else 1)
-  int w_prefetch; // weight K blocks prefetched into L2 ahead by first-tile units (0 = off)
 };
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
@@ -210,16 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
         const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * BM;
         const int brow = g * args.n_acc + (n / args.k_splits) * BN;
         const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
-        // the unit with the first token tile of a weight tile reads it from HBM
-        // (its neighbours hit L2): it alone runs an L2 prefetch far ahead, so
-        // enough HBM reads are in flight to keep the weight stream at full rate
-        const bool first = (m == 0) && args.w_prefetch > 0;
-        if (first)
-          for (int kb = kb0; kb < min(kb1, kb0 + args.w_prefetch); ++kb)
-            tma_prefetch_l2_2d(&args.tmB, kb * BK, brow);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (first && kb + args.w_prefetch < kb1)
-            tma_prefetch_l2_2d(&args.tmB, (kb + args.w_prefetch) * BK, brow);
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs)) {
             ok = false;
             break;
@@ -402,16 +392,6 @@ __global__ void router_split_kernel(const float* __restrict__ R, int N, int d,
 
 }  // namespace
 
-// Weight K blocks to prefetch ahead (MOE_W_PREFETCH; default 0 = off: on
-// the V3 layer prefetching 8/16/32 blocks ahead measured 1.3x/1.5x/1.6x slower).
-int prefetch_blocks() {
-  static const int v = [] {
-    const char* e = std::getenv("MOE_W_PREFETCH");
-    return e ? std::atoi(e) : 0;
-  }();
-  return v;
-}
-
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                        const void* x, const void* w13, const void* w2, void* y_perm,
                        void* y_shared, void* ws, cudaStream_t st) {
@@ -447,7 +427,6 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g1.out_ld = s.f;
   g1.a_rep = 1;
   g1.k_splits = 1;
-  g1.w_prefetch = prefetch_blocks();
   if (launch_gemm<kEpiSwiGLU, 256>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   GemmArgs g2{};
@@ -471,7 +450,6 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g2.out_ld = s.d;
   g2.a_rep = 1;
   g2.k_splits = 1;
-  g2.w_prefetch = prefetch_blocks();
   if (launch_gemm<kEpiStore, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -50,8 +50,6 @@ void note_text(const char* what);
 bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t elem_bytes,
               uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows);
 int num_sms();
-// Weight K blocks the expert GEMMs prefetch into L2 ahead of their loads.
-int prefetch_blocks();
 
 // ---- launchers (return cudaError_t of the launch) -----------------------------
 int launch_route(const moe_shape& s, const void* x, const float* router, const float* bias,
