@@ -13,8 +13,8 @@
 // The per-slice products come from tcgen05.mma kind::f8f6f4 (E4M3 x E4M3,
 // fp32 accumulate, M=128 tokens, N=256 weight columns, K=32 each); every
 // 128-wide slice lands in its own TMEM buffer (two 256-column buffers, so
-// the tensor core fills one while the other is drained).  Eight epilogue
-// warps -- two per TMEM lane quadrant, each owning 128 of the 256 columns --
+// the tensor core fills one while the other is drained).  Sixteen epilogue
+// warps -- four per TMEM lane quadrant, each owning 64 of the 256 columns --
 // fold each slice into fp32 register sums with the product of the two
 // scales.  This per-slice promotion is the tcgen05 counterpart of the
 // article's "accumulate at an interval in fp32 on the CUDA cores" (the
@@ -24,14 +24,15 @@
 //
 // GEMM1 epilogue: h = silu(gate) * up for the 128 hidden features of the
 // tile (gate and up columns of one feature lie in the same tile and thread
-// row), then h is quantised per 1x128 tile along f; the two warps that share
-// a row exchange their half-tile max-abs through shared memory under an
-// mbarrier.  GEMM2 epilogue: bf16 output rows.
+// row), then h is quantised per 1x128 tile along f; the four warps that
+// share a row exchange their quarter-tile max-abs through shared memory
+// under an mbarrier.  GEMM2 epilogue: bf16 output rows.
 // Roles: warp 0 TMA producer (4-stage ring: 128 token rows + 256 weight rows
-// of 128 bytes), warp 1 TMEM owner and MMA issuer, warps 2-9 epilogue.
-// Ten warps put three on some of the SM's four 16K-register banks, which caps
-// a thread at 168 registers: the epilogue keeps its 128 running sums and
-// drains TMEM 16 columns at a time.
+// of 128 bytes), warp 1 TMEM owner and MMA issuer, warps 2-17 epilogue.
+// Sixteen epilogue warps (four per TMEM lane quadrant, 64 running sums each)
+// keep a thread within the register budget of an 18-warp CTA (five warps
+// share some of the SM's four 16K-register banks) and give each scheduler
+// four warps to overlap the TMEM-load latency of the per-slice promotion.
 // All waits are bounded (~2 s) and set the device status word on expiry.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -49,8 +50,8 @@ constexpr int FStages = 4;
 constexpr int FABytes = FBM * FBK;      // 16 KB
 constexpr int FBBytes = FBN * FBK;      // 32 KB
 constexpr int FStageBytes = FABytes + FBBytes;
-constexpr int FThreads = 320;
-constexpr int FEpiWarps = 8;
+constexpr int FThreads = 576;   // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
+constexpr int FEpiWarps = 16;   // four per TMEM lane quadrant
 constexpr uint64_t FTimeoutNs = 2000000000ull;
 
 enum FEpi { kFEpiSwiGLUQuant = 0, kFEpiStore = 1 };
@@ -162,7 +163,7 @@ struct alignas(64) Fp8Args {
 };
 
 constexpr size_t fp8_smem_bytes(int groups) {
-  return 1024 + (size_t)FStages * FStageBytes + 512 + 2 * 2 * FBM * 4 + (size_t)(groups + 1) * 4;
+  return 1024 + (size_t)FStages * FStageBytes + 512 + 2 * 4 * FBM * 4 + (size_t)(groups + 1) * 4;
 }
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
@@ -181,8 +182,8 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
   uint64_t* xbar = sempty + 2;            // [2] amax exchange (8 warps)
   uint64_t* drain = xbar + 2;             // [1]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  float* xchg = reinterpret_cast<float*>(base + (size_t)FStages * FStageBytes + 512);  // [2][2][128]
-  int* tile_start = reinterpret_cast<int*>(xchg + 2 * 2 * FBM);
+  float* xchg = reinterpret_cast<float*>(base + (size_t)FStages * FStageBytes + 512);  // [2][4][128]
+  int* tile_start = reinterpret_cast<int*>(xchg + 2 * 4 * FBM);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -323,11 +324,14 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       mbar_wait_bounded(drain, 0, args.status, FTimeoutNs / 8);
     }
   } else {
-    // ---- epilogue: warps 2..9 ----
-    const int q = warp & 3;             // TMEM lane quadrant
-    const int half = (warp - 2) >> 2;   // which 128 of the 256 columns
-    const int row = q * 32 + lane;      // token row within the tile
-    const int ewarp = warp - 2;
+    // ---- epilogue: warps 2..17 ----
+    // Warp w may read TMEM lanes 32*(w%4)..+31 (its row quadrant); the four
+    // warps of a quadrant split the 256 columns: in GEMM1 warp `sub` owns the
+    // gate columns 32*sub.. and the up columns 128+32*sub.. (hidden features
+    // 32*sub..+31 of the tile), in GEMM2 the 64 columns 64*sub..
+    const int q = warp & 3;
+    const int sub = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
     uint32_t slice = 0;
     int local = 0;
     bool ok = true;
@@ -343,30 +347,22 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       const float* sa_row = ((g < args.N) ? args.sa_routed : args.sa_shared) +
                             (valid ? arow_idx : 0) * KB;
       const long long wblk0 = ((long long)g * args.n_acc + (long long)n * FBN) / QB;
-      float acc[128];
+      // weight-block scales this warp needs: GEMM1 gate (block 0) and up
+      // (block 1); GEMM2 the block of its 64 columns
+      const float* swA = args.sw + (kEpi == kFEpiSwiGLUQuant ? wblk0 : wblk0 + (sub >> 1)) * KB;
+      const float* swB = args.sw + (kEpi == kFEpiSwiGLUQuant ? wblk0 + 1 : wblk0 + (sub >> 1)) * KB;
+      float acc[64];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
-      // scales are read two slices ahead so their latency hides behind the
-      // previous slices' work
-      const float* sw0p = args.sw + wblk0 * KB;
-      const float* sw1p = args.sw + (wblk0 + 1) * KB;
-      float sa_n0 = valid ? __ldg(sa_row) : 0.f, sw0_n0 = __ldg(sw0p), sw1_n0 = __ldg(sw1p);
-      float sa_n1 = 0.f, sw0_n1 = 0.f, sw1_n1 = 0.f;
-      if (KB > 1) {
-        sa_n1 = valid ? __ldg(sa_row + 1) : 0.f;
-        sw0_n1 = __ldg(sw0p + 1);
-        sw1_n1 = __ldg(sw1p + 1);
-      }
+      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      // scales are read one slice ahead so their latency hides behind a slice
+      float sa_n = valid ? __ldg(sa_row) : 0.f, swA_n = __ldg(swA), swB_n = __ldg(swB);
       for (int kb = 0; kb < KB; ++kb, ++slice) {
         const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
-        const float sa = sa_n0, sw0 = sw0_n0, sw1 = sw1_n0;
-        sa_n0 = sa_n1;
-        sw0_n0 = sw0_n1;
-        sw1_n0 = sw1_n1;
-        if (kb + 2 < KB) {
-          sa_n1 = valid ? __ldg(sa_row + kb + 2) : 0.f;
-          sw0_n1 = __ldg(sw0p + kb + 2);
-          sw1_n1 = __ldg(sw1p + kb + 2);
+        const float sA = sa_n * swA_n, sB = sa_n * swB_n;
+        if (kb + 1 < KB) {
+          sa_n = valid ? __ldg(sa_row + kb + 1) : 0.f;
+          swA_n = __ldg(swA + kb + 1);
+          swB_n = __ldg(swB + kb + 1);
         }
         if (!mbar_wait_bounded(&sfull[sb], sph, args.status, FTimeoutNs)) {
           ok = false;
@@ -374,26 +370,20 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * FBN;
-        // 16 columns per TMEM load keeps 128 sums + 16 loads within the
-        // register budget of a 10-warp CTA (3 warps share a 16K-register bank)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           int col;
-          float s;
-          if constexpr (kEpi == kFEpiSwiGLUQuant) {
-            // gate columns (W1 block) then up columns (W3 block) of features 64*half..
-            col = (c < 4) ? 64 * half + 16 * c : 128 + 64 * half + 16 * (c - 4);
-            s = sa * ((c < 4) ? sw0 : sw1);
-          } else {
-            col = 128 * half + 16 * c;
-            s = sa * (half ? sw1 : sw0);
-          }
+          if constexpr (kEpi == kFEpiSwiGLUQuant)
+            col = (c < 2) ? 32 * sub + 16 * c : 128 + 32 * sub + 16 * (c - 2);
+          else
+            col = 64 * sub + 16 * c;
+          const float sc = (c < 2) ? sA : sB;
           uint32_t p[16];
           tmem_ld16(taddr + col, p);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            acc[c * 16 + i] = fmaf(__uint_as_float(p[i]), s, acc[c * 16 + i]);
+            acc[c * 16 + i] = fmaf(__uint_as_float(p[i]), sc, acc[c * 16 + i]);
         }
         tc_fence_before();
         __syncwarp();
@@ -402,29 +392,29 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       if (!ok) break;
 
       if constexpr (kEpi == kFEpiSwiGLUQuant) {
-        // h for hidden features n*128 + 64*half + i, i < 64
+        // h for hidden features n*128 + 32*sub + i, i < 32
         float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          acc[i] = silu_f(acc[i]) * acc[64 + i];
+        for (int i = 0; i < 32; ++i) {
+          acc[i] = silu_f(acc[i]) * acc[32 + i];
           amax = fmaxf(amax, fabsf(acc[i]));
         }
-        // exchange the half-tile max-abs with the warp holding the other 64 features
-        float* xb = xchg + (local & 1) * 2 * FBM;
-        xb[half * FBM + row] = amax;
+        // the row's 1x128 tile spans the four warps of this quadrant
+        float* xb = xchg + (local & 1) * 4 * FBM;
+        xb[sub * FBM + row] = amax;
         __syncwarp();
         if (lane == 0) mbar_arrive(&xbar[local & 1]);
         if (!mbar_wait_bounded(&xbar[local & 1], (local >> 1) & 1, args.status, FTimeoutNs)) break;
-        amax = fmaxf(xb[row], xb[FBM + row]);
+        amax = fmaxf(fmaxf(xb[row], xb[FBM + row]), fmaxf(xb[2 * FBM + row], xb[3 * FBM + row]));
         const bool zero = amax == 0.f;
         const float scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
         const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
         if (valid) {
           uint8_t* qrow = ((g < args.N) ? args.q_routed + (long long)args.offsets[g] * args.out_ld
                                         : args.q_shared) +
-                          (long long)r * args.out_ld + n * QB + 64 * half;
+                          (long long)r * args.out_ld + n * QB + 32 * sub;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < 2; ++v) {
             uint32_t w4[4];
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {
@@ -443,7 +433,7 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
             }
             reinterpret_cast<uint4*>(qrow)[v] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-          if (half == 0) {
+          if (sub == 0) {
             float* srow = (g < args.N) ? args.qs_routed + ((long long)args.offsets[g] + r) *
                                                             (args.out_ld / QB)
                                        : args.qs_shared + (long long)r * (args.out_ld / QB);
@@ -455,9 +445,9 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           __nv_bfloat16* yrow =
               ((g < args.N) ? args.y_routed + ((long long)args.offsets[g] + r) * args.out_ld
                             : args.y_shared + (long long)r * args.out_ld) +
-              n * FBN + 128 * half;
+              n * FBN + 64 * sub;
 #pragma unroll
-          for (int v = 0; v < 16; ++v) {
+          for (int v = 0; v < 8; ++v) {
             uint4 w;
             __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&w);
 #pragma unroll
@@ -467,7 +457,6 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           }
         }
       }
-      (void)ewarp;
     }
   }
 
