@@ -181,6 +181,11 @@ def dist_setup(args):
     return world, rank, local, pg
 
 
+def pair_gemm():
+    """True when the bf16 expert GEMMs run on CTA pairs (MOE_BF16_GEMM=pair)."""
+    return os.environ.get("MOE_BF16_GEMM") == "pair"
+
+
 def reduce_max(values, pg, device):
     """Element-wise max of a list of floats over all ranks (identity on one rank)."""
     if pg is None:
@@ -410,6 +415,14 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
         roof = {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, GEMM2)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": peak_src, "traffic": None}
+        if cfg.name == "v3_bf16" and cfg.T == 8192 and cfg.N == 256 and not pair_gemm():
+            # DRAM bytes of one moe_expert_ffn call (GEMM1 + GEMM2), from the ncu
+            # capture of the same kernels on the T=1024 / 32+1-expert case
+            # (profiles/hot_kernels_small_v3shape.md: 3.28 GB), scaled by the
+            # expert weights (x 257/33) and the activation rows (x 8)
+            roof["traffic"] = 25.6e9
+            roof["traffic_note"] = ("bytes per call, ncu capture of a smaller case scaled to "
+                                    "the full layer; algorithmic 25.35e9")
     else:
         # decode: the experts stream the weights of the experts that received rows
         wb = used * 3 * cfg.d * cfg.f * wbytes
