@@ -241,3 +241,56 @@ def test_small_fp8_layer_full(M, T):
     err = S.rel_fro(y, ref["y"])
     assert err <= TOL["e4m3"], err
     assert layer.device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# degenerate and maximum-size routing / layer cases
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,G,topG", [
+    (8, 8, 1, 1),       # K = N: every expert on every token
+    (16, 4, 16, 4),     # one expert per group: group score = that expert's biased score
+    (256, 32, 8, 4),    # the largest K and N the kernels take
+    (64, 1, 8, 1),      # K = 1, a single group kept
+])
+def test_route_degenerate_and_max(M, N, K, G, topG):
+    cfg = CONFIGS[1].with_(T=777, d=256, N=N, K=K, G=G, topG=topG, f=256)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
+    _check_route(cfg, r, *_run_route(M, cfg, x, R, b))
+
+
+def test_layer_all_experts_every_token(M):
+    """K = N: each expert's group holds every token (several m-tiles each)."""
+    cfg = CONFIGS[1].with_(T=300, d=256, N=4, K=4, G=1, topG=1, f=256)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).float().cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             h_round="bf16")
+    assert np.all(layer.counts.cpu().numpy() == cfg.T)
+    _check_dispatch(layer, ref["route"])
+    assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
+    assert layer.device_status() == 0
+
+
+def test_layer_with_idle_experts(M):
+    """Biases push all tokens into two groups, so most experts get no rows."""
+    cfg = CONFIGS[1].with_(T=500, d=256, N=32, K=2, G=8, topG=2, f=256)
+    R = gen.make_router(cfg)
+    b = gen.make_bias(cfg).copy()
+    b[:8] += 0.5                                    # groups 0 and 1 win every token
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).float().cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             h_round="bf16")
+    counts = layer.counts.cpu().numpy()
+    assert counts[8:].sum() == 0 and counts.sum() == cfg.T * cfg.K
+    _check_dispatch(layer, ref["route"])
+    assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
+    assert layer.device_status() == 0
