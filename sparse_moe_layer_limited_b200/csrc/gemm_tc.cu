@@ -11,7 +11,8 @@
 // the shared expert (T rows).
 //
 // Work unit: a 128 x 256 output tile (tcgen05.mma cta_group::1, M=128,
-// N=256, K=16 per instruction), ordered group-major, then n-tile, then
+// N=256, K=16 per instruction; M=64 when an expert's last tile has at most
+// 64 rows), ordered group-major, then n-tile, then
 // m-tile, so CTAs running side by side share the same weight tile through
 // L2 and each expert's weights stream from HBM about once.  Each CTA (one
 // per SM) walks tiles blockIdx.x, +gridDim.x, ... with three roles:
@@ -235,7 +236,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   } else if (warp == 1) {
     // ---- MMA issuer -----------------------------------------------------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -244,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
         int g, n, m, mt;
         decode(tile, g, n, m, mt);
         const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
+        // a tile with at most 64 real rows (an expert's ragged tail) runs the
+        // M=64 MMA: half the tensor work for the same weight stream
+        const int rows_g = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
+        const uint32_t idesc = idesc_bf16_f32(rows_g - m * BM <= 64 ? 64 : BM, kBN);
         const int acc = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aphase ^ 1u, args.status, kTimeoutNs)) break;
@@ -285,7 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
       if (!mbar_wait_bounded(&tfull[acc], aphase, args.status, kTimeoutNs)) break;
       tc_fence_after();
       const int rows_g = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
-      const int r = m * BM + row;
+      // M=64 tiles (<= 64 rows) hold row 16*q + i in TMEM lane 32*q + i (i < 16)
+      const bool m64 = rows_g - m * BM <= 64;
+      const int r = m * BM + (m64 ? (lane < 16 ? 16 * q + lane : BM) : row);
       // rows past the group's end belong to the next group (or are padding);
       // the second test keeps a corrupted offsets[] from writing out of range
       const bool valid = r < rows_g && (g == args.N || args.offsets[g] + r < args.rows_routed);
