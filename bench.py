@@ -42,6 +42,10 @@ def parse():
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--cpu-sample", type=int, default=2, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak"], default=None,
+                   help="measurement probes behind the profiles: expert GEMMs on uniform "
+                        "expert loads, cuBLAS batched GEMM at the expert shapes, FP8 GEMM peak")
+    p.add_argument("--rows", type=int, default=256, help="rows per expert for --probe uniform")
     p.add_argument("--no-extra", action="store_true",
                    help="skip the FP8 and decode workloads reported beside the headline")
     p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
@@ -226,6 +230,90 @@ def run_reference(args, cfg):
         pg.destroy_process_group()
 
 
+def _time_ms(fn, iters=10, warm=3, best=False):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    if best:
+        out = 1e30
+        for _ in range(iters):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            out = min(out, e0.elapsed_time(e1))
+        return out
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def run_probe(args, cfg):
+    """Probes behind profiles/expert_gemm_experiments_v3.md; one JSON line each.
+    uniform: moe_expert_ffn alone with exactly --rows rows per routed expert
+             (random activations), routed + shared experts;
+    cublas:  torch.bmm over N experts x 256 rows at the expert GEMM shapes (the
+             ideal grouped problem, routed part only), and a dense GEMM;
+    fp8peak: torch._scaled_mm E4M3 8192^3, best of 10."""
+    import torch
+    import sparse_moe_layer_limited_b200 as M
+    from synth import device as sdev
+    dev = torch.device("cuda")
+    out = {"probe": args.probe}
+    if args.probe == "fp8peak":
+        n = 8192
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.tensor(1.0, device=dev)
+        ms = _time_ms(lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,
+                                               out_dtype=torch.bfloat16), best=True)
+        out.update(ms=ms, tflops=2 * n ** 3 / ms / 1e9)
+    elif args.probe == "cublas":
+        E, R, d, f = cfg.N, 256, cfg.d, cfg.f
+        A = torch.randn(E, R, d, device=dev, dtype=torch.bfloat16)
+        W13 = torch.randn(E, d, 2 * f, device=dev, dtype=torch.bfloat16)
+        H = torch.randn(E, R, f, device=dev, dtype=torch.bfloat16)
+        W2 = torch.randn(E, f, d, device=dev, dtype=torch.bfloat16)
+        t1 = _time_ms(lambda: torch.bmm(A, W13))
+        t2 = _time_ms(lambda: torch.bmm(H, W2))
+        Ad = torch.randn(E * R, d, device=dev, dtype=torch.bfloat16)
+        t3 = _time_ms(lambda: Ad @ W13[0])
+        t4 = _time_ms(lambda: W13.sum(dtype=torch.float32))
+        out.update(gemm1_ms=t1, gemm1_tflops=2 * E * R * d * 2 * f / t1 / 1e9,
+                   gemm1_weight_tbs=W13.numel() * 2 / t1 / 1e9,
+                   gemm2_ms=t2, gemm2_tflops=2 * E * R * f * d / t2 / 1e9,
+                   gemm2_weight_tbs=W2.numel() * 2 / t2 / 1e9,
+                   dense_ms=t3, dense_tflops=2 * E * R * d * 2 * f / t3 / 1e9,
+                   weight_read_tbs=W13.numel() * 2 / t4 / 1e9)
+    else:
+        rows = args.rows
+        T = rows * cfg.N // cfg.K
+        s = M.shape(T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f, M.DTYPE_BF16)
+        w1 = sdev.expert_weights_bf16(cfg, 0, "w1", dev)
+        w3 = sdev.expert_weights_bf16(cfg, 0, "w3", dev)
+        w13 = torch.empty(cfg.N + 1, 2 * cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
+        M.moe_pack_w13(s, w1, w3, w13)
+        del w1, w3
+        w2 = sdev.expert_weights_bf16(cfg, 0, "w2", dev)
+        offs = torch.arange(cfg.N + 1, dtype=torch.int32, device=dev) * rows
+        xp = torch.randn(T * cfg.K, cfg.d, device=dev).to(torch.bfloat16)
+        x = torch.randn(T, cfg.d, device=dev).to(torch.bfloat16)
+        yp, ysh = torch.empty_like(xp), torch.empty_like(x)
+        ws = torch.zeros(M.workspace_size(s), dtype=torch.uint8, device=dev)
+        ms = _time_ms(lambda: M.moe_expert_ffn(s, xp, None, offs, x, w13, w2, None, None, yp,
+                                                ysh, ws))
+        fl = 6.0 * cfg.d * cfg.f * (T * cfg.K + T)
+        out.update(rows_per_expert=rows, kernel="pair" if pair_gemm() else "one-CTA", ms=ms,
+                   tflops=fl / ms / 1e9)
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
     cfg = BY_NAME[args.config]
@@ -235,6 +323,8 @@ def main():
         cfg = cfg.with_(N=args.N)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.probe:
+        return run_probe(args, cfg)
 
     import torch
 
