@@ -42,7 +42,7 @@ def parse():
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--cpu-sample", type=int, default=2, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak"], default=None,
+    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak", "mma"], default=None,
                    help="measurement probes behind the profiles: expert GEMMs on uniform "
                         "expert loads, cuBLAS batched GEMM at the expert shapes, FP8 GEMM peak")
     p.add_argument("--rows", type=int, default=256, help="rows per expert for --probe uniform")
@@ -260,7 +260,14 @@ def run_probe(args, cfg):
              (random activations), routed + shared experts;
     cublas:  torch.bmm over N experts x 256 rows at the expert GEMM shapes (the
              ideal grouped problem, routed part only), and a dense GEMM;
-    fp8peak: torch._scaled_mm E4M3 8192^3, best of 10."""
+    fp8peak: torch._scaled_mm E4M3 8192^3, best of 10;
+    mma:     the tcgen05.mma issue-rate probe (SM cycles per instruction shape)."""
+    if args.probe == "mma":
+        import subprocess
+        from sparse_moe_layer_limited_b200 import build as B
+        if not os.path.exists(B.PROBE_PATH):
+            B.build_probe()
+        return subprocess.run([B.PROBE_PATH], check=True)
     import torch
     import sparse_moe_layer_limited_b200 as M
     from synth import device as sdev

@@ -49,6 +49,10 @@ void note_text(const char* what);
 // 128-byte swizzle; out-of-range rows read as zero.
 bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t elem_bytes,
               uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows);
+// `rank`-D tensor (2..5) given by its dims (innermost first), the byte strides of
+// dims 1..rank-1 and the box; 128-byte swizzle, out-of-range elements read as zero.
+bool make_map_nd(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int rank,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
 int num_sms();
 
 // ---- launchers (return cudaError_t of the launch) -----------------------------

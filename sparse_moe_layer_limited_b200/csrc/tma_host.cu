@@ -39,6 +39,24 @@ bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t 
   return r == CUDA_SUCCESS;
 }
 
+bool make_map_nd(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int rank,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) st[i] = strides_bytes[i];
+  CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(ptr), d, st, b, e,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   static int n = 0;
   if (n == 0) {
