@@ -146,8 +146,11 @@ int moe_route(const moe_shape* shape, const void* x, const float* router_w, cons
  *   slot       [T, K]  int32 out, row holding (t, topk_idx[t, k])
  *   x_perm     [T*K, d] out: bf16 copy of x rows (BF16), fp32 (FP32), or E4M3
  *                      codes (E4M3 mode, one byte per element)
- *   x_perm_scales [T*K, d/128] fp32 out, E4M3 mode only (NULL otherwise):
- *                      per-1x128-tile scale amax/448 ([P1] §4.1)
+ *   x_perm_scales [d/128, L] fp32 out, E4M3 mode only (NULL otherwise), with
+ *                      L = T*K rounded up to a multiple of 4: the scale
+ *                      amax/448 of row r's 1x128 tile j is at [j, r] ([P1]
+ *                      §4.1).  Block-major, so a tile of rows at one K block
+ *                      is contiguous; columns r >= T*K are not written.
  * Sets MOE_DEV_COUNT_MISMATCH if counts disagree with topk_idx. */
 int moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                  const int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* slot,

@@ -28,11 +28,11 @@ WsLayout ws_layout(const moe_shape& s) {
   off = align256(off + rows * s.f * dtype_bytes(s.dtype));
   if (s.dtype == MOE_DTYPE_E4M3) {
     L.h_scales = off;
-    off = align256(off + rows * (s.f / 128) * 4);
+    off = align256(off + (size_t)scale_ld((long long)rows) * (s.f / 128) * 4);
     L.xq = off;
     off = align256(off + (size_t)s.T * s.d);
     L.xq_scales = off;
-    off = align256(off + (size_t)s.T * (s.d / 128) * 4);
+    off = align256(off + (size_t)scale_ld(s.T) * (s.d / 128) * 4);
   }
   L.total = off;
   return L;

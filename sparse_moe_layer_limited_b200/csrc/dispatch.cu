@@ -168,12 +168,12 @@ __global__ void __launch_bounds__(256) scatter_gather_kernel(
 
 // E4M3 layer: slots as above, then each x row is quantised once per 1x128
 // tile (a half-warp per tile) and its codes and scales are written to the
-// token's K destination rows.
+// token's K destination rows (scales block-major: [d/128][sc_ld]).
 __global__ void __launch_bounds__(256) scatter_gather_fp8_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ chunk_base, int T, int d, int K, int N,
     int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot, uint8_t* __restrict__ x_perm,
-    float* __restrict__ x_perm_scales) {
+    float* __restrict__ x_perm_scales, long long sc_ld) {
   __shared__ int sidx[kChunkTokens * kMaxK];
   __shared__ int sslot[kChunkTokens * kMaxK];
   const int c = blockIdx.x;
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(256) scatter_gather_fp8_kernel(
         const int r = sslot[tl * K + k];
         if (r < 0) continue;
         *reinterpret_cast<uint2*>(x_perm + (size_t)r * d + tc * QB + 8 * l16) = codes;
-        if (l16 == 0) x_perm_scales[(size_t)r * tiles + tc] = sc;
+        if (l16 == 0) x_perm_scales[(size_t)tc * sc_ld + r] = sc;
       }
     }
   }
@@ -229,7 +229,7 @@ cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* id
   else
     scatter_gather_fp8_kernel<<<nch, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
-        slot, static_cast<uint8_t*>(x_perm), x_perm_scales);
+        slot, static_cast<uint8_t*>(x_perm), x_perm_scales, scale_ld((long long)s.T * s.K));
   return cudaGetLastError();
 }
 

@@ -33,6 +33,12 @@
 // keep a thread within the register budget of an 18-warp CTA (five warps
 // share some of the SM's four 16K-register banks) and give each scheduler
 // four warps to overlap the TMEM-load latency of the per-slice promotion.
+// Activation scales are block-major ([K/128][rows rounded up to 4]); for each
+// slice the producer copies the tile's 128 scales (a 132-float box starting at
+// the tile's first row rounded down to 4) into a ring of eight shared-memory
+// slots that the epilogue releases, so the promotion reads its per-row scale
+// from shared memory.  Weight-block scales are the same for a whole warp and
+// come through L1.
 // All waits are bounded (~2 s) and set the device status word on expiry.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -52,13 +58,18 @@ constexpr int FBBytes = FBN * FBK;      // 32 KB
 constexpr int FStageBytes = FABytes + FBBytes;
 constexpr int FThreads = 576;   // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
 constexpr int FEpiWarps = 16;   // four per TMEM lane quadrant
+constexpr int FScaleSlots = 8;      // ring of per-slice activation-scale boxes
+constexpr int FScaleBox = 132;      // floats per box: 128 rows + up to 3 of alignment
+constexpr int FScaleSlotBytes = 640;
 constexpr uint64_t FTimeoutNs = 2000000000ull;
 
 enum FEpi { kFEpiSwiGLUQuant = 0, kFEpiStore = 1 };
 
-// x [rows, d] bf16 -> codes [rows, d], scales [rows, d/128]; one half-warp per tile.
+// x [rows, d] bf16 -> codes [rows, d], scales block-major [d/128][sc_ld]; one
+// half-warp per tile.
 __global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ x, long long rows, int d,
-                                  uint8_t* __restrict__ q, float* __restrict__ sc) {
+                                  uint8_t* __restrict__ q, float* __restrict__ sc,
+                                  long long sc_ld) {
   const int tiles_per_row = d / QB;
   const long long tiles = rows * tiles_per_row;
   const int half = (threadIdx.x >> 4) & 1, l16 = threadIdx.x & 15;
@@ -79,7 +90,7 @@ __global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ x, long long
     const float s = quant_tile_16lanes(v, codes);
     if (live) {
       *reinterpret_cast<uint2*>(q + r * d + tc * QB + 8 * l16) = codes;
-      if (l16 == 0) sc[r * tiles_per_row + tc] = s;
+      if (l16 == 0) sc[(long long)tc * sc_ld + r] = s;
     }
   }
 }
@@ -143,14 +154,15 @@ struct alignas(64) Fp8Args {
   CUtensorMap tmA_routed;
   CUtensorMap tmA_shared;
   CUtensorMap tmB;
+  CUtensorMap tmS_routed;  // activation scales [KB][ld] (row index as in tmA_routed), box {132, 1}
+  CUtensorMap tmS_shared;  // the same for tmA_shared's rows
   const int32_t* offsets;
-  const float* sa_routed;  // [rows, KB] activation scales (row index as in tmA_routed)
-  const float* sa_shared;  // [rows, KB] (row index as in tmA_shared)
   const float* sw;         // [(N+1) * n_acc / 128, KB] weight block scales
   uint8_t* q_routed;       // GEMM1: h codes, row (offsets[g] + r)
   uint8_t* q_shared;       // GEMM1: h codes, row r
-  float* qs_routed;        // GEMM1: h scales [row, out_ld/128]
-  float* qs_shared;
+  float* qs_routed;        // GEMM1: h scales, block-major [out_ld/128][qs_ld], routed rows
+  float* qs_shared;        // ... shared-expert rows (same array, column TK onwards)
+  long long qs_ld;
   __nv_bfloat16* y_routed;  // GEMM2 outputs
   __nv_bfloat16* y_shared;
   uint32_t* status;
@@ -163,7 +175,8 @@ struct alignas(64) Fp8Args {
 };
 
 constexpr size_t fp8_smem_bytes(int groups) {
-  return 1024 + (size_t)FStages * FStageBytes + 512 + 2 * 4 * FBM * 4 + (size_t)(groups + 1) * 4;
+  return 1024 + (size_t)FStages * FStageBytes + (size_t)FScaleSlots * FScaleSlotBytes + 512 +
+         2 * 4 * FBM * 4 + (size_t)(groups + 1) * 4;
 }
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
@@ -174,15 +187,19 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)FStages * FStageBytes);
+  float* sc_ring = reinterpret_cast<float*>(base + (size_t)FStages * FStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)FStages * FStageBytes +
+                                               (size_t)FScaleSlots * FScaleSlotBytes);
   uint64_t* full = bars;                  // [FStages]
   uint64_t* empty = bars + FStages;       // [FStages]
   uint64_t* sfull = bars + 2 * FStages;   // [2] slice buffer written
   uint64_t* sempty = sfull + 2;           // [2] slice buffer drained (8 warps)
   uint64_t* xbar = sempty + 2;            // [2] amax exchange (8 warps)
   uint64_t* drain = xbar + 2;             // [1]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  float* xchg = reinterpret_cast<float*>(base + (size_t)FStages * FStageBytes + 512);  // [2][4][128]
+  uint64_t* scfull = drain + 1;           // [FScaleSlots] scale box landed
+  uint64_t* scempty = scfull + FScaleSlots;  // [FScaleSlots] scale box read (16 warps)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(scempty + FScaleSlots);
+  float* xchg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);  // [2][4][128]
   int* tile_start = reinterpret_cast<int*>(xchg + 2 * 4 * FBM);
 
   const int tid = threadIdx.x;
@@ -202,6 +219,10 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       mbar_init(&xbar[a], FEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int c = 0; c < FScaleSlots; ++c) {
+      mbar_init(&scfull[c], 1);
+      mbar_init(&scempty[c], FEpiWarps);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -257,17 +278,23 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       tma_prefetch_desc(&args.tmA_routed);
       tma_prefetch_desc(&args.tmA_shared);
       tma_prefetch_desc(&args.tmB);
+      tma_prefetch_desc(&args.tmS_routed);
+      tma_prefetch_desc(&args.tmS_shared);
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_parity = 0;
+      uint32_t sslice = 0, sc_issued = 0, sc_parity = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int g, n, m;
         decode(tile, g, n, m);
         const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
+        const CUtensorMap* smap = (g < args.N) ? &args.tmS_routed : &args.tmS_shared;
         const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * FBM;
         const int brow = g * args.n_acc + n * FBN;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, FTimeoutNs)) {
+          const uint32_t cs = sslice % FScaleSlots, cph = (sslice / FScaleSlots) & 1u;
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, FTimeoutNs) ||
+              !mbar_wait_bounded(&scempty[cs], cph ^ 1u, args.status, FTimeoutNs)) {
             ok = false;
             break;
           }
@@ -275,8 +302,15 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           mbar_arrive_expect_tx(&full[stage], FStageBytes);
           tma_load_2d(sa, am, kb * FBK, arow, &full[stage]);
           tma_load_2d(sa + FABytes, &args.tmB, kb * FBK, brow, &full[stage]);
+          // this slice's activation scales for the tile's rows
+          mbar_arrive_expect_tx(&scfull[cs], FScaleBox * 4);
+          tma_load_2d(reinterpret_cast<uint8_t*>(sc_ring) + cs * FScaleSlotBytes, smap, arow & ~3,
+                      kb, &scfull[cs]);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          sc_issued |= 1u << cs;
+          sc_parity = (sc_parity & ~(1u << cs)) | (cph << cs);
+          ++sslice;
           if (++stage == FStages) {
             stage = 0;
             phase ^= 1u;
@@ -287,6 +321,9 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
         for (int s = 0; s < FStages; ++s)
           if ((issued >> s) & 1u)
             mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.status, FTimeoutNs / 8);
+        for (int c = 0; c < FScaleSlots; ++c)
+          if ((sc_issued >> c) & 1u)
+            mbar_wait_bounded(&scfull[c], (sc_parity >> c) & 1u, args.status, FTimeoutNs / 8);
       }
     }
   } else if (warp == 1) {
@@ -342,10 +379,9 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       const int r = m * FBM + row;
       const bool valid =
           r < rows_g && (g == args.N || args.offsets[g] + r < args.rows_routed);
-      const long long arow_idx =
-          (g < args.N) ? (long long)args.offsets[g] + r : (long long)args.a_shared_row0 + r;
-      const float* sa_row = ((g < args.N) ? args.sa_routed : args.sa_shared) +
-                            (valid ? arow_idx : 0) * KB;
+      // the scale box starts at the tile's first row rounded down to 4
+      const int arow0 = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * FBM;
+      const int sc_off = (arow0 & 3) + row;
       const long long wblk0 = ((long long)g * args.n_acc + (long long)n * FBN) / QB;
       // weight-block scales this warp needs: GEMM1 gate (block 0) and up
       // (block 1); GEMM2 the block of its 64 columns
@@ -354,13 +390,21 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-      // scales are read one slice ahead so their latency hides behind a slice
-      float sa_n = valid ? __ldg(sa_row) : 0.f, swA_n = __ldg(swA), swB_n = __ldg(swB);
+      // weight-block scales are read one slice ahead (the same address for the
+      // whole warp, so they come through L1)
+      float swA_n = __ldg(swA), swB_n = __ldg(swB);
       for (int kb = 0; kb < KB; ++kb, ++slice) {
         const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
-        const float sA = sa_n * swA_n, sB = sa_n * swB_n;
+        const uint32_t cs = slice % FScaleSlots, cph = (slice / FScaleSlots) & 1u;
+        if (!mbar_wait_bounded(&scfull[cs], cph, args.status, FTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        const float sa = sc_ring[cs * (FScaleSlotBytes / 4) + sc_off];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&scempty[cs]);
+        const float sA = sa * swA_n, sB = sa * swB_n;
         if (kb + 1 < KB) {
-          sa_n = valid ? __ldg(sa_row + kb + 1) : 0.f;
           swA_n = __ldg(swA + kb + 1);
           swB_n = __ldg(swB + kb + 1);
         }
@@ -434,10 +478,8 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
             reinterpret_cast<uint4*>(qrow)[v] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
           if (sub == 0) {
-            float* srow = (g < args.N) ? args.qs_routed + ((long long)args.offsets[g] + r) *
-                                                            (args.out_ld / QB)
-                                       : args.qs_shared + (long long)r * (args.out_ld / QB);
-            srow[n] = scale;
+            float* qs = (g < args.N) ? args.qs_routed + args.offsets[g] : args.qs_shared;
+            qs[(long long)n * args.qs_ld + r] = scale;
           }
         }
       } else {
@@ -483,13 +525,13 @@ cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
-                              cudaStream_t st) {
+                              long long sc_ld, cudaStream_t st) {
   const long long tiles = rows * (d / QB);
   long long blocks = (tiles * 16 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
   quant_rows_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rows, d,
-                                                 q, sc);
+                                                 q, sc, sc_ld);
   return note_cuda(cudaGetLastError(), "1x128 quantisation launch");
 }
 
@@ -525,25 +567,29 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
   const uint64_t TK = (uint64_t)s.T * s.K;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
 
+  // scale arrays are block-major [K/128][ld]
+  const long long ld_routed = scale_ld((long long)TK), ld_x = scale_ld(s.T);
+  const long long ld_h = scale_ld((long long)TK + s.T);
   // the shared expert reads x: quantise it per 1x128 tile first
-  if (launch_quant_rows(x, s.T, s.d, xq, xs, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_quant_rows(x, s.T, s.d, xq, xs, ld_x, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   Fp8Args g1{};
   bool ok = make_map(&g1.tmA_routed, x_perm, U8, 1, s.d, TK, FBK, FBM) &&
             make_map(&g1.tmA_shared, xq, U8, 1, s.d, s.T, FBK, FBM) &&
-            make_map(&g1.tmB, w13, U8, 1, s.d, (uint64_t)(s.N + 1) * 2 * s.f, FBK, FBN);
+            make_map(&g1.tmB, w13, U8, 1, s.d, (uint64_t)(s.N + 1) * 2 * s.f, FBK, FBN) &&
+            make_map_f32_rows(&g1.tmS_routed, x_perm_scales, ld_routed, s.d / QB, FScaleBox) &&
+            make_map_f32_rows(&g1.tmS_shared, xs, ld_x, s.d / QB, FScaleBox);
   if (!ok) {
     note_text("fp8 GEMM1: tensor-map encoding failed");
     return MOE_ERR_CUDA;
   }
   g1.offsets = offsets;
-  g1.sa_routed = x_perm_scales;
-  g1.sa_shared = xs;
   g1.sw = w13_scales;
   g1.q_routed = Hq;
   g1.q_shared = Hq + TK * s.f;
   g1.qs_routed = Hs;
-  g1.qs_shared = Hs + TK * (s.f / QB);
+  g1.qs_shared = Hs + TK;
+  g1.qs_ld = ld_h;
   g1.status = status;
   g1.N = s.N;
   g1.T = s.T;
@@ -557,14 +603,14 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
   Fp8Args g2{};
   ok = make_map(&g2.tmA_routed, Hq, U8, 1, s.f, TK + s.T, FBK, FBM) &&
        make_map(&g2.tmA_shared, Hq, U8, 1, s.f, TK + s.T, FBK, FBM) &&
-       make_map(&g2.tmB, w2, U8, 1, s.f, (uint64_t)(s.N + 1) * s.d, FBK, FBN);
+       make_map(&g2.tmB, w2, U8, 1, s.f, (uint64_t)(s.N + 1) * s.d, FBK, FBN) &&
+       make_map_f32_rows(&g2.tmS_routed, Hs, ld_h, s.f / QB, FScaleBox) &&
+       make_map_f32_rows(&g2.tmS_shared, Hs, ld_h, s.f / QB, FScaleBox);
   if (!ok) {
     note_text("fp8 GEMM2: tensor-map encoding failed");
     return MOE_ERR_CUDA;
   }
   g2.offsets = offsets;
-  g2.sa_routed = Hs;
-  g2.sa_shared = Hs;
   g2.sw = w2_scales;
   g2.y_routed = static_cast<__nv_bfloat16*>(y_perm);
   g2.y_shared = static_cast<__nv_bfloat16*>(y_shared);

@@ -44,6 +44,11 @@ inline int pack_block(int f) { return f < 128 ? f : 128; }
 cudaError_t note_cuda(cudaError_t e, const char* where);
 void note_text(const char* what);
 
+// FP8 activation scales are stored block-major, [K/128][ld] with ld = the row
+// count rounded up to 4, so the 128 scales of a token tile at one K block are
+// contiguous and one TMA copy (16-byte aligned row pitch) brings them in.
+inline long long scale_ld(long long rows) { return (rows + 3) & ~3LL; }
+
 // ---- host helpers (tma_host.cu) ------------------------------------------------
 // 2-D row-major tensor [rows, inner] with a (box_inner x box_rows) box and the
 // 128-byte swizzle; out-of-range rows read as zero.
@@ -53,6 +58,10 @@ bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t 
 // dims 1..rank-1 and the box; 128-byte swizzle, out-of-range elements read as zero.
 bool make_map_nd(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int rank,
                  const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
+// fp32 matrix [rows, inner] (inner a multiple of 4) read one row segment at a
+// time: box {box_inner, 1}, no swizzle, out-of-range elements read as zero.
+bool make_map_f32_rows(CUtensorMap* map, const float* ptr, uint64_t inner, uint64_t rows,
+                       uint32_t box_inner);
 int num_sms();
 
 // ---- launchers (return cudaError_t of the launch) -----------------------------
@@ -90,6 +99,7 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
                        void* y_shared, void* ws, cudaStream_t st);
 // x [rows, d] bf16 -> E4M3 codes [rows, d] and fp32 scales [rows, d/128].
 cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
+                              long long sc_ld,
                               cudaStream_t st);
 cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const void* w2,
                                     void* w13_q, float* w13_scales, void* w2_q,

@@ -1,9 +1,14 @@
-// Issue-rate probe for tcgen05.mma: SM cycles per MMA instruction with both
+// Issue-rate probes for the tensor-core path.
+// (1) tcgen05.mma: SM cycles per MMA instruction with both
 // operands resident in shared memory (no loads, no epilogue), for the
 // instruction shapes the expert GEMMs use.  One thread issues `iters` K steps;
 // each K step issues `chains` MMAs into separate accumulators (chains = 1 is a
 // dependent accumulation chain, as in a GEMM main loop).  Operand values are
-// zero: only the timing is of interest.  Prints one JSON line per shape.
+// zero: only the timing is of interest.
+// (2) tcgen05.ld: cycles per round of `inflight` loads of 32 lanes x W columns
+// followed by one tcgen05.wait::ld, per warp, with 4 or 16 warps per CTA; gives
+// the load latency (inflight = 1) and the TMEM read bandwidth per SM.
+// Prints one JSON line per configuration.
 // Build: nvcc -O3 -std=c++17 -gencode arch=compute_100a,code=sm_100a mma_rate.cu
 #include <cstdint>
 #include <cstdio>
@@ -78,6 +83,69 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int M, int N, int chai
   }
 }
 
+template <int W>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, uint32_t (&r)[W]) {
+  if constexpr (W == 16) {
+    tmem_ld16(taddr, r);
+  } else {
+#pragma unroll
+    for (int h = 0; h < W / 32; ++h) {
+      uint32_t (&part)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32 * h]);
+      tmem_ld32(taddr + 32 * h, part);
+    }
+  }
+}
+
+__device__ float g_sink;
+
+template <int W, int kInflight>
+__global__ void __launch_bounds__(512, 1) tmem_ld_kernel(int iters) {
+  __shared__ uint32_t holder;
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    tmem_alloc(&holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = holder + ((uint32_t)((warp & 3) * 32) << 16);
+  float acc = 0.f;
+  const unsigned long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    uint32_t v[kInflight][W];
+#pragma unroll
+    for (int j = 0; j < kInflight; ++j) ld_cols<W>(tb + (uint32_t)(((it + j) * W) & 511), v[j]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < kInflight; ++j) acc += __uint_as_float(v[j][0] ^ v[j][W - 1]);
+  }
+  const unsigned long long cyc = clock64() - t0;
+  if ((threadIdx.x & 31) == 0 && warp == 0) g_cycles = cyc;
+  if (acc == 12345.f) g_sink = acc;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(holder, 512);
+  }
+}
+
+template <int W, int kInflight>
+static int run_ld(int warps) {
+  const int iters = 4000;
+  tmem_ld_kernel<W, kInflight><<<1, 32 * warps>>>(iters);
+  if (cudaDeviceSynchronize() != cudaSuccess) return 1;
+  unsigned long long cyc = 0;
+  cudaMemcpyFromSymbol(&cyc, g_cycles, sizeof(cyc));
+  const double per = (double)cyc / iters;
+  const double bytes = (double)warps * kInflight * W * 32 * 4;
+  printf("{\"kind\": \"tmem_ld\", \"warps\": %d, \"cols\": %d, \"inflight\": %d, "
+         "\"cycles_per_round\": %.1f, \"bytes_per_sm_cycle\": %.0f}\n",
+         warps, W, kInflight, per, bytes / per);
+  return 0;
+}
+
 template <bool kFp8, bool kPair>
 static int run(int M, int N, int chains) {
   const int iters = 2000;
@@ -121,5 +189,13 @@ int main() {
       bad |= run<true, false>(128, N, c);
       bad |= run<false, true>(256, N, c);
     }
+  for (int w : {4, 16}) {
+    bad |= run_ld<16, 1>(w);
+    bad |= run_ld<16, 2>(w);
+    bad |= run_ld<16, 4>(w);
+    bad |= run_ld<32, 1>(w);
+    bad |= run_ld<32, 2>(w);
+    bad |= run_ld<64, 1>(w);
+  }
   return bad;
 }

@@ -57,6 +57,20 @@ bool make_map_nd(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int 
   return r == CUDA_SUCCESS;
 }
 
+bool make_map_f32_rows(CUtensorMap* map, const float* ptr, uint64_t inner, uint64_t rows,
+                       uint32_t box_inner) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {box_inner, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   static int n = 0;
   if (n == 0) {

@@ -35,7 +35,8 @@ class MoELayer:
         self.slot = torch.empty(s.T, s.K, **i32)
         pdt = torch.float8_e4m3fn if s.dtype == L.DTYPE_E4M3 else xdt
         self.x_perm = torch.empty(s.T * s.K, s.d, dtype=pdt, device=dev)
-        self.x_perm_scales = (torch.empty(s.T * s.K, s.d // 128, dtype=torch.float32, device=dev)
+        self.x_perm_scales = (torch.empty(s.d // 128, (s.T * s.K + 3) // 4 * 4, dtype=torch.float32,
+                                          device=dev)
                               if s.dtype == L.DTYPE_E4M3 else None)
         self.y_perm = torch.empty(s.T * s.K, s.d, dtype=xdt, device=dev)
         self.y_shared = torch.empty(s.T, s.d, dtype=xdt, device=dev)

@@ -229,7 +229,10 @@ def test_small_fp8_layer_full(M, T):
     # dispatched rows are quantised per 1x128 tile exactly as the oracle does
     codes, scales = oracle.quant_rows_1x128(x[d["perm_tok"]])
     np.testing.assert_array_equal(layer.x_perm.view(torch.uint8).cpu().numpy(), codes)
-    np.testing.assert_array_equal(layer.x_perm_scales.cpu().numpy(), scales)
+    # scales are stored block-major, [d/128, T*K rounded up to 4]
+    got = layer.x_perm_scales.cpu().numpy()
+    assert got.shape == (cfg.d // 128, (cfg.T * cfg.K + 3) // 4 * 4)
+    np.testing.assert_array_equal(got[:, :cfg.T * cfg.K], scales.T)
     get = S.host_weights(cfg)
     yp = layer.y_perm.float().cpu().numpy()
     for e in range(cfg.N):
