@@ -16,11 +16,11 @@
 // the tensor core fills one while the other is drained).  Sixteen epilogue
 // warps -- four per TMEM lane quadrant, each owning 64 of the 256 columns --
 // fold each slice into fp32 register sums with the product of the two
-// scales.  This per-slice promotion is the tcgen05 counterpart of the
-// article's "accumulate at an interval in fp32 on the CUDA cores" (the
-// kaiyunto.com walk-through describes the same H800 step); on sm_100 the
-// partial sums already sit in TMEM in fp32, so only the scale product is
-// applied per slice.
+// scales (packed fp32x2 FMAs).  This per-slice promotion is the tcgen05
+// counterpart of the article's "accumulate at an interval in fp32 on the CUDA
+// cores" (the kaiyunto.com walk-through describes the same H800 step); on
+// sm_100 the partial sums already sit in TMEM in fp32, so only the scale
+// product is applied per slice.
 //
 // GEMM1 epilogue: h = silu(gate) * up for the 128 hidden features of the
 // tile (gate and up columns of one feature lie in the same tile and thread
@@ -177,6 +177,15 @@ struct alignas(64) Fp8Args {
 constexpr size_t fp8_smem_bytes(int groups) {
   return 1024 + (size_t)FStages * FStageBytes + (size_t)FScaleSlots * FScaleSlotBytes + 512 +
          2 * 4 * FBM * 4 + (size_t)(groups + 1) * 4;
+}
+
+// a0 += x0 * s and a1 += x1 * s as one packed fp32x2 FMA (two independent
+// round-to-nearest FMAs, the same results as two fmaf, half the issue slots)
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float x0, float x1, float s) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(s));
 }
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
@@ -426,8 +435,9 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           tmem_ld16(taddr + col, p);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            acc[c * 16 + i] = fmaf(__uint_as_float(p[i]), sc, acc[c * 16 + i]);
+          for (int i = 0; i < 16; i += 2)
+            ffma2(acc[c * 16 + i], acc[c * 16 + i + 1], __uint_as_float(p[i]),
+                  __uint_as_float(p[i + 1]), sc);
         }
         tc_fence_before();
         __syncwarp();
