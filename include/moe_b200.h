@@ -107,8 +107,9 @@ int moe_check_shape(const moe_shape* shape);
 
 /* Bytes of scratch every entry point of this shape may use (one buffer serves
  * all of them; calls on the same stream may share it).  The first 256 bytes
- * hold the device status word: zero them once after allocating
- * (moe_workspace_init) and read them with moe_read_device_status.
+ * hold the device status word and the expert GEMMs' work counters (each
+ * launch leaves them at zero): zero them once after allocating
+ * (moe_workspace_init) and read the status with moe_read_device_status.
  * Returns 0 for an invalid shape. */
 size_t moe_workspace_size(const moe_shape* shape);
 

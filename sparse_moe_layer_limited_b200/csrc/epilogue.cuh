@@ -1,0 +1,21 @@
+// Epilogue helpers shared by the bf16 expert GEMM kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace moe {
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
+
+// 32 fp32 values -> 32 bf16 (round to nearest even), four 16-byte stores.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) {
+  uint4 w[4];
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = w[i];
+}
+
+}  // namespace moe

@@ -49,6 +49,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "epilogue.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -92,18 +93,6 @@ struct alignas(64) GemmArgs {
   int n_valid; // columns to store (score epilogue)
   int k_splits; // K ranges computed by separate units (score epilogue; else 1)
 };
-
-__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
-
-__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) {
-  uint4 w[4];
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) d4[i] = w[i];
-}
 
 template <int kEpi, int kBN>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
@@ -401,11 +390,16 @@ __global__ void router_split_kernel(const float* __restrict__ R, int N, int d,
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                        const void* x, const void* w13, const void* w2, void* y_perm,
                        void* y_shared, void* ws, cudaStream_t st) {
-  static const bool pair = [] {
+  // MOE_BF16_GEMM selects the expert GEMM kernel: "dual" (two token tiles per
+  // weight tile, gemm_dual.cu), "pair" (CTA pairs, gemm2sm.cu); default: this file's
+  static const int kind = [] {
     const char* v = std::getenv("MOE_BF16_GEMM");
-    return v != nullptr && std::strcmp(v, "pair") == 0;
+    if (v != nullptr && std::strcmp(v, "pair") == 0) return 2;
+    if (v != nullptr && std::strcmp(v, "dual") == 0) return 1;
+    return 0;
   }();
-  if (pair) return launch_ffn_tc_bf16_pair(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
+  if (kind == 2) return launch_ffn_tc_bf16_pair(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
+  if (kind == 1) return launch_ffn_tc_bf16_dual(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
   const WsLayout L = ws_layout(s);
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(w + L.h);

@@ -90,6 +90,9 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
                        const void* x, const void* w13, const void* w2, void* y_perm,
                        void* y_shared, void* ws, cudaStream_t st);
 // The same two GEMMs on CTA pairs (tcgen05 cta_group::2), gemm2sm.cu.
+int launch_ffn_tc_bf16_dual(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                            const void* x, const void* w13, const void* w2, void* y_perm,
+                            void* y_shared, void* ws, cudaStream_t st);
 int launch_ffn_tc_bf16_pair(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                             const void* x, const void* w13, const void* w2, void* y_perm,
                             void* y_shared, void* ws, cudaStream_t st);

@@ -3,7 +3,10 @@
 // operands resident in shared memory (no loads, no epilogue), for the
 // instruction shapes the expert GEMMs use.  One thread issues `iters` K steps;
 // each K step issues `chains` MMAs into separate accumulators (chains = 1 is a
-// dependent accumulation chain, as in a GEMM main loop).  Operand values are
+// dependent accumulation chain, as in a GEMM main loop).  With `blocked`, a
+// 64-wide K stage issues its four K steps on one accumulator before the next
+// (the order a kernel sharing one weight tile between two token tiles uses);
+// otherwise the accumulators alternate every K step.  Operand values are
 // zero: only the timing is of interest.
 // (2) tcgen05.ld: cycles per round of `inflight` loads of 32 lanes x W columns
 // followed by one tcgen05.wait::ld, per warp, with 4 or 16 warps per CTA; gives
@@ -23,7 +26,8 @@ __device__ unsigned long long g_cycles;
 __device__ uint32_t g_err;
 
 template <bool kFp8, bool kPair>
-__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int M, int N, int chains, int iters) {
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int M, int N, int chains, int iters,
+                                                          int blocked) {
   extern __shared__ uint8_t sm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -58,10 +62,11 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int M, int N, int chai
     const uint32_t id = kFp8 ? idesc_e4m3_f32(M, N) : idesc_bf16_f32(M, N);
     const unsigned long long t0 = clock64();
     for (int it = 0; it < iters; ++it)
-      for (int k = 0; k < 4; ++k)
-        for (int c = 0; c < chains; ++c) {
+      for (int j = 0; j < 4 * chains; ++j) {
+          const int k = blocked ? j % 4 : j / chains, c = blocked ? j / 4 : j % chains;
           const uint64_t ad = smem_desc_sw128(a0 + 32 * k), bd = smem_desc_sw128(b0 + 32 * k);
-          const uint32_t d = tb + 128u * (uint32_t)c, acc = (it | k) != 0;
+          // disjoint accumulators: chain c at column c * max(N, 128)
+          const uint32_t d = tb + (uint32_t)(c * (N > 128 ? N : 128)), acc = (it | k) != 0;
           if (kPair) {
             mma_bf16_2sm(d, ad, bd, id, acc);
           } else if (kFp8) {
@@ -147,7 +152,7 @@ static int run_ld(int warps) {
 }
 
 template <bool kFp8, bool kPair>
-static int run(int M, int N, int chains) {
+static int run(int M, int N, int chains, int blocked = 0, bool print = true) {
   const int iters = 2000;
   const size_t smem = 50 * 1024;
   auto kern = mma_rate_kernel<kFp8, kPair>;
@@ -163,7 +168,7 @@ static int run(int M, int N, int chains) {
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, M, N, chains, iters) != cudaSuccess) return 1;
+  if (cudaLaunchKernelEx(&cfg, kern, M, N, chains, iters, blocked) != cudaSuccess) return 1;
   if (cudaDeviceSynchronize() != cudaSuccess) return 1;
   unsigned long long cyc = 0;
   uint32_t err = 0;
@@ -173,22 +178,32 @@ static int run(int M, int N, int chains) {
   // MACs per SM and K step: M rows (M/2 per SM for a pair) x N x K
   const double k = kFp8 ? 32.0 : 16.0;
   const double macs = (kPair ? M / 2 : M) * (double)N * k * chains;
-  printf("{\"kind\": \"%s\", \"cta_group\": %d, \"M\": %d, \"N\": %d, \"chains\": %d, "
-         "\"cycles_per_mma\": %.1f, \"macs_per_sm_cycle\": %.0f, \"status\": %u}\n",
-         kFp8 ? "f8f6f4" : "f16", kPair ? 2 : 1, M, N, chains, per_step / chains,
+  if (print)
+    printf("{\"kind\": \"%s\", \"cta_group\": %d, \"M\": %d, \"N\": %d, \"chains\": %d, "
+         "\"blocked\": %d, \"cycles_per_mma\": %.1f, \"macs_per_sm_cycle\": %.0f, "
+         "\"status\": %u}\n",
+         kFp8 ? "f8f6f4" : "f16", kPair ? 2 : 1, M, N, chains, blocked, per_step / chains,
          macs / per_step, err);
   return err != 0;
 }
 
 int main() {
   int bad = 0;
+  // the tensor pipe of an idle GPU runs slower for a while after it wakes:
+  // keep it busy for about a second before measuring anything
+  for (int i = 0; i < 200; ++i) bad |= run<false, false>(128, 256, 1, 0, false);
   for (int N : {256, 128, 64, 16})
     for (int c : {1, 2, 3}) {
+      if (N > 128 && c > 2) continue;  // accumulators must fit in 512 columns
       bad |= run<false, false>(128, N, c);
       bad |= run<false, false>(64, N, c);
       bad |= run<true, false>(128, N, c);
       bad |= run<false, true>(256, N, c);
     }
+  bad |= run<false, false>(128, 256, 2, 1);
+  bad |= run<true, false>(128, 256, 2, 1);
+  bad |= run<false, true>(256, 256, 2, 1);
+  bad |= run<false, false>(128, 128, 3, 1);
   for (int w : {4, 16}) {
     bad |= run_ld<16, 1>(w);
     bad |= run_ld<16, 2>(w);
