@@ -11,8 +11,8 @@
 // a token tile of at most 64 rows -- N=256).  Operand bytes per MMA cycle
 // drop from 96 to 64 against one token tile per weight tile, and issuing
 // each accumulator's K steps back to back keeps the tensor pipe at its full
-// rate (128 cycles per N=256 MMA in the issue-rate probe,
-// csrc/probe/mma_rate.cu).  An expert with an odd number of token tiles ends
+// rate (the issue-rate probe, csrc/probe/mma_rate.cu: 128 cycles per N=256
+// MMA this way, 149.5 when the two accumulators alternate every K step).  An expert with an odd number of token tiles ends
 // with a one-tile unit, so a ragged tail costs one tile's MMA work, as in the
 // one-tile kernel.
 //

@@ -61,20 +61,31 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int M, int N, int chai
     const uint32_t a0 = smem_u32(base), b0 = a0 + 16384;
     const uint32_t id = kFp8 ? idesc_e4m3_f32(M, N) : idesc_bf16_f32(M, N);
     const unsigned long long t0 = clock64();
-    for (int it = 0; it < iters; ++it)
-      for (int j = 0; j < 4 * chains; ++j) {
-          const int k = blocked ? j % 4 : j / chains, c = blocked ? j / 4 : j % chains;
-          const uint64_t ad = smem_desc_sw128(a0 + 32 * k), bd = smem_desc_sw128(b0 + 32 * k);
-          // disjoint accumulators: chain c at column c * max(N, 128)
-          const uint32_t d = tb + (uint32_t)(c * (N > 128 ? N : 128)), acc = (it | k) != 0;
-          if (kPair) {
-            mma_bf16_2sm(d, ad, bd, id, acc);
-          } else if (kFp8) {
-            mma_e4m3(d, ad, bd, id, acc);
-          } else {
-            mma_bf16(d, ad, bd, id, acc);
-          }
-        }
+    // the issuing thread must stay far below one MMA's duration per
+    // instruction: plain loop nests, no division by a runtime value
+    auto issue = [&](int k, int c, uint32_t acc) {
+      const uint64_t ad = smem_desc_sw128(a0 + 32 * k), bd = smem_desc_sw128(b0 + 32 * k);
+      // disjoint accumulators: chain c at column c * max(N, 128)
+      const uint32_t d = tb + (uint32_t)(c * (N > 128 ? N : 128));
+      if (kPair) {
+        mma_bf16_2sm(d, ad, bd, id, acc);
+      } else if (kFp8) {
+        mma_e4m3(d, ad, bd, id, acc);
+      } else {
+        mma_bf16(d, ad, bd, id, acc);
+      }
+    };
+    for (int it = 0; it < iters; ++it) {
+      if (blocked) {
+        for (int c = 0; c < chains; ++c)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) issue(k, c, (it | k) != 0);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          for (int c = 0; c < chains; ++c) issue(k, c, (it | k) != 0);
+      }
+    }
     if (kPair) mma_commit_2sm(&bar); else mma_commit(&bar);
     mbar_wait_bounded(&bar, 0, &g_err, 2000000000ull);
     g_cycles = clock64() - t0;
