@@ -36,9 +36,9 @@
 // Activation scales are block-major ([K/128][rows rounded up to 4]); for each
 // slice the producer copies the tile's 128 scales (a 132-float box starting at
 // the tile's first row rounded down to 4) into a ring of eight shared-memory
-// slots that the epilogue releases, so the promotion reads its per-row scale
-// from shared memory.  Weight-block scales are the same for a whole warp and
-// come through L1.
+// slots that the epilogue releases, together with the slice's two weight-block
+// scales (two 4-byte cp.async copies completing on the same barrier), so the
+// promotion reads every scale from shared memory.
 // All waits are bounded (~2 s) and set the device status word on expiry.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -300,6 +300,8 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
         const CUtensorMap* smap = (g < args.N) ? &args.tmS_routed : &args.tmS_shared;
         const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * FBM;
         const int brow = g * args.n_acc + n * FBN;
+        // the tile's two 128-row weight blocks, scales [block][KB]
+        const float* sw_tile = args.sw + ((long long)brow / QB) * KB;
         for (int kb = 0; kb < KB; ++kb) {
           const uint32_t cs = sslice % FScaleSlots, cph = (sslice / FScaleSlots) & 1u;
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, FTimeoutNs) ||
@@ -311,10 +313,16 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           mbar_arrive_expect_tx(&full[stage], FStageBytes);
           tma_load_2d(sa, am, kb * FBK, arow, &full[stage]);
           tma_load_2d(sa + FABytes, &args.tmB, kb * FBK, brow, &full[stage]);
-          // this slice's activation scales for the tile's rows
+          // this slice's scales: the two weight-block scales by cp.async, whose
+          // pending arrival is registered on the slot's barrier before the
+          // expect-tx arrival (so the phase cannot complete without them), then
+          // the activation box for the tile's rows by TMA
+          uint8_t* slot_dst = reinterpret_cast<uint8_t*>(sc_ring) + cs * FScaleSlotBytes;
+          cp_async_4(slot_dst + FScaleBox * 4, sw_tile + kb);
+          cp_async_4(slot_dst + FScaleBox * 4 + 4, sw_tile + KB + kb);
+          cp_async_mbar_arrive(&scfull[cs]);
           mbar_arrive_expect_tx(&scfull[cs], FScaleBox * 4);
-          tma_load_2d(reinterpret_cast<uint8_t*>(sc_ring) + cs * FScaleSlotBytes, smap, arow & ~3,
-                      kb, &scfull[cs]);
+          tma_load_2d(slot_dst, smap, arow & ~3, kb, &scfull[cs]);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           sc_issued |= 1u << cs;
@@ -391,17 +399,14 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       // the scale box starts at the tile's first row rounded down to 4
       const int arow0 = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * FBM;
       const int sc_off = (arow0 & 3) + row;
-      const long long wblk0 = ((long long)g * args.n_acc + (long long)n * FBN) / QB;
-      // weight-block scales this warp needs: GEMM1 gate (block 0) and up
-      // (block 1); GEMM2 the block of its 64 columns
-      const float* swA = args.sw + (kEpi == kFEpiSwiGLUQuant ? wblk0 : wblk0 + (sub >> 1)) * KB;
-      const float* swB = args.sw + (kEpi == kFEpiSwiGLUQuant ? wblk0 + 1 : wblk0 + (sub >> 1)) * KB;
+      // the slot's two weight-block scales follow the activation box: GEMM1
+      // uses the gate block for its first 32 columns and the up block for the
+      // rest, GEMM2 the block of its 64 columns
+      const int wA = (kEpi == kFEpiSwiGLUQuant) ? 0 : (sub >> 1);
+      const int wB = (kEpi == kFEpiSwiGLUQuant) ? 1 : (sub >> 1);
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-      // weight-block scales are read one slice ahead (the same address for the
-      // whole warp, so they come through L1)
-      float swA_n = __ldg(swA), swB_n = __ldg(swB);
       for (int kb = 0; kb < KB; ++kb, ++slice) {
         const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
         const uint32_t cs = slice % FScaleSlots, cph = (slice / FScaleSlots) & 1u;
@@ -409,14 +414,11 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           ok = false;
           break;
         }
-        const float sa = sc_ring[cs * (FScaleSlotBytes / 4) + sc_off];
+        const float* slot_sc = sc_ring + cs * (FScaleSlotBytes / 4);
+        const float sa = slot_sc[sc_off];
+        const float sA = sa * slot_sc[FScaleBox + wA], sB = sa * slot_sc[FScaleBox + wB];
         __syncwarp();
         if (lane == 0) mbar_arrive(&scempty[cs]);
-        const float sA = sa * swA_n, sB = sa * swB_n;
-        if (kb + 1 < KB) {
-          swA_n = __ldg(swA + kb + 1);
-          swB_n = __ldg(swB + kb + 1);
-        }
         if (!mbar_wait_bounded(&sfull[sb], sph, args.status, FTimeoutNs)) {
           ok = false;
           break;
