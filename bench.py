@@ -542,9 +542,15 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
 
     P = peaks()
     fp8 = cfg.dtype == "e4m3"
-    # FP8 peak = the measured bf16 peak x the nominal dense ratio (4.5 / 2.25 PFLOP/s)
-    peak = P["bf16"] * (2.0 if fp8 else 1.0)
-    peak_src = P["source"] + (" bf16 burst x nominal fp8/bf16 ratio 2" if fp8 else " burst")
+    # The expert GEMMs are timed inside back-to-back layer steps (the clock
+    # settles under the power cap), so the denominator is the measured
+    # sustained bf16 GEMM rate; the burst fraction is reported beside it.  FP8
+    # peak = the measured bf16 figure x the nominal dense ratio (4.5 / 2.25 PFLOP/s).
+    ratio = 2.0 if fp8 else 1.0
+    peak = P["bf16_sustained"] * ratio
+    peak_burst = P["bf16"] * ratio
+    peak_src = P["source"] + (" bf16 sustained x nominal fp8/bf16 ratio 2" if fp8
+                              else " sustained (kernel timed inside a long step loop)")
     ffn_ms = statistics.mean(per_phase["experts"])
     wbytes = 1 if fp8 else 2
     fl = flops_per_forward(cfg)
@@ -556,7 +562,8 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
         achieved = ffn_flops(cfg) / (ffn_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, GEMM2)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": peak_src, "traffic": None}
+                "peak_source": peak_src, "peak_burst": peak_burst,
+                "frac_of_burst": achieved / peak_burst, "traffic": None}
         if cfg.name == "v3_bf16" and cfg.T == 8192 and cfg.N == 256 and not pair_gemm():
             # DRAM bytes of one moe_expert_ffn call (GEMM1 + GEMM2), from the ncu
             # capture of the same kernels on the T=1024 / 32+1-expert case
