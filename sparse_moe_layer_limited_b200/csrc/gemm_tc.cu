@@ -234,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
         decode(tile, g, n, m, mt);
         const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
         // a tile with at most 64 real rows (an expert's ragged tail) runs the
-        // M=64 MMA: half the tensor work for the same weight stream
+        // M=64 MMA: the tensor pipe takes as long as for M=128 (tcgen05
+        // issue-rate probe), but half the products are computed and drained
         const int rows_g = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
         const uint32_t idesc = idesc_bf16_f32(rows_g - m * BM <= 64 ? 64 : BM, kBN);
         const int acc = local & 1;
