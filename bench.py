@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--rows", type=int, default=256, help="rows per expert for --probe uniform")
     p.add_argument("--no-extra", action="store_true",
                    help="skip the FP8 and decode workloads reported beside the headline")
+    p.add_argument("--gather", choices=["on", "off"], default="off",
+                   help="bf16: GEMM1 gathers routed rows from x through perm_tok (on) or "
+                        "reads the permuted copy written by dispatch (off)")
     p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
     p.add_argument("--N", type=int, default=None, help="override routed experts (profiling)")
     return p.parse_args()
@@ -322,7 +325,9 @@ def run_probe(args, cfg):
 
 
 def main():
+    global GATHER
     args = parse()
+    GATHER = args.gather == "on"
     cfg = BY_NAME[args.config]
     if args.T:
         cfg = cfg.with_(T=args.T)
@@ -425,8 +430,7 @@ def run_e2e(M, s, layer, x, w13, w2, s13, s2, cfg, steps, stream):
                         layer.counts, layer.ws, stream)
             M.moe_dispatch(s, xb, layer.topk_idx, layer.counts, layer.offsets, layer.perm_tok,
                            layer.slot, layer.x_perm, layer.x_perm_scales, layer.ws, stream)
-            M.moe_expert_ffn(s, layer.x_perm, layer.x_perm_scales, layer.offsets, xb, w13, w2,
-                             s13, s2, layer.y_perm, layer.y_shared, layer.ws, stream)
+            layer.experts(xb, stream)
             M.moe_combine(s, layer.y_perm, layer.y_shared, layer.slot, layer.topk_gate, ys[b],
                           stream)
             M.moe_bias_update(s, layer.counts, layer.bias, cfg.gamma, stream)
@@ -450,6 +454,9 @@ def run_e2e(M, s, layer, x, w13, w2, s13, s2, cfg, steps, stream):
     e1.record(h2d)          # after the last download
     torch.cuda.synchronize()
     return e0.elapsed_time(e1)
+
+
+GATHER = False  # set from --gather in main()
 
 
 def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
@@ -485,7 +492,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
         x = sdev.x_bf16(cfg, 0, 0, dev)
     else:
         x = torch.from_numpy(gen.make_x(cfg)).to(torch.bfloat16).to(dev)
-    layer = M.MoELayer(s, router, bias, w13, w2, s13, s2, gamma=cfg.gamma)
+    layer = M.MoELayer(s, router, bias, w13, w2, s13, s2, gamma=cfg.gamma, gather=GATHER)
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream(dev)
@@ -502,8 +509,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
                        layer.slot, layer.x_perm, layer.x_perm_scales, layer.ws, stream)
         if ev is not None:
             ev[2].record(stream)
-        M.moe_expert_ffn(s, layer.x_perm, layer.x_perm_scales, layer.offsets, x, w13, w2,
-                         s13, s2, layer.y_perm, layer.y_shared, layer.ws, stream)
+        layer.experts(x, stream)
         if ev is not None:
             ev[3].record(stream)
         M.moe_combine(s, layer.y_perm, layer.y_shared, layer.slot, layer.topk_gate, layer.y,

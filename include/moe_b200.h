@@ -146,7 +146,9 @@ int moe_route(const moe_shape* shape, const void* x, const float* router_w, cons
  *   perm_tok   [T*K]   int32 out, token of each row
  *   slot       [T, K]  int32 out, row holding (t, topk_idx[t, k])
  *   x_perm     [T*K, d] out: bf16 copy of x rows (BF16), fp32 (FP32), or E4M3
- *                      codes (E4M3 mode, one byte per element)
+ *                      codes (E4M3 mode, one byte per element).  May be NULL
+ *                      in BF16 and FP32 modes: then only offsets, perm_tok and
+ *                      slot are written (for moe_expert_ffn_gathered)
  *   x_perm_scales [d/128, L] fp32 out, E4M3 mode only (NULL otherwise), with
  *                      L = T*K rounded up to a multiple of 4: the scale
  *                      amax/448 of row r's 1x128 tile j is at [j, r] ([P1]
@@ -176,6 +178,19 @@ int moe_expert_ffn(const moe_shape* shape, const void* x_perm, const float* x_pe
                    const int32_t* offsets, const void* x, const void* w13, const void* w2,
                    const float* w13_scales, const float* w2_scales, void* y_perm,
                    void* y_shared, void* ws, void* stream);
+
+/* moe_expert_ffn_gathered (BF16 mode only): moe_expert_ffn without the
+ * permuted copy of x.  GEMM1 reads each routed row straight from x, row
+ * perm_tok[r] for row r of the expert-major order (four rows per TMA
+ * tile::gather4 copy), so moe_dispatch may be called with x_perm = NULL.
+ *   x          [T, d] bf16 layer input
+ *   perm_tok   [T*K] int32, offsets [N+1] int32   from moe_dispatch
+ *   w13, w2, y_perm, y_shared, ws   as at moe_expert_ffn
+ * Same results as moe_expert_ffn on the same inputs (bit-identical rows).
+ * Returns MOE_ERR_UNSUPPORTED for other dtypes. */
+int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t* perm_tok,
+                            const int32_t* offsets, const void* w13, const void* w2,
+                            void* y_perm, void* y_shared, void* ws, void* stream);
 
 /* Combine ([P1] §2.2 COMBINE): y[t] = y_shared[t] + sum_k gate[t,k] *
  * y_perm[slot[t,k]], accumulated in fp32 in k order, rounded once to the

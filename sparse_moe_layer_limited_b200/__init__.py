@@ -6,7 +6,8 @@ loaded on first use, and any call fails loudly when it has not been built.
 """
 from ._lib import (  # noqa: F401
     DTYPE_BF16, DTYPE_E4M3, DTYPE_FP32, MoEError, MoEShape, check_shape, lib, moe_bias_update,
-    moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_expert_ffn, moe_forward, moe_pack_w13, moe_quantize_weights,
+    moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_expert_ffn, moe_expert_ffn_gathered,
+    moe_forward, moe_pack_w13, moe_quantize_weights,
     moe_read_device_status, moe_route, moe_workspace_init, shape, status_string,
     workspace_size, x_torch_dtype, w_torch_dtype,
 )

@@ -48,6 +48,7 @@ _SIGS = {
     "moe_route": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 8),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 10),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
+    "moe_expert_ffn_gathered": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
     "moe_dispatch_noalloc": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, ctypes.c_float,
@@ -158,8 +159,9 @@ def moe_dispatch(s, x, topk_idx, counts, offsets, perm_tok, slot, x_perm, x_perm
     _expect(offsets, torch.int32, s.N + 1, "offsets")
     _expect(perm_tok, torch.int32, s.T * s.K, "perm_tok")
     _expect(slot, torch.int32, s.T * s.K, "slot")
-    _expect(x_perm, w_torch_dtype(s) if s.dtype == DTYPE_E4M3 else x_torch_dtype(s),
-            s.T * s.K * s.d, "x_perm")
+    if x_perm is not None:  # None: rows not copied (BF16/FP32, moe_expert_ffn_gathered)
+        _expect(x_perm, w_torch_dtype(s) if s.dtype == DTYPE_E4M3 else x_torch_dtype(s),
+                s.T * s.K * s.d, "x_perm")
     _call("moe_dispatch", ctypes.byref(s), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
           _ptr(perm_tok), _ptr(slot), _ptr(x_perm), _ptr(x_perm_scales), _ptr(ws),
           _stream(stream))
@@ -185,6 +187,16 @@ def moe_expert_ffn(s, x_perm, x_perm_scales, offsets, x, w13, w2, w13_scales, w2
     _call("moe_expert_ffn", ctypes.byref(s), _ptr(x_perm), _ptr(x_perm_scales), _ptr(offsets),
           _ptr(x), _ptr(w13), _ptr(w2), _ptr(w13_scales), _ptr(w2_scales), _ptr(y_perm),
           _ptr(y_shared), _ptr(ws), _stream(stream))
+
+
+def moe_expert_ffn_gathered(s, x, perm_tok, offsets, w13, w2, y_perm, y_shared, ws,
+                            stream=None):
+    _expect(w13, w_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "w13")
+    _expect(w2, w_torch_dtype(s), (s.N + 1) * s.d * s.f, "w2")
+    _expect(y_perm, x_torch_dtype(s), s.T * s.K * s.d, "y_perm")
+    _expect(y_shared, x_torch_dtype(s), s.T * s.d, "y_shared")
+    _call("moe_expert_ffn_gathered", ctypes.byref(s), _ptr(x), _ptr(perm_tok), _ptr(offsets),
+          _ptr(w13), _ptr(w2), _ptr(y_perm), _ptr(y_shared), _ptr(ws), _stream(stream))
 
 
 def moe_combine(s, y_perm, y_shared, slot, topk_gate, y, stream=None):

@@ -140,9 +140,12 @@ int moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx,
   int rc = check(shape);
   if (rc) return rc;
   if (!ptr_ok(x) || !ptr_ok(topk_idx) || !ptr_ok(counts) || !ptr_ok(offsets) ||
-      !ptr_ok(perm_tok) || !ptr_ok(slot) || !ptr_ok(x_perm))
+      !ptr_ok(perm_tok) || !ptr_ok(slot))
     return MOE_ERR_ARG;
-  if (shape->dtype == MOE_DTYPE_E4M3 && !ptr_ok(x_perm_scales)) return MOE_ERR_ARG;
+  // x_perm may be NULL (rows not copied) except in E4M3 mode, which needs the codes
+  if (x_perm != nullptr && !aligned16(x_perm)) return MOE_ERR_ARG;
+  if (shape->dtype == MOE_DTYPE_E4M3 && (!ptr_ok(x_perm) || !ptr_ok(x_perm_scales)))
+    return MOE_ERR_ARG;
   if ((rc = ws_check(shape, ws))) return rc;
   cudaError_t e = launch_dispatch(*shape, x, topk_idx, counts, offsets, perm_tok, slot, x_perm,
                                   x_perm_scales, ws, static_cast<cudaStream_t>(stream));
@@ -171,11 +174,26 @@ int moe_expert_ffn(const moe_shape* shape, const void* x_perm, const float* x_pe
           static_cast<const float*>(w13), static_cast<const float*>(w2),
           static_cast<float*>(y_perm), static_cast<float*>(y_shared), ws, st));
     case MOE_DTYPE_BF16:
-      return launch_ffn_tc_bf16(*shape, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
+      return launch_ffn_tc_bf16(*shape, x_perm, nullptr, offsets, x, w13, w2, y_perm, y_shared,
+                                ws, st);
     default:
       return launch_ffn_tc_e4m3(*shape, x_perm, x_perm_scales, offsets, x, w13, w2, w13_scales,
                                 w2_scales, y_perm, y_shared, ws, st);
   }
+}
+
+int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t* perm_tok,
+                            const int32_t* offsets, const void* w13, const void* w2,
+                            void* y_perm, void* y_shared, void* ws, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(x) || !ptr_ok(perm_tok) || !ptr_ok(offsets) || !ptr_ok(w13) || !ptr_ok(w2) ||
+      !ptr_ok(y_perm) || !ptr_ok(y_shared))
+    return MOE_ERR_ARG;
+  if ((rc = ws_check(shape, ws))) return rc;
+  return launch_ffn_tc_bf16(*shape, nullptr, perm_tok, offsets, x, w13, w2, y_perm, y_shared,
+                            ws, static_cast<cudaStream_t>(stream));
 }
 
 int moe_combine(const moe_shape* shape, const void* y_perm, const void* y_shared,

@@ -138,7 +138,8 @@ __device__ __forceinline__ void chunk_slots(const int32_t* __restrict__ idx,
   __syncthreads();
 }
 
-// Slots for one chunk, then the row gather (bf16 / fp32 rows copied verbatim).
+// Slots for one chunk, then the row gather (bf16 / fp32 rows copied verbatim;
+// skipped when x_perm is null).
 template <typename XT>
 __global__ void __launch_bounds__(256) scatter_gather_kernel(
     const XT* __restrict__ x, const int32_t* __restrict__ idx,
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(256) scatter_gather_kernel(
   const int t0 = c * kChunkTokens;
   const int nt = min(kChunkTokens, T - t0);
   chunk_slots(idx, chunk_base, c, t0, nt, T, K, N, perm_tok, slot, sidx, sslot);
+  if (x_perm == nullptr) return;  // slots only: the expert GEMM gathers the rows itself
   // gather: warp per token, 16-byte vectors
   constexpr int kElems = 16 / sizeof(XT);
   const int nvec = d / kElems;

@@ -69,16 +69,20 @@ struct TileCfg {
   static constexpr int kBBytes = kBN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * kBN;  // two accumulators
-  static constexpr size_t smem_bytes(int groups) {
-    return 1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(groups + 1) * 4;
+  static constexpr size_t smem_bytes(int groups, bool gather) {
+    return 1024 + (size_t)kStages * kStageBytes + 256 + (gather ? (size_t)BM * 8 : 0) +
+           (size_t)(groups + 1) * 4;
   }
 };
 
 struct alignas(64) GemmArgs {
-  CUtensorMap tmA_routed;
+  CUtensorMap tmA_routed;  // routed rows (unused when a_rows is set)
   CUtensorMap tmA_shared;
   CUtensorMap tmB;
   const int32_t* offsets;
+  const int32_t* a_rows;  // when set: routed A row r of a group is a_src row a_rows[offsets[g] + r]
+  const __nv_bfloat16* a_src;  // gathered rows' source (x), a_ld elements per row
+  int a_ld;
   __nv_bfloat16* out_routed;
   __nv_bfloat16* out_shared;
   float* out_f32;   // score epilogue: fp32 partial sums [k_splits, T, n_valid]
@@ -94,7 +98,7 @@ struct alignas(64) GemmArgs {
   int k_splits; // K ranges computed by separate units (score epilogue; else 1)
 };
 
-template <int kEpi, int kBN>
+template <int kEpi, int kBN, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     const __grid_constant__ GemmArgs args) {
   constexpr int BN = kBN;
@@ -113,7 +117,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   uint64_t* tempty = tfull + 2;          // [2]
   uint64_t* drain = tempty + 2;          // [1]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  int* tile_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + 256);
+  // gathered tiles: the source address of each of the tile's 128 rows
+  const char** rowptr =
+      reinterpret_cast<const char**>(base + (size_t)kStages * kStageBytes + 256);
+  int* tile_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + 256 +
+                                           (kGather ? BM * 8 : 0));
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -125,7 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   // ---- set-up: barriers, TMEM, tile schedule --------------------------------
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      // with gathered rows every producer lane also arrives once per stage,
+      // when its row copies have landed
+      mbar_init(&full[s], kGather ? 33 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -183,11 +193,59 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   };
 
   if (warp == 0) {
-    // ---- TMA producer ---------------------------------------------------------
-    if (lane == 0) {
-      tma_prefetch_desc(&args.tmA_routed);
-      tma_prefetch_desc(&args.tmA_shared);
-      tma_prefetch_desc(&args.tmB);
+    if constexpr (!kGather) {
+      // ---- TMA producer ---------------------------------------------------------
+      if (lane == 0) {
+        tma_prefetch_desc(&args.tmA_routed);
+        tma_prefetch_desc(&args.tmA_shared);
+        tma_prefetch_desc(&args.tmB);
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued = 0, issued_parity = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+          int g, n, m, mt;
+          decode(tile, g, n, m, mt);
+          const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
+          const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * BM;
+          const int brow = g * args.n_acc + (n / args.k_splits) * BN;
+          const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sa = base + (size_t)stage * kStageBytes;
+            mbar_arrive_expect_tx(&full[stage], kStageBytes);
+            tma_load_2d(sa, am, (kb / args.a_rep) * BK, arow, &full[stage]);
+            tma_load_2d(sa + kABytes, &args.tmB, kb * BK, brow, &full[stage]);
+            issued |= 1u << stage;
+            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) {  // let the copies already issued land before the CTA exits
+          for (int s = 0; s < kStages; ++s)
+            if ((issued >> s) & 1u)
+              mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.status, kTimeoutNs / 8);
+        }
+      }
+    } else {
+      // ---- TMA producer (gathered routed rows) -----------------------------------
+      // Lane 0 waits, arms the barrier and loads B (and A for contiguous rows)
+      // by TMA.  With a_rows set, the warp gathers a routed tile's 128 token
+      // rows itself: per stage 32 cp.async instructions of 16 bytes per lane,
+      // four rows of 128 bytes each, written in the 128-byte swizzled layout the
+      // MMA reads (16-byte chunk c of row r at chunk c ^ (r mod 8)); each lane's
+      // copies complete on the stage's barrier, and no permuted copy of x exists.
+      if (lane == 0) {
+        tma_prefetch_desc(&args.tmA_routed);
+        tma_prefetch_desc(&args.tmA_shared);
+        tma_prefetch_desc(&args.tmB);
+      }
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;
@@ -195,19 +253,49 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int g, n, m, mt;
         decode(tile, g, n, m, mt);
+        const bool gather = g < args.N;
         const CUtensorMap* am = (g < args.N) ? &args.tmA_routed : &args.tmA_shared;
         const int arow = ((g < args.N) ? args.offsets[g] : args.a_shared_row0) + m * BM;
         const int brow = g * args.n_acc + (n / args.k_splits) * BN;
         const int kb0 = (n % args.k_splits) * KBs, kb1 = min(KB, kb0 + KBs);
+        if (gather) {  // rows past the group's end read token 0; they are never stored
+          __syncwarp();
+          const int rows_g = args.offsets[g + 1] - args.offsets[g];
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int rr = 4 * lane + j;
+            const int row = m * BM + rr;
+            int t = row < rows_g ? args.a_rows[args.offsets[g] + row] : 0;
+            if (t < 0 || t >= args.T) t = 0;
+            rowptr[rr] = reinterpret_cast<const char*>(args.a_src + (size_t)t * args.a_ld);
+          }
+          __syncwarp();
+        }
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs)) {
+          bool got = true;
+          if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, kTimeoutNs);
+          if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
             ok = false;
             break;
           }
           uint8_t* sa = base + (size_t)stage * kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          tma_load_2d(sa, am, (kb / args.a_rep) * BK, arow, &full[stage]);
-          tma_load_2d(sa + kABytes, &args.tmB, kb * BK, brow, &full[stage]);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], gather ? kBBytes : kStageBytes);
+            if (!gather) tma_load_2d(sa, am, (kb / args.a_rep) * BK, arow, &full[stage]);
+            tma_load_2d(sa + kABytes, &args.tmB, kb * BK, brow, &full[stage]);
+          }
+          if (args.a_rows != nullptr) {
+            if (gather) {
+              const int c = lane & 7;
+              const int koff = (kb * BK + c * 8) * 2;  // byte offset of this lane's chunk
+  #pragma unroll 8
+              for (int i = 0; i < BM / 4; ++i) {
+                const int r = 4 * i + (lane >> 3);
+                cp_async_16(sa + r * (BK * 2) + ((c ^ (r & 7)) << 4), rowptr[r] + koff);
+              }
+            }
+            cp_async_mbar_arrive_noinc(&full[stage]);
+          }
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -216,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           }
         }
       }
-      if (!ok) {  // let the copies already issued land before the CTA exits
+      if (!ok && lane == 0) {  // let the copies already issued land before the CTA exits
         for (int s = 0; s < kStages; ++s)
           if ((issued >> s) & 1u)
             mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.status, kTimeoutNs / 8);
@@ -248,6 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
             ok = false;
             break;
           }
+          // rows copied by the producer lanes are generic-proxy writes
+          if constexpr (kGather) fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(base + (size_t)stage * kStageBytes);
           const uint32_t b0 = a0 + kABytes;
@@ -351,15 +441,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   }
 }
 
-template <int kEpi, int kBN>
+template <int kEpi, int kBN, bool kGather = false>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
-  const size_t smem = TileCfg<kBN>::smem_bytes(a.N + 1);
-  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN>,
+  const size_t smem = TileCfg<kBN>::smem_bytes(a.N + 1, kGather);
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN, kGather>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem),
                             "bf16 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
-  grouped_gemm_bf16_kernel<kEpi, kBN><<<num_sms(), kThreads, smem, st>>>(a);
+  grouped_gemm_bf16_kernel<kEpi, kBN, kGather><<<num_sms(), kThreads, smem, st>>>(a);
   return note_cuda(cudaGetLastError(), "bf16 GEMM launch");
 }
 
@@ -388,9 +478,9 @@ __global__ void router_split_kernel(const float* __restrict__ R, int N, int d,
 
 }  // namespace
 
-int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
-                       const void* x, const void* w13, const void* w2, void* y_perm,
-                       void* y_shared, void* ws, cudaStream_t st) {
+int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* perm_tok,
+                       const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                       void* y_perm, void* y_shared, void* ws, cudaStream_t st) {
   // MOE_BF16_GEMM selects the expert GEMM kernel: "dual" (two token tiles per
   // weight tile, gemm_dual.cu), "pair" (CTA pairs, gemm2sm.cu); default: this file's
   static const int kind = [] {
@@ -399,8 +489,11 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
     if (v != nullptr && std::strcmp(v, "dual") == 0) return 1;
     return 0;
   }();
-  if (kind == 2) return launch_ffn_tc_bf16_pair(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
-  if (kind == 1) return launch_ffn_tc_bf16_dual(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
+  // rows gathered from x through perm_tok always run on this file's kernel
+  if (perm_tok == nullptr && kind == 2)
+    return launch_ffn_tc_bf16_pair(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
+  if (perm_tok == nullptr && kind == 1)
+    return launch_ffn_tc_bf16_dual(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
   const WsLayout L = ws_layout(s);
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(w + L.h);
@@ -408,7 +501,9 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
   GemmArgs g1{};
-  bool ok = make_map(&g1.tmA_routed, x_perm, BF, 2, s.d, TK, BK, BM) &&
+  // gathered rows are copied by the producer warp; the routed map is then unused
+  bool ok = make_map(&g1.tmA_routed, perm_tok ? x : x_perm, BF, 2, s.d, perm_tok ? s.T : TK,
+                     BK, BM) &&
             make_map(&g1.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
             make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * 2 * s.f, BK, 256);
   if (!ok) {
@@ -416,6 +511,9 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
     return MOE_ERR_CUDA;
   }
   g1.offsets = offsets;
+  g1.a_rows = perm_tok;
+  g1.a_src = static_cast<const __nv_bfloat16*>(x);
+  g1.a_ld = s.d;
   g1.out_routed = H;
   g1.out_shared = H + TK * s.f;
   g1.status = reinterpret_cast<uint32_t*>(w + L.status);
@@ -428,7 +526,9 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* of
   g1.out_ld = s.f;
   g1.a_rep = 1;
   g1.k_splits = 1;
-  if (launch_gemm<kEpiSwiGLU, 256>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((perm_tok ? launch_gemm<kEpiSwiGLU, 256, true>(g1, st)
+                : launch_gemm<kEpiSwiGLU, 256>(g1, st)) != cudaSuccess)
+    return MOE_ERR_CUDA;
 
   GemmArgs g2{};
   ok = make_map(&g2.tmA_routed, H, BF, 2, s.f, TK + s.T, BK, BM) &&

@@ -86,9 +86,11 @@ int router_k_splits(const moe_shape& s);
 int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* Z,
                             int k_splits, void* ws, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* status (tensor maps can fail to encode).
-int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
-                       const void* x, const void* w13, const void* w2, void* y_perm,
-                       void* y_shared, void* ws, cudaStream_t st);
+// bf16 expert GEMMs; with perm_tok set, GEMM1 gathers the routed rows from x
+// (x_perm unused), else it reads x_perm.
+int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* perm_tok,
+                       const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                       void* y_perm, void* y_shared, void* ws, cudaStream_t st);
 // The same two GEMMs on CTA pairs (tcgen05 cta_group::2), gemm2sm.cu.
 int launch_ffn_tc_bf16_dual(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                             const void* x, const void* w13, const void* w2, void* y_perm,

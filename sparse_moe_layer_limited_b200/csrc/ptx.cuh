@@ -98,6 +98,23 @@ __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src)
                "l"(gmem_src)
                : "memory");
 }
+// 16-byte global -> shared copy that bypasses L1.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+// One arrival on `bar`, made when this thread's copies issued so far have
+// landed; counted in the barrier's expected arrivals (no extra pending count).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// Make this thread's view of generic-proxy shared-memory writes visible to
+// the async proxy (tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }

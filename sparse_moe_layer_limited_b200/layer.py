@@ -13,10 +13,14 @@ class MoELayer:
     router_w [N, d] fp32, bias [N] fp32 (updated in place by forward), w13
     [N+1, 2f, d] packed (see moe_pack_w13), w2 [N+1, d, f]; for E4M3 the
     quantised weights and their 128x128-block scales.  All tensors must be on
-    the same CUDA device.  Intermediate buffers are allocated once here."""
+    the same CUDA device.  Intermediate buffers are allocated once here.
+
+    gather (BF16 only): GEMM1 reads each routed row straight from x through
+    perm_tok (moe_expert_ffn_gathered) instead of a permuted copy; dispatch
+    then writes no x_perm."""
 
     def __init__(self, shape: L.MoEShape, router_w, bias, w13, w2, w13_scales=None,
-                 w2_scales=None, gamma: float = 0.001):
+                 w2_scales=None, gamma: float = 0.001, gather: bool = False):
         rc = L.check_shape(shape)
         if rc != L.OK:
             raise L.MoEError("moe_check_shape", rc)
@@ -24,6 +28,7 @@ class MoELayer:
         self.router_w, self.bias, self.w13, self.w2 = router_w, bias, w13, w2
         self.w13_scales, self.w2_scales = w13_scales, w2_scales
         self.gamma = float(gamma)
+        self.gather = bool(gather) and s.dtype == L.DTYPE_BF16
         dev = router_w.device
         i32 = dict(dtype=torch.int32, device=dev)
         xdt = L.x_torch_dtype(s)
@@ -34,7 +39,8 @@ class MoELayer:
         self.perm_tok = torch.empty(s.T * s.K, **i32)
         self.slot = torch.empty(s.T, s.K, **i32)
         pdt = torch.float8_e4m3fn if s.dtype == L.DTYPE_E4M3 else xdt
-        self.x_perm = torch.empty(s.T * s.K, s.d, dtype=pdt, device=dev)
+        self.x_perm = (None if self.gather
+                       else torch.empty(s.T * s.K, s.d, dtype=pdt, device=dev))
         self.x_perm_scales = (torch.empty(s.d // 128, (s.T * s.K + 3) // 4 * 4, dtype=torch.float32,
                                           device=dev)
                               if s.dtype == L.DTYPE_E4M3 else None)
@@ -56,13 +62,22 @@ class MoELayer:
                     self.ws, stream)
         L.moe_dispatch(s, x, self.topk_idx, self.counts, self.offsets, self.perm_tok, self.slot,
                        self.x_perm, self.x_perm_scales, self.ws, stream)
-        L.moe_expert_ffn(s, self.x_perm, self.x_perm_scales, self.offsets, x, self.w13, self.w2,
-                         self.w13_scales, self.w2_scales, self.y_perm, self.y_shared, self.ws,
-                         stream)
+        self.experts(x, stream)
         L.moe_combine(s, self.y_perm, self.y_shared, self.slot, self.topk_gate, self.y, stream)
         if update_bias:
             L.moe_bias_update(s, self.counts, self.bias, self.gamma, stream)
         return self.y
+
+    def experts(self, x, stream=None):
+        """The expert GEMMs on the dispatched rows (gathered from x or read from x_perm)."""
+        s = self.shape
+        if self.gather:
+            L.moe_expert_ffn_gathered(s, x, self.perm_tok, self.offsets, self.w13, self.w2,
+                                      self.y_perm, self.y_shared, self.ws, stream)
+        else:
+            L.moe_expert_ffn(s, self.x_perm, self.x_perm_scales, self.offsets, x, self.w13,
+                             self.w2, self.w13_scales, self.w2_scales, self.y_perm,
+                             self.y_shared, self.ws, stream)
 
     def device_status(self, clear: bool = False) -> int:
         return L.moe_read_device_status(self.ws, None, clear)

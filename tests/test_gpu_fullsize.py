@@ -69,6 +69,27 @@ def test_v3_bf16_passes_and_sampled_outputs(M):
     del torch
 
 
+def test_v3_bf16_gathered_rows_bitexact(M):
+    """At the full V3 size the gathered expert GEMMs (no x_perm) reproduce the
+    x_perm path's expert outputs bit for bit."""
+    import torch
+    cfg = CONFIGS[2]
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    W = S.device_weights(cfg)
+    layer = _layer(M, cfg, R, b, W)
+    x, _ = S.tie_free_x(cfg, R, b)
+    xd = S.to_dev_x(x, cfg)
+    layer.forward(xd, update_bias=False)
+    s = layer.shape
+    yp, ysh = torch.empty_like(layer.y_perm), torch.empty_like(layer.y_shared)
+    M.moe_expert_ffn_gathered(s, xd, layer.perm_tok, layer.offsets, layer.w13, layer.w2, yp, ysh,
+                              layer.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(yp, layer.y_perm)
+    assert torch.equal(ysh, layer.y_shared)
+    assert layer.device_status() == 0
+
+
 def test_decode_zipf_200_steps(M):
     import torch
     cfg = CONFIGS[4]

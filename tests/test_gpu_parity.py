@@ -154,6 +154,40 @@ def test_small_bf16_layer_full(M, T):
     assert layer.device_status() == 0
 
 
+@pytest.mark.parametrize("T", [1000, 129, 1])
+def test_gathered_expert_rows_bitexact(M, T):
+    """moe_expert_ffn_gathered (GEMM1 gathers x rows through perm_tok, dispatch
+    copies nothing) gives bit-identical expert outputs to the x_perm path, and
+    the gathered layer matches the oracle."""
+    torch = _torch()
+    cfg = _small_bf16(T)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    layer.forward(xd, update_bias=False)
+    s = layer.shape
+    perm_tok, slot = torch.empty_like(layer.perm_tok), torch.empty_like(layer.slot)
+    offsets = torch.empty_like(layer.offsets)
+    yp, ysh = torch.empty_like(layer.y_perm), torch.empty_like(layer.y_shared)
+    M.moe_dispatch(s, xd, layer.topk_idx, layer.counts, offsets, perm_tok, slot, None, None,
+                   layer.ws)
+    M.moe_expert_ffn_gathered(s, xd, perm_tok, offsets, layer.w13, layer.w2, yp, ysh, layer.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(perm_tok, layer.perm_tok) and torch.equal(slot, layer.slot)
+    assert torch.equal(yp, layer.y_perm)
+    assert torch.equal(ysh, layer.y_shared)
+    # the layer built to gather end to end, against the oracle
+    lg = M.MoELayer(s, layer.router_w, torch.from_numpy(np.asarray(b, np.float32)).cuda(),
+                    W["w13"], W["w2"], gamma=cfg.gamma, gather=True)
+    assert lg.gather and lg.x_perm is None
+    y = lg.forward(xd).float().cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             h_round="bf16")
+    assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
+    assert lg.device_status() == 0 and layer.device_status() == 0
+
+
 def test_mid_bf16_layer_sampled(M):
     """The mid-size bf16 layer: full routing/dispatch, outputs on 256 tokens."""
     torch = _torch()
