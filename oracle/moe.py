@@ -127,6 +127,63 @@ def route_margins(x, router, bias, G: int, topG: int, K: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# the conventional softmax gate (the baseline the method replaces)
+# ---------------------------------------------------------------------------
+
+def route_softmax(x, router, K: int) -> dict:
+    """Softmax top-K routing, the conventional gate that the bias method
+    replaces, kept as a baseline.
+
+    [P4] (gating paragraph): a conventional gating network is a softmax on
+    top of a classifier, balanced by an auxiliary penalty term; [P2] Q3:
+    conventional MoE models add an auxiliary loss for balance.  The pages give
+    no formula; the plainest reading, per token:
+      1. z_i = x . e_i,  p = softmax(z) over all N experts
+      2. idx = the K largest p (no groups, no bias), ascending expert id
+      3. gate_k = p[idx_k] / sum_j p[idx_j]  (the softmax over the selected)
+      4. counts_i as in route(); prob_sum_i = sum_t p[t, i]
+    Returns dict(idx, gate, counts, p, prob_sum)."""
+    z = np.asarray(x, dtype=np.float64) @ np.asarray(router, dtype=np.float64).T
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)
+    T, N = p.shape
+    top = np.argsort(-z, axis=1, kind="stable")[:, :K]
+    idx = np.sort(top, axis=1)
+    sel = np.take_along_axis(p, idx, axis=1)
+    gate = sel / sel.sum(axis=1, keepdims=True)
+    counts = np.bincount(idx.ravel(), minlength=N).astype(np.int64)
+    return dict(idx=idx.astype(np.int64), gate=gate, counts=counts, p=p,
+                prob_sum=p.sum(axis=0))
+
+
+def route_softmax_margins(x, router, K: int) -> np.ndarray:
+    """Per token, the K-th minus the (K+1)-th largest logit z (+inf when
+    K = N): the gap that decides the softmax top-K."""
+    z = np.asarray(x, dtype=np.float64) @ np.asarray(router, dtype=np.float64).T
+    zs = -np.sort(-z, axis=1)
+    if K >= z.shape[1]:
+        return np.full(z.shape[0], np.inf)
+    return zs[:, K - 1] - zs[:, K]
+
+
+def balance_loss(counts, prob_sum, T: int, K: int) -> float:
+    """The conventional auxiliary balance statistic of a routing batch:
+    L = N * sum_i f_i * P_i with f_i = counts_i / (K T), the share of the
+    T*K selections that went to expert i, and P_i = prob_sum_i / T, the mean
+    softmax probability of expert i.  L = 1 when both are uniform and grows
+    as routing concentrates.  [P4]: the penalty discourages over-confident
+    gate outputs; [P1] §1.2: per-sequence load concentration is what it
+    measures when the batch is one sequence.  The product form is the reading
+    this library takes (the pages give no formula)."""
+    counts = np.asarray(counts, dtype=np.float64)
+    prob_sum = np.asarray(prob_sum, dtype=np.float64)
+    N = counts.size
+    f = counts / (K * T)
+    P = prob_sum / T
+    return float(N * np.sum(f * P))
+
+
+# ---------------------------------------------------------------------------
 # dispatch, experts, combine
 # ---------------------------------------------------------------------------
 
