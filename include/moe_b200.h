@@ -137,6 +137,22 @@ int moe_read_device_status(void* ws, void* stream, uint32_t* status_out, int cle
 int moe_route(const moe_shape* shape, const void* x, const float* router_w, const float* bias,
               int32_t* topk_idx, float* topk_gate, int32_t* counts, void* ws, void* stream);
 
+/* moe_route_softmax: the conventional softmax gate that the bias method
+ * replaces, kept as a baseline to contrast with it ([P4] gating paragraph: a
+ * softmax on top of a classifier, balanced by an auxiliary penalty; [P2] Q3).
+ * Per token: p = softmax(x . e_i) over all N experts; the K largest p (no
+ * groups, no bias; shape->G and topG are ignored), ascending expert id;
+ * gate_k = p_k / sum of the selected p.  BF16 and E4M3 shapes (x bf16).
+ *   topk_idx, topk_gate, counts   as at moe_route
+ *   prob_sum   [N] fp32 out or NULL: sum over the T tokens of p[t, i], added
+ *              in a fixed order (deterministic).  With counts it gives the
+ *              conventional balance statistic N * sum_i (counts_i / (K T)) *
+ *              (prob_sum_i / T), 1 for uniform routing.
+ * Returns MOE_ERR_UNSUPPORTED for FP32 shapes. */
+int moe_route_softmax(const moe_shape* shape, const void* x, const float* router_w,
+                      int32_t* topk_idx, float* topk_gate, int32_t* counts, float* prob_sum,
+                      void* ws, void* stream);
+
 /* Dispatch ([P1] §2.2 DISPATCH, single-GPU permutation): group the T*K
  * (token, expert) pairs by expert.  Row order is experts ascending, tokens
  * ascending within an expert, so the result is deterministic.

@@ -8,7 +8,8 @@ from ._lib import (  # noqa: F401
     DTYPE_BF16, DTYPE_E4M3, DTYPE_FP32, MoEError, MoEShape, check_shape, lib, moe_bias_update,
     moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_expert_ffn, moe_expert_ffn_gathered,
     moe_forward, moe_pack_w13, moe_quantize_weights,
-    moe_read_device_status, moe_route, moe_workspace_init, shape, status_string,
+    moe_read_device_status, moe_route, moe_route_softmax, moe_workspace_init, shape,
+    status_string,
     workspace_size, x_torch_dtype, w_torch_dtype,
 )
 from .layer import MoELayer  # noqa: F401

@@ -46,6 +46,7 @@ _SIGS = {
     "moe_read_device_status": (ctypes.c_int, [_c_p, _c_p, ctypes.POINTER(ctypes.c_uint32),
                                               ctypes.c_int]),
     "moe_route": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 8),
+    "moe_route_softmax": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 8),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 10),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
     "moe_expert_ffn_gathered": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
@@ -152,6 +153,17 @@ def moe_route(s, x, router_w, bias, topk_idx, topk_gate, counts, ws, stream=None
     _expect(counts, torch.int32, s.N, "counts")
     _call("moe_route", ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(topk_idx),
           _ptr(topk_gate), _ptr(counts), _ptr(ws), _stream(stream))
+
+
+def moe_route_softmax(s, x, router_w, topk_idx, topk_gate, counts, prob_sum, ws,
+                      stream=None):
+    _expect(topk_idx, torch.int32, s.T * s.K, "topk_idx")
+    _expect(topk_gate, torch.float32, s.T * s.K, "topk_gate")
+    _expect(counts, torch.int32, s.N, "counts")
+    if prob_sum is not None:
+        _expect(prob_sum, torch.float32, s.N, "prob_sum")
+    _call("moe_route_softmax", ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(topk_idx),
+          _ptr(topk_gate), _ptr(counts), _ptr(prob_sum), _ptr(ws), _stream(stream))
 
 
 def moe_dispatch(s, x, topk_idx, counts, offsets, perm_tok, slot, x_perm, x_perm_scales, ws,

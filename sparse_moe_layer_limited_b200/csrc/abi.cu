@@ -22,6 +22,8 @@ WsLayout ws_layout(const moe_shape& s) {
     off = align256(off + (size_t)s.N * 3 * s.d * 2);
     L.scores = off;
     off = align256(off + (size_t)8 * s.T * s.N * 4);
+    L.prob_part = off;
+    off = align256(off + (size_t)((s.T + 7) / 8) * s.N * 4);
   }
   const size_t rows = (size_t)s.T * s.K + s.T;
   L.h = off;
@@ -132,6 +134,21 @@ int moe_route(const moe_shape* shape, const void* x, const float* router_w, cons
   if ((rc = ws_check(shape, ws))) return rc;
   return launch_route(*shape, x, router_w, bias, topk_idx, topk_gate, counts, ws,
                       static_cast<cudaStream_t>(stream));
+}
+
+int moe_route_softmax(const moe_shape* shape, const void* x, const float* router_w,
+                      int32_t* topk_idx, float* topk_gate, int32_t* counts, float* prob_sum,
+                      void* ws, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype == MOE_DTYPE_FP32) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(x) || !ptr_ok(router_w) || !ptr_ok(topk_idx) || !ptr_ok(topk_gate) ||
+      !ptr_ok(counts))
+    return MOE_ERR_ARG;
+  if (prob_sum != nullptr && !aligned16(prob_sum)) return MOE_ERR_ARG;
+  if ((rc = ws_check(shape, ws))) return rc;
+  return launch_route_softmax(*shape, x, router_w, topk_idx, topk_gate, counts, prob_sum, ws,
+                              static_cast<cudaStream_t>(stream));
 }
 
 int moe_dispatch(const moe_shape* shape, const void* x, const int32_t* topk_idx,

@@ -23,10 +23,11 @@ struct WsLayout {
   size_t chunk_base = 0;  // int32 [chunks, N]
   size_t router_split = 0;  // bf16 [N, 3d] exact three-part split of the router (bf16 x)
   size_t scores = 0;        // fp32 [splits <= 8, T, N] partial router logits (bf16 x)
+  size_t prob_part = 0;     // fp32 [ceil(T/8), N] softmax-probability sums per selection CTA
   size_t h = 0;           // hidden activation [T*K + T, f] (bf16 / fp32 / e4m3)
-  size_t h_scales = 0;    // fp32 [T*K + T, f/128] (E4M3)
+  size_t h_scales = 0;    // fp32 block-major [f/128, scale_ld(T*K + T)] (E4M3)
   size_t xq = 0;          // E4M3 codes of x for the shared expert [T, d]
-  size_t xq_scales = 0;   // fp32 [T, d/128]
+  size_t xq_scales = 0;   // fp32 block-major [d/128, scale_ld(T)]
   size_t total = 0;
 };
 WsLayout ws_layout(const moe_shape& s);
@@ -65,6 +66,11 @@ bool make_map_f32_rows(CUtensorMap* map, const float* ptr, uint64_t inner, uint6
 int num_sms();
 
 // ---- launchers (return cudaError_t of the launch) -----------------------------
+// Softmax top-K baseline routing (bf16 / E4M3 shapes): idx, gate, counts and,
+// when prob_sum is set, the per-expert sums of the softmax probabilities.
+int launch_route_softmax(const moe_shape& s, const void* x, const float* router, int32_t* idx,
+                         float* gate, int32_t* counts, float* prob_sum, void* ws,
+                         cudaStream_t st);
 int launch_route(const moe_shape& s, const void* x, const float* router, const float* bias,
                  int32_t* idx, float* gate, int32_t* counts, void* ws, cudaStream_t st);
 cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* idx,

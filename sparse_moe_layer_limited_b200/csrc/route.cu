@@ -231,16 +231,28 @@ __global__ void __launch_bounds__(256) route_kernel(const XT* __restrict__ x,
 // Selection from the tensor-core logits Z [splits, T, N]: z is the sum of
 // the split partials in split order, s = sigmoid(z); one warp per token,
 // 8 tokens per CTA.
+//
+// kSoftmax: the conventional softmax gate kept as a baseline (the DeepSeek-V3
+// walk-through's gating paragraph: a softmax on top of a classifier, balanced
+// by an auxiliary penalty).  The selection score is e = exp(z - max_i z)
+// (monotone in z) with no bias and one group, so the same top-K picks the K
+// largest logits and the gate normalisation gives e_k / sum over the selected,
+// the softmax over the selected logits.  The CTA also writes, per expert, the
+// sum over its tokens (in warp order) of p = e / sum_i e, for the balance
+// statistic.
 constexpr int kSelTokens = 8;
 
+template <bool kSoftmax>
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z, int splits,
                                                      const float* __restrict__ bias, int T, int N,
                                                      int K, int G, int topG,
                                                      int32_t* __restrict__ topk_idx,
                                                      float* __restrict__ topk_gate,
                                                      int32_t* __restrict__ counts,
+                                                     float* __restrict__ prob_part,
                                                      uint32_t* __restrict__ status) {
   __shared__ int hist[kRouteMaxN];
+  __shared__ float pbuf[kSoftmax ? kSelTokens : 1][kSoftmax ? kRouteMaxN : 1];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < N; e += blockDim.x) hist[e] = 0;
@@ -250,23 +262,58 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z
     float bj[kEPL], s[kEPL];
     int grp[kEPL];
     lane_groups(lane, N, G, grp);
+    float zmax = -INFINITY;
 #pragma unroll
     for (int j = 0; j < kEPL; ++j) {
       float z = 0.f;
       bj[j] = 0.f;
       if (grp[j] >= 0) {
-        bj[j] = __ldg(bias + lane + 32 * j);
+        if (!kSoftmax) bj[j] = __ldg(bias + lane + 32 * j);
         z = __ldg(Z + (size_t)t * N + lane + 32 * j);
         for (int p = 1; p < splits; ++p)
           z = __fadd_rn(z, __ldg(Z + ((size_t)p * T + t) * N + lane + 32 * j));
+        zmax = fmaxf(zmax, z);
       }
-      s[j] = 1.f / (1.f + expf(-z));
+      s[j] = kSoftmax ? z : 1.f / (1.f + expf(-z));
+    }
+    if constexpr (kSoftmax) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+      float esum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kEPL; ++j) {
+        s[j] = grp[j] >= 0 ? expf(s[j] - zmax) : 0.f;
+        esum += s[j];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
+#pragma unroll
+      for (int j = 0; j < kEPL; ++j)
+        if (grp[j] >= 0) pbuf[warp][lane + 32 * j] = __fdiv_rn(s[j], esum);
     }
     select_token(s, bj, grp, lane, t, N, K, G, topG, topk_idx, topk_gate, hist, status);
   }
   __syncthreads();
+  if constexpr (kSoftmax) {  // this CTA's per-expert probability sums, tokens in order
+    const int nt = min(kSelTokens, T - (int)blockIdx.x * kSelTokens);
+    for (int e = tid; e < N; e += blockDim.x) {
+      float a = 0.f;
+      for (int w = 0; w < nt; ++w) a += pbuf[w][e];
+      prob_part[(size_t)blockIdx.x * N + e] = a;
+    }
+  }
   for (int e = tid; e < N; e += blockDim.x)
     if (hist[e]) atomicAdd(&counts[e], hist[e]);
+}
+
+// prob_sum[e] = sum over the selection CTAs, in CTA order, of their partials.
+__global__ void prob_sum_kernel(const float* __restrict__ part, int nblocks, int N,
+                                float* __restrict__ prob_sum) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= N) return;
+  float a = 0.f;
+  for (int b = 0; b < nblocks; ++b) a += part[(size_t)b * N + e];
+  prob_sum[e] = a;
 }
 
 }  // namespace
@@ -287,9 +334,29 @@ int launch_route(const moe_shape& s, const void* x, const float* router, const f
     const int splits = router_k_splits(s);
     const int rc = launch_router_scores_tc(s, x, router, Z, splits, ws, st);
     if (rc != MOE_OK) return rc;
-    select_kernel<<<(s.T + kSelTokens - 1) / kSelTokens, 256, 0, st>>>(
-        Z, splits, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate, counts, status);
+    select_kernel<false><<<(s.T + kSelTokens - 1) / kSelTokens, 256, 0, st>>>(
+        Z, splits, bias, s.T, s.N, s.K, s.G, s.topG, idx, gate, counts, nullptr, status);
   }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_route_softmax(const moe_shape& s, const void* x, const float* router, int32_t* idx,
+                         float* gate, int32_t* counts, float* prob_sum, void* ws,
+                         cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * s.N, st) != cudaSuccess) return MOE_ERR_CUDA;
+  float* Z = reinterpret_cast<float*>(w + L.scores);
+  float* part = reinterpret_cast<float*>(w + L.prob_part);
+  const int splits = router_k_splits(s);
+  const int rc = launch_router_scores_tc(s, x, router, Z, splits, ws, st);
+  if (rc != MOE_OK) return rc;
+  const int nb = (s.T + kSelTokens - 1) / kSelTokens;
+  // one group kept of one: plain top-K over all experts
+  select_kernel<true><<<nb, 256, 0, st>>>(Z, splits, nullptr, s.T, s.N, s.K, 1, 1, idx, gate,
+                                          counts, part, status);
+  if (prob_sum != nullptr) prob_sum_kernel<<<1, 256, 0, st>>>(part, nb, s.N, prob_sum);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

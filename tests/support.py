@@ -19,14 +19,18 @@ NEAR_TIE = 1e-4
 
 
 def tie_free_x(cfg: MoEConfig, router, bias, seed: int = 0, batch: int = 0, x=None,
-               max_attempts: int = 64):
+               max_attempts: int = 64, margins=None):
     """x [T, d] (float32 array of stored values) with no near-tie token under
-    (router, bias).  Returns (x, number of rows re-drawn)."""
+    (router, bias), or under `margins` (x rows -> per-row decision gaps) when
+    given.  Returns (x, number of rows re-drawn)."""
     x = gen.make_x(cfg, seed, batch) if x is None else x.copy()
     rows = np.arange(cfg.T)
     redrawn = 0
+    if margins is None:
+        def margins(xr):
+            return oracle.route_margins(xr, router, bias, cfg.G, cfg.topG, cfg.K)
     for attempt in range(max_attempts):
-        m = oracle.route_margins(x[rows], router, bias, cfg.G, cfg.topG, cfg.K)
+        m = margins(x[rows])
         bad = rows[m < NEAR_TIE]
         if bad.size == 0:
             return x, redrawn

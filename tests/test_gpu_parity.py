@@ -298,6 +298,53 @@ def test_route_degenerate_and_max(M, N, K, G, topG):
     _check_route(cfg, r, *_run_route(M, cfg, x, R, b))
 
 
+@pytest.mark.parametrize("N,K,T", [(64, 6, 1000), (256, 8, 777), (256, 13, 500), (16, 16, 97)])
+def test_softmax_route_baseline(M, N, K, T):
+    """moe_route_softmax against the oracle's softmax top-K: indices and
+    counts bit-exact, gates within fp32 rounding, per-expert probability sums
+    and the balance statistic within fp32 summation error."""
+    torch = _torch()
+    cfg = CONFIGS[1].with_(T=T, d=256, N=N, K=K, G=1, topG=1, f=256)
+    R = gen.make_router(cfg)
+    x, _ = S.tie_free_x(cfg, R, None,
+                        margins=lambda xr: oracle.route_softmax_margins(xr, R, cfg.K))
+    ref = oracle.route_softmax(x, R, cfg.K)
+    s = S.moe_shape(cfg)
+    idx = torch.empty(s.T, s.K, dtype=torch.int32, device="cuda")
+    gate = torch.empty(s.T, s.K, dtype=torch.float32, device="cuda")
+    counts = torch.empty(s.N, dtype=torch.int32, device="cuda")
+    psum = torch.empty(s.N, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(M.workspace_size(s), dtype=torch.uint8, device="cuda")
+    M.moe_route_softmax(s, S.to_dev_x(x, cfg), torch.from_numpy(R).cuda(), idx, gate, counts,
+                        psum, ws)
+    assert M.moe_read_device_status(ws) == 0
+    _check_route(cfg, ref, idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy())
+    ps = psum.cpu().numpy()
+    np.testing.assert_allclose(ps, ref["prob_sum"], rtol=1e-5, atol=1e-6 * T)
+    assert abs(ps.sum() - T) <= 1e-4 * T
+    got = oracle.balance_loss(counts.cpu().numpy(), ps, T, K)
+    assert got == pytest.approx(oracle.balance_loss(ref["counts"], ref["prob_sum"], T, K),
+                                rel=1e-5)
+
+
+def test_layer_k13_same_node_budget(M):
+    """K = 13 experts per token within the same 4 of 8 groups, the larger
+    expert count the pages give for the same communication budget."""
+    cfg = CONFIGS[1].with_(T=600, d=256, N=256, K=13, G=8, topG=4, f=256)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    layer, xd = _layer(M, cfg, x, R, b, W)
+    y = layer.forward(xd).float().cpu().numpy()
+    ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
+                             h_round="bf16")
+    _check_route(cfg, ref["route"], layer.topk_idx.cpu().numpy(),
+                 layer.topk_gate.cpu().numpy(), layer.counts.cpu().numpy())
+    _check_dispatch(layer, ref["route"])
+    assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
+    assert layer.device_status() == 0
+
+
 def test_layer_all_experts_every_token(M):
     """K = N: each expert's group holds every token (several m-tiles each)."""
     cfg = CONFIGS[1].with_(T=300, d=256, N=4, K=4, G=1, topG=1, f=256)
