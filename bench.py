@@ -378,6 +378,8 @@ def main():
             "device_status": r["status"],
             "load_max_over_mean": r["load_max_over_mean"],
         }
+        if r.get("softmax_route"):
+            line["softmax_route"] = r["softmax_route"]
         for k, v in extra.items():
             line[k] = {"workload": workload_name(v["cfg"]),
                        "value": world * v["cfg"].T * v["steps"] / (v["total_ms"] / 1e3),
@@ -457,6 +459,34 @@ def run_e2e(M, s, layer, x, w13, w2, s13, s2, cfg, steps, stream):
 
 
 GATHER = False  # set from --gather in main()
+
+
+def softmax_route_baseline(M, s, x, router, layer, cfg, stream, reps=20):
+    """The conventional softmax top-K router (moe_route_softmax) on the same
+    input, for contrast with the method's routing: time per call (CUDA events,
+    after 3 warm-up calls) and the balance statistic N * sum f_i P_i of its
+    selections (1 = uniform)."""
+    import torch
+    dev = x.device
+    idx = torch.empty(s.T, s.K, dtype=torch.int32, device=dev)
+    gate = torch.empty(s.T, s.K, dtype=torch.float32, device=dev)
+    cnt = torch.empty(s.N, dtype=torch.int32, device=dev)
+    psum = torch.empty(s.N, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        M.moe_route_softmax(s, x, router, idx, gate, cnt, psum, layer.ws, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        M.moe_route_softmax(s, x, router, idx, gate, cnt, psum, layer.ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    c = cnt.cpu().numpy().astype(np.float64)
+    P = psum.cpu().numpy().astype(np.float64) / s.T
+    f = c / (s.K * s.T)
+    return {"ms": e0.elapsed_time(e1) / reps, "balance": float(s.N * np.sum(f * P)),
+            "load_max_over_mean": float(c.max() / c.mean()),
+            "note": "softmax top-K over all experts, no bias or group limit (the baseline "
+                    "the method replaces); balance = N * sum_i f_i * P_i"}
 
 
 def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
@@ -541,8 +571,11 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
     status = layer.device_status()
 
     e2e_ms = None
+    baseline = None
     if e2e:
         e2e_ms = run_e2e(M, s, layer, x, w13, w2, s13, s2, cfg, steps, stream)
+        if cfg.dtype != "fp32":  # the softmax router takes bf16 activations
+            baseline = softmax_route_baseline(M, s, x, router, layer, cfg, stream)
 
     total_ms, e2e_ms = reduce_max([total_ms, e2e_ms or 0.0], pg, dev)
 
@@ -595,6 +628,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
                 "frac": achieved / P["hbm"], "peak_source": P["source"] + " copy",
                 "traffic": None, "experts_hit": used - 1}
     return {"cfg": cfg, "steps": steps, "total_ms": total_ms, "e2e_ms": e2e_ms,
+            "softmax_route": baseline,
             "phases_ms": {p: statistics.mean(v) for p, v in per_phase.items()},
             "roofline": roof,
             "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step, "flops": fl, "bytes": by},

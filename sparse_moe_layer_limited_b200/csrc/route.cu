@@ -306,14 +306,23 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z
     if (hist[e]) atomicAdd(&counts[e], hist[e]);
 }
 
-// prob_sum[e] = sum over the selection CTAs, in CTA order, of their partials.
+// prob_sum[e]: the selection CTAs' partials summed in a fixed order (eight
+// running sums over the CTAs b = j mod 8, then added j = 0..7), so the result
+// does not depend on scheduling.
 __global__ void prob_sum_kernel(const float* __restrict__ part, int nblocks, int N,
                                 float* __restrict__ prob_sum) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= N) return;
-  float a = 0.f;
-  for (int b = 0; b < nblocks; ++b) a += part[(size_t)b * N + e];
-  prob_sum[e] = a;
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int b = 0;
+  for (; b + 8 <= nblocks; b += 8)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] += part[(size_t)(b + j) * N + e];
+  for (int j = 0; b + j < nblocks; ++j) a[j] += part[(size_t)(b + j) * N + e];
+  float sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sum += a[j];
+  prob_sum[e] = sum;
 }
 
 }  // namespace
