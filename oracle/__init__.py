@@ -37,7 +37,8 @@ cases, the exhaustive E4M3 table, a hand-worked routing fixture).
 from .moe import (  # noqa: F401
     affinity, biased_scores, group_scores, kept_groups, route, route_margins,
     route_softmax, route_softmax_margins, balance_loss,
-    dispatch, swiglu_expert, expert_outputs, combine, bias_update, moe_forward,
+    dispatch, swiglu_expert, swiglu_expert_backward, expert_outputs, combine, bias_update,
+    moe_forward,
     round_bf16, silu,
 )
 from .fp8 import (  # noqa: F401

@@ -225,6 +225,40 @@ def swiglu_expert(a, w1, w3, w2, h_round: str = "none") -> np.ndarray:
     return h @ np.asarray(w2, np.float64).T
 
 
+def swiglu_expert_backward(a, w1, w3, w2, dy, gu_round: str = "none",
+                           dgu_round: str = "none") -> dict:
+    """Gradients of one expert FFN y = (silu(a W1^T) * (a W3^T)) W2^T given
+    dy = dL/dy [M, d].
+
+    [P1] §2.2: the backward pass runs COMBINE -> MLP_B (input gradients) ->
+    MLP_W (weight gradients) -> DISPATCH.  With g = a W1^T and u = a W3^T
+    (the gate and up products) and h = silu(g) * u, the chain rule gives
+        dh  = dy W2
+        dg  = dh * u * silu'(g),  silu'(g) = sigma(g) (1 + g (1 - sigma(g)))
+        du  = dh * silu(g)
+        da  = dg W1 + du W3
+        dW2 = dy^T h,  dW1 = dg^T a,  dW3 = du^T a
+    ``gu_round='bf16'``: g and u are the bf16 values a recompute stores;
+    ``dgu_round='bf16'``: dg and du are rounded to bf16 (a GEMM operand)
+    before the da and dW contractions.  Returns dict(da, dw1, dw3, dw2, dg,
+    du, dh)."""
+    a = np.asarray(a, dtype=np.float64)
+    w1, w3, w2 = (np.asarray(w, np.float64) for w in (w1, w3, w2))
+    dy = np.asarray(dy, dtype=np.float64)
+    g, u = a @ w1.T, a @ w3.T
+    if gu_round == "bf16":
+        g, u = round_bf16(g), round_bf16(u)
+    sig = 1.0 / (1.0 + np.exp(-g))
+    h = g * sig * u
+    dh = dy @ w2
+    dg = dh * u * sig * (1.0 + g * (1.0 - sig))
+    du = dh * g * sig
+    if dgu_round == "bf16":
+        dg, du = round_bf16(dg), round_bf16(du)
+    return dict(da=dg @ w1 + du @ w3, dw1=dg.T @ a, dw3=du.T @ a, dw2=dy.T @ h, dg=dg, du=du,
+                dh=dh)
+
+
 def expert_outputs(x, idx, get_weights, N: int, tokens=None, h_round: str = "none",
                    expert_fn=None) -> dict:
     """Per-expert outputs for the selected tokens.
