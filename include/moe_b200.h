@@ -208,6 +208,31 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
                             const int32_t* offsets, const void* w13, const void* w2,
                             void* y_perm, void* y_shared, void* ws, void* stream);
 
+/* Backward of the expert FFNs, input gradients ([P1] §2.2: the backward
+ * pass runs COMBINE -> MLP_B -> MLP_W -> DISPATCH; this is MLP_B), BF16 mode.
+ * With g = a W1^T, u = a W3^T (a = a dispatched row, or an x row for the
+ * shared expert) and dy the gradient of that expert's output row:
+ *   dh = dy W2;  dg = dh * u * silu'(g);  du = dh * silu(g);  da = dg W1 + du W3
+ * g and u are recomputed (GEMM1) and stored bf16; dh accumulates in fp32;
+ * dg, du are rounded to bf16 (operands of the last GEMM); da is bf16.
+ *   x_perm, offsets, x, w13   as at moe_expert_ffn
+ *   w13t [N+1, d, 2f], w2t [N+1, f, d]  bf16, from moe_transpose_weights
+ *   dy_perm [T*K, d], dy_shared [T, d]  bf16 output gradients (y_perm order)
+ *   dx_perm [T*K, d], dx_shared [T, d]  bf16 out: input gradients per
+ *              dispatched row and for the shared expert's rows
+ *   ws_bwd     moe_backward_workspace_size(shape) bytes; its first 256 bytes
+ *              are a status word like the forward workspace's (zero them once)
+ * MOE_ERR_UNSUPPORTED for other dtypes.  The weight gradients (MLP_W) are not
+ * provided. */
+size_t moe_backward_workspace_size(const moe_shape* shape);
+int moe_transpose_weights(const moe_shape* shape, const void* w13, const void* w2, void* w13t,
+                          void* w2t, void* stream);
+int moe_expert_ffn_backward_dx(const moe_shape* shape, const void* x_perm,
+                               const int32_t* offsets, const void* x, const void* w13,
+                               const void* w13t, const void* w2t, const void* dy_perm,
+                               const void* dy_shared, void* dx_perm, void* dx_shared,
+                               void* ws_bwd, void* stream);
+
 /* Combine ([P1] §2.2 COMBINE): y[t] = y_shared[t] + sum_k gate[t,k] *
  * y_perm[slot[t,k]], accumulated in fp32 in k order, rounded once to the
  * output dtype (fp32 in FP32 mode, else bf16).  No atomics: deterministic. */

@@ -51,6 +51,9 @@ _SIGS = {
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
     "moe_expert_ffn_gathered": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
+    "moe_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
+    "moe_transpose_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 5),
+    "moe_expert_ffn_backward_dx": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
     "moe_dispatch_noalloc": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, ctypes.c_float,
                                        _c_p]),
@@ -209,6 +212,26 @@ def moe_expert_ffn_gathered(s, x, perm_tok, offsets, w13, w2, y_perm, y_shared, 
     _expect(y_shared, x_torch_dtype(s), s.T * s.d, "y_shared")
     _call("moe_expert_ffn_gathered", ctypes.byref(s), _ptr(x), _ptr(perm_tok), _ptr(offsets),
           _ptr(w13), _ptr(w2), _ptr(y_perm), _ptr(y_shared), _ptr(ws), _stream(stream))
+
+
+def backward_workspace_size(s) -> int:
+    return lib().moe_backward_workspace_size(ctypes.byref(s))
+
+
+def moe_transpose_weights(s, w13, w2, w13t, w2t, stream=None):
+    _expect(w13t, w_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "w13t")
+    _expect(w2t, w_torch_dtype(s), (s.N + 1) * s.d * s.f, "w2t")
+    _call("moe_transpose_weights", ctypes.byref(s), _ptr(w13), _ptr(w2), _ptr(w13t), _ptr(w2t),
+          _stream(stream))
+
+
+def moe_expert_ffn_backward_dx(s, x_perm, offsets, x, w13, w13t, w2t, dy_perm, dy_shared,
+                               dx_perm, dx_shared, ws_bwd, stream=None):
+    _expect(dx_perm, x_torch_dtype(s), s.T * s.K * s.d, "dx_perm")
+    _expect(dx_shared, x_torch_dtype(s), s.T * s.d, "dx_shared")
+    _call("moe_expert_ffn_backward_dx", ctypes.byref(s), _ptr(x_perm), _ptr(offsets), _ptr(x),
+          _ptr(w13), _ptr(w13t), _ptr(w2t), _ptr(dy_perm), _ptr(dy_shared), _ptr(dx_perm),
+          _ptr(dx_shared), _ptr(ws_bwd), _stream(stream))
 
 
 def moe_combine(s, y_perm, y_shared, slot, topk_gate, y, stream=None):

@@ -213,6 +213,37 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
                             ws, static_cast<cudaStream_t>(stream));
 }
 
+size_t moe_backward_workspace_size(const moe_shape* shape) {
+  if (check(shape) != MOE_OK || shape->dtype != MOE_DTYPE_BF16) return 0;
+  return backward_ws_bytes(*shape);
+}
+
+int moe_transpose_weights(const moe_shape* shape, const void* w13, const void* w2, void* w13t,
+                          void* w2t, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(w13) || !ptr_ok(w2) || !ptr_ok(w13t) || !ptr_ok(w2t)) return MOE_ERR_ARG;
+  return cuda_status(launch_transpose_weights(*shape, w13, w2, w13t, w2t,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_ffn_backward_dx(const moe_shape* shape, const void* x_perm,
+                               const int32_t* offsets, const void* x, const void* w13,
+                               const void* w13t, const void* w2t, const void* dy_perm,
+                               const void* dy_shared, void* dx_perm, void* dx_shared,
+                               void* ws_bwd, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(x_perm) || !ptr_ok(offsets) || !ptr_ok(x) || !ptr_ok(w13) || !ptr_ok(w13t) ||
+      !ptr_ok(w2t) || !ptr_ok(dy_perm) || !ptr_ok(dy_shared) || !ptr_ok(dx_perm) ||
+      !ptr_ok(dx_shared) || !ptr_ok(ws_bwd))
+    return MOE_ERR_ARG;
+  return launch_ffn_bwd_dx_bf16(*shape, x_perm, offsets, x, w13, w13t, w2t, dy_perm, dy_shared,
+                                dx_perm, dx_shared, ws_bwd, static_cast<cudaStream_t>(stream));
+}
+
 int moe_combine(const moe_shape* shape, const void* y_perm, const void* y_shared,
                 const int32_t* slot, const float* topk_gate, void* y, void* stream) {
   int rc = check(shape);

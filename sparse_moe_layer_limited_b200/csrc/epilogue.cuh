@@ -18,4 +18,16 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) 
   for (int i = 0; i < 4; ++i) d4[i] = w[i];
 }
 
+// 8 bf16 (one 16-byte load) -> 8 fp32.
+__device__ __forceinline__ void bf16x8_load(const __nv_bfloat16* src, float* v) {
+  const uint4 w = *reinterpret_cast<const uint4*>(src);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
 }  // namespace moe

@@ -62,7 +62,7 @@ constexpr int kABytes = BM * BK * 2;
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiScores = 2 };
+enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiScores = 2, kEpiSwiGLUBwd = 3 };
 
 template <int kBN>
 struct TileCfg {
@@ -86,6 +86,11 @@ struct alignas(64) GemmArgs {
   __nv_bfloat16* out_routed;
   __nv_bfloat16* out_shared;
   float* out_f32;   // score epilogue: fp32 partial sums [k_splits, T, n_valid]
+  // SwiGLU-backward epilogue: the stored gate/up products [rows, 2f] (packed
+  // like W13: per 128 features, gate columns then up columns), routed rows at
+  // offsets[g] + r of aux_routed, shared-expert rows r of aux_shared
+  const __nv_bfloat16* aux_routed;
+  const __nv_bfloat16* aux_shared;
   uint32_t* status;
   int N, T;
   int rows_routed;  // T*K
@@ -403,6 +408,38 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
           if (valid) store_row32(orow + n * BN + c, y);
         }
+      } else if constexpr (kEpi == kEpiSwiGLUBwd) {
+        // the accumulator is dh for hidden features n*BN + c; with g, u the
+        // stored gate/up products: dg = dh * u * silu'(g), du = dh * silu(g),
+        // written bf16 into the packed [rows, 2f] layout (gate block, up block)
+        const __nv_bfloat16* arow =
+            (g < args.N) ? args.aux_routed + (size_t)(args.offsets[g] + r) * args.out_ld
+                         : args.aux_shared + (size_t)r * args.out_ld;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          const int j0 = n * BN + c;                       // first feature of the chunk
+          const int col = (j0 / 128) * 256 + (j0 % 128);   // its gate column; up at +128
+          if (valid) {
+            float gt[32], up[32], dg[32], du[32];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              bf16x8_load(arow + col + 8 * q4, gt + 8 * q4);
+              bf16x8_load(arow + col + 128 + 8 * q4, up + 8 * q4);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float dh = __uint_as_float(v[i]);
+              const float sg = 1.f / (1.f + expf(-gt[i]));
+              dg[i] = dh * up[i] * (sg * (1.f + gt[i] * (1.f - sg)));
+              du[i] = dh * (gt[i] * sg);
+            }
+            store_row32(orow + col, dg);
+            store_row32(orow + col + 128, du);
+          }
+        }
       } else {  // raw fp32 scores of this K split, columns < n_valid
         float* srow = args.out_f32 +
                       ((size_t)(n % args.k_splits) * args.T + r) * args.n_valid;
@@ -602,6 +639,91 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
                   : bn == 128 ? launch_gemm<kEpiScores, 128>(a, st)
                               : launch_gemm<kEpiScores, 256>(a, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Backward of the expert FFNs, input gradients ([P1] §2.2 MLP_B), bf16:
+//   GU  = [x_perm | x] W13^T      (GEMM1 recomputed, gate/up stored bf16)
+//   dGU = SwiGLU'(dY W2, GU)      (dH in fp32 in TMEM; dg, du bf16 per feature)
+//   dX  = dGU W13                 (against W13^T, K = 2f)
+// Three launches of the grouped kernel; W2^T and W13^T come from
+// moe_transpose_weights.  ws_bwd: status word, GU and dGU (backward_ws_bytes).
+size_t backward_ws_bytes(const moe_shape& s) {
+  const size_t rows = (size_t)s.T * s.K + s.T;
+  const size_t gu = (rows * 2 * s.f * 2 + 255) & ~size_t(255);
+  return 256 + 2 * gu;
+}
+
+int launch_ffn_bwd_dx_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                           const void* x, const void* w13, const void* w13t, const void* w2t,
+                           const void* dy_perm, const void* dy_shared, void* dx_perm,
+                           void* dx_shared, void* ws_bwd, cudaStream_t st) {
+  uint8_t* w = static_cast<uint8_t*>(ws_bwd);
+  const uint64_t TK = (uint64_t)s.T * s.K;
+  const size_t rows = TK + s.T;
+  const size_t gu_bytes = (rows * 2 * s.f * 2 + 255) & ~size_t(255);
+  __nv_bfloat16* GU = reinterpret_cast<__nv_bfloat16*>(w + 256);
+  __nv_bfloat16* dGU = reinterpret_cast<__nv_bfloat16*>(w + 256 + gu_bytes);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w);
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t twof = 2ull * s.f;
+
+  auto base_args = [&](GemmArgs& a) {
+    a.offsets = offsets;
+    a.status = status;
+    a.N = s.N;
+    a.T = s.T;
+    a.rows_routed = (int)TK;
+    a.a_rep = 1;
+    a.k_splits = 1;
+  };
+  // 1. GU = A W13^T (routed rows from x_perm, shared rows from x)
+  GemmArgs g1{};
+  bool ok = make_map(&g1.tmA_routed, x_perm, BF, 2, s.d, TK, BK, BM) &&
+            make_map(&g1.tmA_shared, x, BF, 2, s.d, s.T, BK, BM) &&
+            make_map(&g1.tmB, w13, BF, 2, s.d, (uint64_t)(s.N + 1) * twof, BK, 256);
+  // 2. dH = dY W2 (B = W2^T, [f, d] per expert), SwiGLU-backward epilogue -> dGU
+  GemmArgs g2{};
+  ok = ok && make_map(&g2.tmA_routed, dy_perm, BF, 2, s.d, TK, BK, BM) &&
+       make_map(&g2.tmA_shared, dy_shared, BF, 2, s.d, s.T, BK, BM) &&
+       make_map(&g2.tmB, w2t, BF, 2, s.d, (uint64_t)(s.N + 1) * s.f, BK, 256);
+  // 3. dX = dGU W13 (B = W13^T, [d, 2f] per expert)
+  GemmArgs g3{};
+  ok = ok && make_map(&g3.tmA_routed, dGU, BF, 2, twof, rows, BK, BM) &&
+       make_map(&g3.tmA_shared, dGU, BF, 2, twof, rows, BK, BM) &&
+       make_map(&g3.tmB, w13t, BF, 2, twof, (uint64_t)(s.N + 1) * s.d, BK, 256);
+  if (!ok) {
+    note_text("expert backward: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
+  base_args(g1);
+  g1.out_routed = GU;
+  g1.out_shared = GU + TK * twof;
+  g1.a_shared_row0 = 0;
+  g1.n_acc = (int)twof;
+  g1.k_dim = s.d;
+  g1.out_ld = (int)twof;
+  if (launch_gemm<kEpiStore, 256>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  base_args(g2);
+  g2.aux_routed = GU;
+  g2.aux_shared = GU + TK * twof;
+  g2.out_routed = dGU;
+  g2.out_shared = dGU + TK * twof;
+  g2.a_shared_row0 = 0;
+  g2.n_acc = s.f;
+  g2.k_dim = s.d;
+  g2.out_ld = (int)twof;
+  if (launch_gemm<kEpiSwiGLUBwd, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  base_args(g3);
+  g3.out_routed = static_cast<__nv_bfloat16*>(dx_perm);
+  g3.out_shared = static_cast<__nv_bfloat16*>(dx_shared);
+  g3.a_shared_row0 = (int)TK;
+  g3.n_acc = s.d;
+  g3.k_dim = (int)twof;
+  g3.out_ld = s.d;
+  if (launch_gemm<kEpiStore, 256>(g3, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 }  // namespace moe

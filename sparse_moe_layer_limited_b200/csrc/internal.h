@@ -92,6 +92,14 @@ int router_k_splits(const moe_shape& s);
 int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* Z,
                             int k_splits, void* ws, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* status (tensor maps can fail to encode).
+// Expert backward, input gradients (bf16); ws_bwd of backward_ws_bytes(s).
+size_t backward_ws_bytes(const moe_shape& s);
+int launch_ffn_bwd_dx_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                           const void* x, const void* w13, const void* w13t, const void* w2t,
+                           const void* dy_perm, const void* dy_shared, void* dx_perm,
+                           void* dx_shared, void* ws_bwd, cudaStream_t st);
+cudaError_t launch_transpose_weights(const moe_shape& s, const void* w13, const void* w2,
+                                     void* w13t, void* w2t, cudaStream_t st);
 // bf16 expert GEMMs; with perm_tok set, GEMM1 gathers the routed rows from x
 // (x_perm unused), else it reads x_perm.
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* perm_tok,

@@ -158,4 +158,35 @@ cudaError_t launch_pack_w13(const moe_shape& s, const void* w1, const void* w3, 
   return cudaGetLastError();
 }
 
+// [B, R, C] bf16 -> [B, C, R]: 32x32 tiles through shared memory (padded
+// against bank conflicts), block (32, 8).
+namespace {
+__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src,
+                                      __nv_bfloat16* __restrict__ dst, int R, int C) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const size_t b = blockIdx.z;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < R && c < C) tile[i][threadIdx.x] = src[(b * R + r) * C + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < C && r < R) dst[(b * C + c) * R + r] = tile[threadIdx.x][i];
+  }
+}
+}  // namespace
+
+cudaError_t launch_transpose_weights(const moe_shape& s, const void* w13, const void* w2,
+                                     void* w13t, void* w2t, cudaStream_t st) {
+  const dim3 blk(32, 8);
+  const unsigned E = (unsigned)(s.N + 1);
+  transpose_bf16_kernel<<<dim3((s.d + 31) / 32, (2 * s.f + 31) / 32, E), blk, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w13), static_cast<__nv_bfloat16*>(w13t), 2 * s.f, s.d);
+  transpose_bf16_kernel<<<dim3((s.f + 31) / 32, (s.d + 31) / 32, E), blk, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w2), static_cast<__nv_bfloat16*>(w2t), s.d, s.f);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -1,0 +1,69 @@
+"""Expert backward, input gradients (moe_expert_ffn_backward_dx) against the
+oracle's SwiGLU backward, and the weight transposes it uses."""
+import numpy as np
+import pytest
+
+import oracle
+from synth import CONFIGS, gen
+from tests import support as S
+
+pytestmark = pytest.mark.gpu
+TOL_BF16 = 1e-2
+
+
+@pytest.fixture(scope="module")
+def M():
+    import sparse_moe_layer_limited_b200 as M
+    return M
+
+
+def _grads(cfg, seed):
+    """Seeded output gradients dy_perm [T*K, d] and dy_shared [T, d] (bf16 values)."""
+    dyp = gen.make_x(cfg.with_(T=cfg.T * cfg.K), seed=seed)
+    dys = gen.make_x(cfg, seed=seed + 1)
+    return dyp, dys
+
+
+@pytest.mark.parametrize("T", [600, 129, 1])
+def test_backward_dx_matches_oracle(M, T):
+    import torch
+    cfg = CONFIGS[1].with_(T=T, d=256, N=8, K=2, G=2, topG=1, f=256)
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    s = S.moe_shape(cfg)
+    layer = M.MoELayer(s, torch.from_numpy(R).cuda(),
+                       torch.from_numpy(np.asarray(b, np.float32)).cuda(), W["w13"], W["w2"],
+                       gamma=cfg.gamma)
+    xd = S.to_dev_x(x, cfg)
+    layer.forward(xd, update_bias=False)
+    w13t = torch.empty(cfg.N + 1, cfg.d, 2 * cfg.f, dtype=torch.bfloat16, device="cuda")
+    w2t = torch.empty(cfg.N + 1, cfg.f, cfg.d, dtype=torch.bfloat16, device="cuda")
+    M.moe_transpose_weights(s, W["w13"], W["w2"], w13t, w2t)
+    torch.cuda.synchronize()
+    assert torch.equal(w13t, W["w13"].transpose(1, 2))
+    assert torch.equal(w2t, W["w2"].transpose(1, 2))
+
+    dyp, dys = _grads(cfg, 31)
+    dyp_d, dys_d = S.to_dev_x(dyp, cfg), S.to_dev_x(dys, cfg)
+    dxp = torch.empty_like(layer.x_perm)
+    dxs = torch.empty_like(xd)
+    ws = torch.zeros(M.backward_workspace_size(s), dtype=torch.uint8, device="cuda")
+    M.moe_expert_ffn_backward_dx(s, layer.x_perm, layer.offsets, xd, W["w13"], w13t, w2t,
+                                 dyp_d, dys_d, dxp, dxs, ws)
+    assert M.moe_read_device_status(ws) == 0
+
+    get = S.host_weights(cfg)
+    offs = layer.offsets.cpu().numpy()
+    perm = layer.perm_tok.cpu().numpy()
+    dxp_h = dxp.float().cpu().numpy()
+    for e in range(cfg.N):
+        a, z = offs[e], offs[e + 1]
+        if z == a:
+            continue
+        want = oracle.swiglu_expert_backward(x[perm[a:z]], *get(e), dyp[a:z], gu_round="bf16",
+                                             dgu_round="bf16")["da"]
+        assert S.rel_fro(dxp_h[a:z], want) <= TOL_BF16, e
+    want = oracle.swiglu_expert_backward(x, *get(cfg.N), dys, gu_round="bf16",
+                                         dgu_round="bf16")["da"]
+    assert S.rel_fro(dxs.float().cpu().numpy(), want) <= TOL_BF16
