@@ -351,6 +351,9 @@ def main():
         extra["fp8"] = run_layer(BY_NAME["v3_fp8"], dev, max(5, args.steps // 5), 3, pg, local)
         extra["decode"] = run_layer(BY_NAME["decode_zipf"], dev, max(20, args.steps), 3, pg,
                                     local)
+    bwd = None
+    if not args.no_extra and cfg.dtype == "bf16" and world == 1:
+        bwd = run_backward(cfg, dev)
 
     if rank == 0:
         P = peaks()
@@ -388,6 +391,8 @@ def main():
                        "layer_roofline": v["layer_roofline"], "phases_ms": v["phases_ms"],
                        "clocks": v["clocks"], "device_status": v["status"],
                        "load_max_over_mean": v["load_max_over_mean"]}
+        if bwd is not None:
+            line["backward_dx"] = bwd
         if world == 1 and not args.no_cpu_baseline:
             v, cores, note = cpu_oracle_baseline(cfg, args.cpu_sample)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
@@ -459,6 +464,62 @@ def run_e2e(M, s, layer, x, w13, w2, s13, s2, cfg, steps, stream):
 
 
 GATHER = False  # set from --gather in main()
+
+
+def run_backward(cfg, dev, calls=10, warmup=3):
+    """The expert backward, input gradients (moe_expert_ffn_backward_dx), on the
+    layer's routing of one synthetic batch: GEMM1 recomputed, dY W2^T with the
+    SwiGLU-backward epilogue, dGU W13 -- 10*d*f FLOP per dispatched or shared
+    row.  dY is seeded synthetic N(0, 1) bf16.  CUDA events over `calls` calls
+    after `warmup`."""
+    import torch
+    import sparse_moe_layer_limited_b200 as M
+    from synth import device as sdev
+    s = M.shape(cfg.T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f, M.DTYPE_BF16)
+    w1 = sdev.expert_weights_bf16(cfg, 0, "w1", dev)
+    w3 = sdev.expert_weights_bf16(cfg, 0, "w3", dev)
+    w13 = torch.empty(cfg.N + 1, 2 * cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
+    M.moe_pack_w13(s, w1, w3, w13)
+    del w1, w3
+    w2 = sdev.expert_weights_bf16(cfg, 0, "w2", dev)
+    w13t = torch.empty(cfg.N + 1, cfg.d, 2 * cfg.f, dtype=torch.bfloat16, device=dev)
+    w2t = torch.empty(cfg.N + 1, cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
+    M.moe_transpose_weights(s, w13, w2, w13t, w2t)
+    router = torch.from_numpy(gen.make_router(cfg)).to(dev)
+    bias = torch.from_numpy(gen.make_bias(cfg)).to(dev)
+    layer = M.MoELayer(s, router, bias, w13, w2, gamma=cfg.gamma)
+    x = sdev.x_bf16(cfg, 0, device=dev)
+    layer.forward(x, update_bias=False)
+    g = torch.Generator(device=dev).manual_seed(7)
+    dyp = torch.randn(cfg.T * cfg.K, cfg.d, generator=g, device=dev).to(torch.bfloat16)
+    dys = torch.randn(cfg.T, cfg.d, generator=g, device=dev).to(torch.bfloat16)
+    dxp, dxs = torch.empty_like(dyp), torch.empty_like(dys)
+    ws = torch.zeros(M.backward_workspace_size(s), dtype=torch.uint8, device=dev)
+
+    def call():
+        M.moe_expert_ffn_backward_dx(s, layer.x_perm, layer.offsets, x, w13, w13t, w2t, dyp, dys,
+                                     dxp, dxs, ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / calls
+    status = M.moe_read_device_status(ws)
+    fl = 10.0 * cfg.d * cfg.f * (cfg.T * cfg.K + cfg.T)
+    P = peaks()
+    achieved = fl / (ms / 1e3) / 1e12
+    return {"workload": workload_name(cfg), "ms": ms, "tokens_per_s": cfg.T / (ms / 1e3),
+            "roofline": {"bound": "tensor", "achieved": achieved, "unit": "TFLOP/s",
+                         "peak": P["bf16_sustained"], "frac": achieved / P["bf16_sustained"],
+                         "flops_per_call": fl},
+            "gpu_launches_per_call": 3, "device_status": status,
+            "note": "expert FFN input gradients (GEMM1 recomputed, dh with the SwiGLU-backward "
+                    "epilogue, dx); weight gradients not built"}
 
 
 def softmax_route_baseline(M, s, x, router, layer, cfg, stream, reps=20):

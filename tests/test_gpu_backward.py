@@ -67,3 +67,42 @@ def test_backward_dx_matches_oracle(M, T):
     want = oracle.swiglu_expert_backward(x, *get(cfg.N), dys, gu_round="bf16",
                                          dgu_round="bf16")["da"]
     assert S.rel_fro(dxs.float().cpu().numpy(), want) <= TOL_BF16
+
+
+def test_v3_backward_dx_sampled(M):
+    """The full V3 layer shape: input gradients of three routed experts (every
+    row) and of 192 shared-expert rows against the oracle (rows are
+    independent in the backward, so the oracle takes only the sampled ones)."""
+    import torch
+    cfg = CONFIGS[2]
+    R, b = gen.make_router(cfg), gen.make_bias(cfg)
+    x, _ = S.tie_free_x(cfg, R, b)
+    W = S.device_weights(cfg)
+    s = S.moe_shape(cfg)
+    layer = M.MoELayer(s, torch.from_numpy(R).cuda(),
+                       torch.from_numpy(np.asarray(b, np.float32)).cuda(), W["w13"], W["w2"],
+                       gamma=cfg.gamma)
+    xd = S.to_dev_x(x, cfg)
+    layer.forward(xd, update_bias=False)
+    w13t = torch.empty(cfg.N + 1, cfg.d, 2 * cfg.f, dtype=torch.bfloat16, device="cuda")
+    w2t = torch.empty(cfg.N + 1, cfg.f, cfg.d, dtype=torch.bfloat16, device="cuda")
+    M.moe_transpose_weights(s, W["w13"], W["w2"], w13t, w2t)
+    dyp, dys = _grads(cfg, 41)
+    dxp = torch.empty_like(layer.x_perm)
+    dxs = torch.empty_like(xd)
+    ws = torch.zeros(M.backward_workspace_size(s), dtype=torch.uint8, device="cuda")
+    M.moe_expert_ffn_backward_dx(s, layer.x_perm, layer.offsets, xd, W["w13"], w13t, w2t,
+                                 S.to_dev_x(dyp, cfg), S.to_dev_x(dys, cfg), dxp, dxs, ws)
+    assert M.moe_read_device_status(ws) == 0
+    get = S.streaming_weights(cfg)
+    offs = layer.offsets.cpu().numpy()
+    perm = layer.perm_tok.cpu().numpy()
+    for e in (0, 101, 255):
+        a, z = offs[e], offs[e + 1]
+        want = oracle.swiglu_expert_backward(x[perm[a:z]], *get(e), dyp[a:z], gu_round="bf16",
+                                             dgu_round="bf16")["da"]
+        assert S.rel_fro(dxp[a:z].float().cpu().numpy(), want) <= TOL_BF16, e
+    rows = np.random.default_rng(3).choice(cfg.T, 192, replace=False)
+    want = oracle.swiglu_expert_backward(x[rows], *get(cfg.N), dys[rows], gu_round="bf16",
+                                         dgu_round="bf16")["da"]
+    assert S.rel_fro(dxs.float().cpu().numpy()[rows], want) <= TOL_BF16
