@@ -222,8 +222,7 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
  *              dispatched row and for the shared expert's rows
  *   ws_bwd     moe_backward_workspace_size(shape) bytes; its first 256 bytes
  *              are a status word like the forward workspace's (zero them once)
- * MOE_ERR_UNSUPPORTED for other dtypes.  The weight gradients (MLP_W) are not
- * provided. */
+ * MOE_ERR_UNSUPPORTED for other dtypes. */
 size_t moe_backward_workspace_size(const moe_shape* shape);
 int moe_transpose_weights(const moe_shape* shape, const void* w13, const void* w2, void* w13t,
                           void* w2t, void* stream);
@@ -232,6 +231,21 @@ int moe_expert_ffn_backward_dx(const moe_shape* shape, const void* x_perm,
                                const void* w13t, const void* w2t, const void* dy_perm,
                                const void* dy_shared, void* dx_perm, void* dx_shared,
                                void* ws_bwd, void* stream);
+
+/* moe_expert_ffn_backward_dw: the weight gradients ([P1] §2.2 MLP_W), BF16
+ * mode with f % 256 == 0, to be called after moe_expert_ffn_backward_dx with
+ * the same ws_bwd (it reads the g, u and dg, du that call leaves there):
+ *   dW2_e = dY_e^T H_e,  H = silu(g) * u          -> dw2  [N+1, d, f]
+ *   dW13_e = [dg du]_e^T A_e (packed like W13)     -> dw13 [N+1, 2f, d]
+ * for every routed expert e on its dispatched rows and the shared expert on
+ * x.  Each product contracts over the expert's rows in fp32 (tensor cores,
+ * the rows transposed into zero-padded per-expert column blocks first); the
+ * gradients are bf16.  An expert without rows gets zeros.
+ *   x_perm, offsets, x, dy_perm, dy_shared   as at the _dx call */
+int moe_expert_ffn_backward_dw(const moe_shape* shape, const void* x_perm,
+                               const int32_t* offsets, const void* x, const void* dy_perm,
+                               const void* dy_shared, void* dw13, void* dw2, void* ws_bwd,
+                               void* stream);
 
 /* Combine ([P1] §2.2 COMBINE): y[t] = y_shared[t] + sum_k gate[t,k] *
  * y_perm[slot[t,k]], accumulated in fp32 in k order, rounded once to the

@@ -54,6 +54,7 @@ _SIGS = {
     "moe_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
     "moe_transpose_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 5),
     "moe_expert_ffn_backward_dx": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
+    "moe_expert_ffn_backward_dw": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_dispatch_noalloc": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, ctypes.c_float,
                                        _c_p]),
@@ -232,6 +233,14 @@ def moe_expert_ffn_backward_dx(s, x_perm, offsets, x, w13, w13t, w2t, dy_perm, d
     _call("moe_expert_ffn_backward_dx", ctypes.byref(s), _ptr(x_perm), _ptr(offsets), _ptr(x),
           _ptr(w13), _ptr(w13t), _ptr(w2t), _ptr(dy_perm), _ptr(dy_shared), _ptr(dx_perm),
           _ptr(dx_shared), _ptr(ws_bwd), _stream(stream))
+
+
+def moe_expert_ffn_backward_dw(s, x_perm, offsets, x, dy_perm, dy_shared, dw13, dw2, ws_bwd,
+                               stream=None):
+    _expect(dw13, w_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "dw13")
+    _expect(dw2, w_torch_dtype(s), (s.N + 1) * s.d * s.f, "dw2")
+    _call("moe_expert_ffn_backward_dw", ctypes.byref(s), _ptr(x_perm), _ptr(offsets), _ptr(x),
+          _ptr(dy_perm), _ptr(dy_shared), _ptr(dw13), _ptr(dw2), _ptr(ws_bwd), _stream(stream))
 
 
 def moe_combine(s, y_perm, y_shared, slot, topk_gate, y, stream=None):

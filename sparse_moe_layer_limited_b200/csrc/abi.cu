@@ -244,6 +244,20 @@ int moe_expert_ffn_backward_dx(const moe_shape* shape, const void* x_perm,
                                 dx_perm, dx_shared, ws_bwd, static_cast<cudaStream_t>(stream));
 }
 
+int moe_expert_ffn_backward_dw(const moe_shape* shape, const void* x_perm,
+                               const int32_t* offsets, const void* x, const void* dy_perm,
+                               const void* dy_shared, void* dw13, void* dw2, void* ws_bwd,
+                               void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_BF16 || shape->f % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(x_perm) || !ptr_ok(offsets) || !ptr_ok(x) || !ptr_ok(dy_perm) ||
+      !ptr_ok(dy_shared) || !ptr_ok(dw13) || !ptr_ok(dw2) || !ptr_ok(ws_bwd))
+    return MOE_ERR_ARG;
+  return launch_ffn_bwd_dw_bf16(*shape, x_perm, offsets, x, dy_perm, dy_shared, dw13, dw2,
+                                ws_bwd, static_cast<cudaStream_t>(stream));
+}
+
 int moe_combine(const moe_shape* shape, const void* y_perm, const void* y_shared,
                 const int32_t* slot, const float* topk_gate, void* y, void* stream) {
   int rc = check(shape);

@@ -646,12 +646,35 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
 //   dGU = SwiGLU'(dY W2, GU)      (dH in fp32 in TMEM; dg, du bf16 per feature)
 //   dX  = dGU W13                 (against W13^T, K = 2f)
 // Three launches of the grouped kernel; W2^T and W13^T come from
-// moe_transpose_weights.  ws_bwd: status word, GU and dGU (backward_ws_bytes).
-size_t backward_ws_bytes(const moe_shape& s) {
+// moe_transpose_weights.  ws_bwd (bwd_layout): status word, GU and dGU, which
+// the weight-gradient pass (gemm_wgrad.cu) reads afterwards.
+BwdLayout bwd_layout(const moe_shape& s) {
+  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
+  BwdLayout B;
   const size_t rows = (size_t)s.T * s.K + s.T;
-  const size_t gu = (rows * 2 * s.f * 2 + 255) & ~size_t(255);
-  return 256 + 2 * gu;
+  const size_t R = (size_t)wgrad_cols(s);
+  size_t off = 256;
+  B.gu = off;
+  off = al(off + rows * 2 * s.f * 2);
+  B.dgu = off;
+  off = al(off + rows * 2 * s.f * 2);
+  B.colbase = off;
+  off = al(off + (size_t)(s.N + 2) * 4);
+  B.col_of_row = off;
+  off = al(off + rows * 4);
+  B.at = off;
+  off = al(off + (size_t)s.d * R * 2);
+  B.dyt = off;
+  off = al(off + (size_t)s.d * R * 2);
+  B.ht = off;
+  off = al(off + (size_t)s.f * R * 2);
+  B.dgut = off;
+  off = al(off + (size_t)2 * s.f * R * 2);
+  B.total = off;
+  return B;
 }
+
+size_t backward_ws_bytes(const moe_shape& s) { return bwd_layout(s).total; }
 
 int launch_ffn_bwd_dx_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                            const void* x, const void* w13, const void* w13t, const void* w2t,
@@ -660,9 +683,9 @@ int launch_ffn_bwd_dx_bf16(const moe_shape& s, const void* x_perm, const int32_t
   uint8_t* w = static_cast<uint8_t*>(ws_bwd);
   const uint64_t TK = (uint64_t)s.T * s.K;
   const size_t rows = TK + s.T;
-  const size_t gu_bytes = (rows * 2 * s.f * 2 + 255) & ~size_t(255);
-  __nv_bfloat16* GU = reinterpret_cast<__nv_bfloat16*>(w + 256);
-  __nv_bfloat16* dGU = reinterpret_cast<__nv_bfloat16*>(w + 256 + gu_bytes);
+  const BwdLayout B = bwd_layout(s);
+  __nv_bfloat16* GU = reinterpret_cast<__nv_bfloat16*>(w + B.gu);
+  __nv_bfloat16* dGU = reinterpret_cast<__nv_bfloat16*>(w + B.dgu);
   uint32_t* status = reinterpret_cast<uint32_t*>(w);
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t twof = 2ull * s.f;

@@ -92,8 +92,19 @@ int router_k_splits(const moe_shape& s);
 int launch_router_scores_tc(const moe_shape& s, const void* x, const float* router, float* Z,
                             int k_splits, void* ws, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* status (tensor maps can fail to encode).
-// Expert backward, input gradients (bf16); ws_bwd of backward_ws_bytes(s).
+// Expert backward workspace: status word, the recomputed gate/up GU and the
+// input pass's dGU [T*K+T, 2f] bf16, then the weight-gradient pass's column
+// blocks and transposed operands (gemm_wgrad.cu).
+struct BwdLayout {
+  size_t gu = 0, dgu = 0, colbase = 0, col_of_row = 0, at = 0, dyt = 0, ht = 0, dgut = 0;
+  size_t total = 0;
+};
+long long wgrad_cols(const moe_shape& s);
+BwdLayout bwd_layout(const moe_shape& s);
 size_t backward_ws_bytes(const moe_shape& s);
+int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                           const void* x, const void* dy_perm, const void* dy_shared,
+                           void* dw13, void* dw2, void* ws_bwd, cudaStream_t st);
 int launch_ffn_bwd_dx_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                            const void* x, const void* w13, const void* w13t, const void* w2t,
                            const void* dy_perm, const void* dy_shared, void* dx_perm,
