@@ -42,7 +42,8 @@ def parse():
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--cpu-sample", type=int, default=2, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak", "mma"], default=None,
+    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak", "mma", "backward"],
+                   default=None,
                    help="measurement probes behind the profiles: expert GEMMs on uniform "
                         "expert loads, cuBLAS batched GEMM at the expert shapes, FP8 GEMM peak")
     p.add_argument("--rows", type=int, default=256, help="rows per expert for --probe uniform")
@@ -264,7 +265,13 @@ def run_probe(args, cfg):
     cublas:  torch.bmm over N experts x 256 rows at the expert GEMM shapes (the
              ideal grouped problem, routed part only), and a dense GEMM;
     fp8peak: torch._scaled_mm E4M3 8192^3, best of 10;
-    mma:     the tcgen05.mma issue-rate probe (SM cycles per instruction shape)."""
+    mma:     the tcgen05.mma issue-rate probe (SM cycles per instruction shape);
+    backward: the expert backward (input and weight gradients) alone."""
+    if args.probe == "backward":
+        import torch
+        out = run_backward(cfg, torch.device("cuda"))
+        print(json.dumps(out), flush=True)
+        return out
     if args.probe == "mma":
         import subprocess
         from sparse_moe_layer_limited_b200 import build as B
@@ -496,30 +503,49 @@ def run_backward(cfg, dev, calls=10, warmup=3):
     dxp, dxs = torch.empty_like(dyp), torch.empty_like(dys)
     ws = torch.zeros(M.backward_workspace_size(s), dtype=torch.uint8, device=dev)
 
-    def call():
+    dw13, dw2 = torch.empty_like(w13), torch.empty_like(w2)
+
+    def call_dx():
         M.moe_expert_ffn_backward_dx(s, layer.x_perm, layer.offsets, x, w13, w13t, w2t, dyp, dys,
                                      dxp, dxs, ws)
-    for _ in range(warmup):
-        call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(calls):
-        call()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / calls
+
+    def call_dw():
+        M.moe_expert_ffn_backward_dw(s, layer.x_perm, layer.offsets, x, dyp, dys, dw13, dw2, ws)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(calls):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / calls
+
+    ms = timed(call_dx)
+    call_dx()                # the weight pass reads what the input pass leaves in ws
+    ms_dw = timed(call_dw)
     status = M.moe_read_device_status(ws)
-    fl = 10.0 * cfg.d * cfg.f * (cfg.T * cfg.K + cfg.T)
+    rows = cfg.T * cfg.K + cfg.T
+    fl = 10.0 * cfg.d * cfg.f * rows
+    fl_dw = 6.0 * cfg.d * cfg.f * rows
     P = peaks()
+    pk = P["bf16_sustained"]
     achieved = fl / (ms / 1e3) / 1e12
+    achieved_dw = fl_dw / (ms_dw / 1e3) / 1e12
     return {"workload": workload_name(cfg), "ms": ms, "tokens_per_s": cfg.T / (ms / 1e3),
             "roofline": {"bound": "tensor", "achieved": achieved, "unit": "TFLOP/s",
-                         "peak": P["bf16_sustained"], "frac": achieved / P["bf16_sustained"],
-                         "flops_per_call": fl},
+                         "peak": pk, "frac": achieved / pk, "flops_per_call": fl},
             "gpu_launches_per_call": 3, "device_status": status,
-            "note": "expert FFN input gradients (GEMM1 recomputed, dh with the SwiGLU-backward "
-                    "epilogue, dx); weight gradients not built"}
+            "weight_gradients": {"ms": ms_dw, "achieved": achieved_dw, "unit": "TFLOP/s",
+                                 "frac": achieved_dw / pk, "flops_per_call": fl_dw,
+                                 "gpu_launches_per_call": 12,
+                                 "note": "dW2 and dW13 of every expert (6 d f FLOP per row), "
+                                         "including the transposes into per-expert blocks"},
+            "note": "expert FFN input gradients: GEMM1 recomputed, dh with the SwiGLU-backward "
+                    "epilogue, dx (3 launches); weight gradients beside them"}
 
 
 def softmax_route_baseline(M, s, x, router, layer, cfg, stream, reps=20):

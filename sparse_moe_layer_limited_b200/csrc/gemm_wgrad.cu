@@ -13,8 +13,8 @@
 // Then one persistent tensor-core kernel runs all products: a unit is one
 // 128 x 256 output tile of one expert, its K loop the expert's column block
 // (tcgen05.mma cta_group::1, M=128, N=256, K=16, fp32 accumulate in TMEM,
-// two accumulators in turn), the tile is rounded to bf16 and stored into the
-// gradient laid out like the weight.  An expert without rows gets zeros.
+// two accumulators in turn); eight epilogue warps round the tile to bf16 and
+// store it into the gradient laid out like the weight.  An expert without rows gets zeros.
 // Every mbarrier wait is bounded (~2 s) and sets the device status word.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,7 +31,7 @@ constexpr int WStages = 4;
 constexpr int WABytes = WBM * WBK * 2;
 constexpr int WBBytes = WBN * WBK * 2;
 constexpr int WStageBytes = WABytes + WBBytes;
-constexpr int WThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int WThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue (2 per quadrant)
 constexpr uint64_t WTimeoutNs = 2000000000ull;
 
 // ---- layout: column blocks per group --------------------------------------------
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -270,7 +270,10 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
       mbar_wait_bounded(drain, 0, args.status, WTimeoutNs / 8);
     }
   } else {
+    // units are short (a few K blocks) and each stores a 64 KB tile, so two
+    // warps per TMEM lane quadrant drain it, 128 columns each
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     int local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
                                            args.N_total + (size_t)n * WBN;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * WBN;
 #pragma unroll 1
-      for (int c = 0; c < WBN; c += 32) {
+      for (int c = half * (WBN / 2); c < (half + 1) * (WBN / 2); c += 32) {
         float y[32];
         if (kcnt > 0) {  // a group without rows has a zero gradient
           uint32_t v[32];
