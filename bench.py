@@ -527,6 +527,8 @@ def run_backward(cfg, dev, calls=10, warmup=3):
     ms = timed(call_dx)
     call_dx()                # the weight pass reads what the input pass leaves in ws
     ms_dw = timed(call_dw)
+    ms_wt = timed(lambda: M.moe_transpose_weights(s, w13, w2, w13t, w2t))
+    wt_bytes = 2.0 * 2 * (cfg.N + 1) * 3 * cfg.d * cfg.f  # read + write, bf16
     status = M.moe_read_device_status(ws)
     rows = cfg.T * cfg.K + cfg.T
     fl = 10.0 * cfg.d * cfg.f * rows
@@ -541,9 +543,14 @@ def run_backward(cfg, dev, calls=10, warmup=3):
             "gpu_launches_per_call": 3, "device_status": status,
             "weight_gradients": {"ms": ms_dw, "achieved": achieved_dw, "unit": "TFLOP/s",
                                  "frac": achieved_dw / pk, "flops_per_call": fl_dw,
-                                 "gpu_launches_per_call": 12,
+                                 "gpu_launches_per_call": 7,
                                  "note": "dW2 and dW13 of every expert (6 d f FLOP per row), "
                                          "including the transposes into per-expert blocks"},
+            "weight_transpose": {"ms": ms_wt, "bytes": wt_bytes,
+                                 "achieved_gbs": wt_bytes / (ms_wt / 1e3) / 1e9,
+                                 "frac_of_hbm": wt_bytes / (ms_wt / 1e3) / 1e9 / P["hbm"],
+                                 "note": "moe_transpose_weights (W13^T, W2^T of every expert), "
+                                         "once per weight update, outside the timed steps"},
             "note": "expert FFN input gradients: GEMM1 recomputed, dh with the SwiGLU-backward "
                     "epilogue, dx (3 launches); weight gradients beside them"}
 

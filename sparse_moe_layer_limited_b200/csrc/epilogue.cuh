@@ -18,6 +18,12 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) 
   for (int i = 0; i < 4; ++i) d4[i] = w[i];
 }
 
+// Two fp32 -> bf16x2 bits (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // 8 bf16 (one 16-byte load) -> 8 fp32.
 __device__ __forceinline__ void bf16x8_load(const __nv_bfloat16* src, float* v) {
   const uint4 w = *reinterpret_cast<const uint4*>(src);

@@ -660,8 +660,6 @@ BwdLayout bwd_layout(const moe_shape& s) {
   off = al(off + rows * 2 * s.f * 2);
   B.colbase = off;
   off = al(off + (size_t)(s.N + 2) * 4);
-  B.col_of_row = off;
-  off = al(off + rows * 4);
   B.at = off;
   off = al(off + (size_t)s.d * R * 2);
   B.dyt = off;

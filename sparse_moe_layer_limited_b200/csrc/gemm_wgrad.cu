@@ -14,7 +14,8 @@
 // 128 x 256 output tile of one expert, its K loop the expert's column block
 // (tcgen05.mma cta_group::1, M=128, N=256, K=16, fp32 accumulate in TMEM,
 // two accumulators in turn); eight epilogue warps round the tile to bf16 and
-// store it into the gradient laid out like the weight.  An expert without rows gets zeros.
+// write it with TMA tensor stores into the gradient laid out like the weight.
+// An expert without rows gets zeros.
 // Every mbarrier wait is bounded (~2 s) and sets the device status word.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -22,6 +23,7 @@
 #include "epilogue.cuh"
 #include "internal.h"
 #include "ptx.cuh"
+#include "tile_transpose.cuh"
 
 namespace moe {
 namespace {
@@ -32,6 +34,9 @@ constexpr int WABytes = WBM * WBK * 2;
 constexpr int WBBytes = WBN * WBK * 2;
 constexpr int WStageBytes = WABytes + WBBytes;
 constexpr int WThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue (2 per quadrant)
+constexpr int WStgBytes = 32 * 128;  // per epilogue warp: 32 rows x 64 bf16, 128B-swizzled
+constexpr int WSmemBytes = 1024 + WStages * WStageBytes + 8 * WStgBytes + 256;
+static_assert(WSmemBytes <= 232448, "weight-gradient kernel exceeds the shared-memory opt-in");
 constexpr uint64_t WTimeoutNs = 2000000000ull;
 
 // ---- layout: column blocks per group --------------------------------------------
@@ -63,79 +68,66 @@ __global__ void colbase_kernel(const int32_t* __restrict__ offsets, int N, int T
   if (lane == 31) colbase[G1] = inc;
 }
 
-// col_of_row[r]: the column of dispatched row r (r < T*K) or of shared row
-// r - T*K in the transposed layouts.
-__global__ void col_of_row_kernel(const int32_t* __restrict__ offsets,
-                                  const int32_t* __restrict__ colbase, int N, int T, int TK,
-                                  int32_t* __restrict__ col_of_row) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= TK + T) return;
-  if (r >= TK) {
-    col_of_row[r] = colbase[N] + (r - TK);
-    return;
-  }
-  int lo = 0, hi = N;  // the group g with offsets[g] <= r < offsets[g+1]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (offsets[mid] <= r) lo = mid; else hi = mid;
-  }
-  col_of_row[r] = colbase[lo] + (r - offsets[lo]);
-}
-
-// Zero the padding columns of each group in a [C, R] layout.
-__global__ void zero_padding_kernel(const int32_t* __restrict__ offsets,
-                                    const int32_t* __restrict__ colbase, int N, int T, int C,
-                                    long long ld, __nv_bfloat16* __restrict__ dst) {
-  const int g = blockIdx.y;
-  const int rows = (g < N) ? offsets[g + 1] - offsets[g] : T;
-  // columns stay inside the layout even if offsets[] is inconsistent
-  const int c0 = (int)min((long long)colbase[g] + max(rows, 0), ld);
-  const int c1 = (int)min((long long)colbase[g + 1], ld);
-  const int npad = c1 - c0;
-  if (npad <= 0) return;
-  const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)C * npad;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long c = i / npad;
-    dst[c * ld + c0 + (i - c * npad)] = z;
-  }
-}
-
 // Rows [rows, C] (dispatched rows from `routed`, then the shared expert's
-// from `shared`) -> dst [C, R] at the rows' columns.  kSwiGLUH: the source
-// holds the packed gate/up products [rows, 2f] and the value moved is
-// h = silu(g) * u for feature c (C = f).
+// from `shared`) -> dst [C, R]: group g's rows go, in order, to its columns
+// colbase[g] .. colbase[g] + rows_g - 1, and its padding columns up to
+// colbase[g + 1] get zeros.  One 64 x 64 tile per CTA (tile_transpose.cuh);
+// the colbase values are multiples of 64, so a column tile lies in one group.
+// kSwiGLUH: the source holds the packed gate/up products [rows, 2f] and the
+// value moved is h = silu(g) * u of feature c (C = f), rounded to bf16.
 template <bool kSwiGLUH>
-__global__ void transpose_rows_kernel(const __nv_bfloat16* __restrict__ routed,
-                                      const __nv_bfloat16* __restrict__ shared, int TK, int T,
-                                      int C, int src_ld, const int32_t* __restrict__ col_of_row,
-                                      long long ld, __nv_bfloat16* __restrict__ dst) {
-  __shared__ float tile[32][33];
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  const int rows = TK + T;
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    float v = 0.f;
-    if (r < rows && c < C) {
+__global__ void __launch_bounds__(kTileThreads) transpose_groups_kernel(
+    const __nv_bfloat16* __restrict__ routed, const __nv_bfloat16* __restrict__ shared, int TK,
+    int T, int N, int C, int src_ld, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ colbase, long long ld, __nv_bfloat16* __restrict__ dst) {
+  __shared__ alignas(16) uint8_t sm[kTileBytes];
+  __shared__ int s_group;
+  const long long col0 = (long long)blockIdx.y * kTile;
+  const int f0 = blockIdx.x * kTile;
+  const int G1 = N + 1;
+  if (col0 >= colbase[G1]) return;  // past the last group's block
+  if (threadIdx.x == 0) {
+    int lo = 0, hi = G1;  // colbase[lo] <= col0 < colbase[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (colbase[mid] <= col0) lo = mid; else hi = mid;
+    }
+    s_group = lo;
+  }
+  __syncthreads();
+  const int g = s_group;
+  const long long first = g < N ? offsets[g] : TK;
+  const long long count = g < N ? (long long)offsets[g + 1] - offsets[g] : T;
+  const long long limit = g < N ? TK : (long long)TK + T;  // a group's rows stay below
+  const long long local0 = col0 - colbase[g];
+  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
+    const int i = it >> 3, p = it & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    const long long r = first + local0 + i;
+    if (local0 + i < count && r >= 0 && r < limit && f0 + p * 8 + 8 <= C) {
       const __nv_bfloat16* row =
           r < TK ? routed + (size_t)r * src_ld : shared + (size_t)(r - TK) * src_ld;
       if constexpr (kSwiGLUH) {
-        const int col = (c / 128) * 256 + (c % 128);
-        const float gt = __bfloat162float(row[col]), up = __bfloat162float(row[col + 128]);
-        v = silu_f(gt) * up;
+        const int col = (f0 / 128) * 256 + (f0 % 128) + p * 8;
+        float gt[8], up[8];
+        bf16x8_load(row + col, gt);
+        bf16x8_load(row + col + 128, up);
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          h[e] = __floats2bfloat162_rn(silu_f(gt[2 * e]) * up[2 * e],
+                                       silu_f(gt[2 * e + 1]) * up[2 * e + 1]);
       } else {
-        v = __bfloat162float(row[c]);
+        v = __ldg(reinterpret_cast<const uint4*>(row + f0 + p * 8));
       }
     }
-    tile[i][threadIdx.x] = v;
+    tile_put(sm, i, p, v);
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (c < C && r < rows) {
-      const int col = col_of_row[r];
-      if (col >= 0 && col < ld) dst[(size_t)c * ld + col] = __float2bfloat16_rn(tile[threadIdx.x][i]);
-    }
+  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
+    const int c = it >> 3, q = it & 7;
+    if (f0 + c < C && col0 + q * 8 + 8 <= ld)
+      *reinterpret_cast<uint4*>(dst + (size_t)(f0 + c) * ld + col0 + q * 8) = tile_get(sm, c, q);
   }
 }
 
@@ -143,8 +135,8 @@ __global__ void transpose_rows_kernel(const __nv_bfloat16* __restrict__ routed,
 struct alignas(64) WgradArgs {
   CUtensorMap tmL;  // left operand [M_total, R] (rows of the gradient), box {64, 128}
   CUtensorMap tmR;  // right operand [N_total, R] (its columns), box {64, 256}
+  CUtensorMap tmOut;  // gradient [G1 * M_total, N_total], box {64, 32}, 128B swizzle
   const int32_t* colbase;  // [G1 + 1] column block of each group
-  __nv_bfloat16* out;      // [G1, M_total, N_total]
   uint32_t* status;
   int G1, M_total, N_total;
 };
@@ -154,7 +146,8 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)WStages * WStageBytes);
+  uint8_t* staging = base + (size_t)WStages * WStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + 8 * WStgBytes);
   uint64_t* full = bars;
   uint64_t* empty = full + WStages;
   uint64_t* tfull = empty + WStages;   // [2]
@@ -270,11 +263,14 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
       mbar_wait_bounded(drain, 0, args.status, WTimeoutNs / 8);
     }
   } else {
-    // units are short (a few K blocks) and each stores a 64 KB tile, so two
-    // warps per TMEM lane quadrant drain it, 128 columns each
+    // Units are short (a few K blocks) and each stores a 64 KB tile.  Two
+    // warps per TMEM lane quadrant drain it, 128 columns each, in 64-column
+    // pieces: TMEM -> registers -> bf16 -> this warp's 128B-swizzled staging
+    // buffer -> one TMA tensor store of 32 rows x 64 columns (whole 128-byte
+    // lines, off the load/store pipeline).
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int row = q * 32 + lane;
+    uint8_t* stg = staging + (size_t)(warp - 2) * WStgBytes;
     int local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
       int g, n, m, kb0, kcnt;
@@ -282,28 +278,45 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
       const int acc = local & 1;
       if (!mbar_wait_bounded(&tfull[acc], (local >> 1) & 1, args.status, WTimeoutNs)) break;
       tc_fence_after();
-      __nv_bfloat16* orow = args.out + ((size_t)g * args.M_total + (size_t)m * WBM + row) *
-                                           args.N_total + (size_t)n * WBN;
+      const int grow = g * args.M_total + m * WBM + q * 32;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * WBN;
 #pragma unroll 1
-      for (int c = half * (WBN / 2); c < (half + 1) * (WBN / 2); c += 32) {
-        float y[32];
+      for (int c = half * (WBN / 2); c < (half + 1) * (WBN / 2); c += 64) {
+        uint32_t packed[32];
         if (kcnt > 0) {  // a group without rows has a zero gradient
-          uint32_t v[32];
-          tmem_ld32(taddr + c, v);
+          uint32_t v0[32], v1[32];
+          tmem_ld32(taddr + c, v0);
+          tmem_ld32(taddr + c + 32, v1);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
+          for (int i = 0; i < 16; ++i) {
+            packed[i] = bf16x2_bits(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+            packed[16 + i] =
+                bf16x2_bits(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+          }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = 0.f;
+          for (int i = 0; i < 32; ++i) packed[i] = 0u;
         }
-        store_row32(orow + c, y);
+        if (lane == 0) bulk_wait_read_all();  // the previous piece has left the buffer
+        __syncwarp();
+        uint8_t* my_row = stg + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(my_row + ((j ^ (lane & 7)) << 4)) =
+              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&args.tmOut, stg, n * WBN + c, grow);
+          bulk_commit_group();
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -314,7 +327,7 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
 }
 
 cudaError_t launch_wgrad(const WgradArgs& a, cudaStream_t st) {
-  const size_t smem = 1024 + (size_t)WStages * WStageBytes + 256;
+  const size_t smem = WSmemBytes;
   cudaError_t e = note_cuda(cudaFuncSetAttribute(wgrad_gemm_kernel,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem),
@@ -341,36 +354,27 @@ int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t
   const __nv_bfloat16* GU = reinterpret_cast<const __nv_bfloat16*>(w + B.gu);
   const __nv_bfloat16* dGU = reinterpret_cast<const __nv_bfloat16*>(w + B.dgu);
   int32_t* colbase = reinterpret_cast<int32_t*>(w + B.colbase);
-  int32_t* col_of_row = reinterpret_cast<int32_t*>(w + B.col_of_row);
   __nv_bfloat16* AT = reinterpret_cast<__nv_bfloat16*>(w + B.at);
   __nv_bfloat16* dYT = reinterpret_cast<__nv_bfloat16*>(w + B.dyt);
   __nv_bfloat16* HT = reinterpret_cast<__nv_bfloat16*>(w + B.ht);
   __nv_bfloat16* dGUT = reinterpret_cast<__nv_bfloat16*>(w + B.dgut);
-  const int TK = s.T * s.K, rows = TK + s.T;
+  const int TK = s.T * s.K;
   const long long R = wgrad_cols(s);
   const int twof = 2 * s.f;
   const auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
 
   colbase_kernel<<<1, 32, 0, st>>>(offsets, s.N, s.T, colbase);
-  col_of_row_kernel<<<(rows + 255) / 256, 256, 0, st>>>(offsets, colbase, s.N, s.T, TK,
-                                                         col_of_row);
-  const dim3 blk(32, 8);
-  auto zero_pad = [&](int C, __nv_bfloat16* dst) {
-    zero_padding_kernel<<<dim3(64, s.N + 1), 256, 0, st>>>(offsets, colbase, s.N, s.T, C, R, dst);
-  };
   // AT = [x_perm; x]^T, dYT = [dy_perm; dy_shared]^T, HT from GU, dGUT = dGU^T
-  transpose_rows_kernel<false><<<dim3((s.d + 31) / 32, (rows + 31) / 32), blk, 0, st>>>(
-      bf(x_perm), bf(x), TK, s.T, s.d, s.d, col_of_row, R, AT);
-  zero_pad(s.d, AT);
-  transpose_rows_kernel<false><<<dim3((s.d + 31) / 32, (rows + 31) / 32), blk, 0, st>>>(
-      bf(dy_perm), bf(dy_shared), TK, s.T, s.d, s.d, col_of_row, R, dYT);
-  zero_pad(s.d, dYT);
-  transpose_rows_kernel<true><<<dim3((s.f + 31) / 32, (rows + 31) / 32), blk, 0, st>>>(
-      GU, GU + (size_t)TK * twof, TK, s.T, s.f, twof, col_of_row, R, HT);
-  zero_pad(s.f, HT);
-  transpose_rows_kernel<false><<<dim3((twof + 31) / 32, (rows + 31) / 32), blk, 0, st>>>(
-      dGU, dGU + (size_t)TK * twof, TK, s.T, twof, twof, col_of_row, R, dGUT);
-  zero_pad(twof, dGUT);
+  const unsigned col_tiles = (unsigned)(R / kTile);
+  auto layout = [&](auto kernel, const __nv_bfloat16* routed, const __nv_bfloat16* shared, int C,
+                    int src_ld, __nv_bfloat16* dst) {
+    kernel<<<dim3(C / kTile, col_tiles), kTileThreads, 0, st>>>(routed, shared, TK, s.T, s.N, C,
+                                                                src_ld, offsets, colbase, R, dst);
+  };
+  layout(transpose_groups_kernel<false>, bf(x_perm), bf(x), s.d, s.d, AT);
+  layout(transpose_groups_kernel<false>, bf(dy_perm), bf(dy_shared), s.d, s.d, dYT);
+  layout(transpose_groups_kernel<true>, GU, GU + (size_t)TK * twof, s.f, twof, HT);
+  layout(transpose_groups_kernel<false>, dGU, dGU + (size_t)TK * twof, twof, twof, dGUT);
   if (note_cuda(cudaGetLastError(), "weight-gradient layout kernels") != cudaSuccess)
     return MOE_ERR_CUDA;
 
@@ -383,6 +387,9 @@ int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t
   WgradArgs a13{};
   ok = ok && make_map(&a13.tmL, dGUT, BF, 2, R, twof, WBK, WBM) &&
        make_map(&a13.tmR, AT, BF, 2, R, s.d, WBK, WBN);
+  const uint64_t G1 = (uint64_t)s.N + 1;
+  ok = ok && make_map(&a2.tmOut, dw2, BF, 2, s.f, G1 * s.d, 64, 32) &&
+       make_map(&a13.tmOut, dw13, BF, 2, s.d, G1 * twof, 64, 32);
   if (!ok) {
     note_text("weight-gradient GEMM: tensor-map encoding failed");
     return MOE_ERR_CUDA;
@@ -390,10 +397,8 @@ int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t
   a2.colbase = a13.colbase = colbase;
   a2.status = a13.status = status;
   a2.G1 = a13.G1 = s.N + 1;
-  a2.out = static_cast<__nv_bfloat16*>(dw2);
   a2.M_total = s.d;
   a2.N_total = s.f;
-  a13.out = static_cast<__nv_bfloat16*>(dw13);
   a13.M_total = twof;
   a13.N_total = s.d;
   if (launch_wgrad(a2, st) != cudaSuccess || launch_wgrad(a13, st) != cudaSuccess)

@@ -96,7 +96,7 @@ int launch_router_scores_tc(const moe_shape& s, const void* x, const float* rout
 // input pass's dGU [T*K+T, 2f] bf16, then the weight-gradient pass's column
 // blocks and transposed operands (gemm_wgrad.cu).
 struct BwdLayout {
-  size_t gu = 0, dgu = 0, colbase = 0, col_of_row = 0, at = 0, dyt = 0, ht = 0, dgut = 0;
+  size_t gu = 0, dgu = 0, colbase = 0, at = 0, dyt = 0, ht = 0, dgut = 0;
   size_t total = 0;
 };
 long long wgrad_cols(const moe_shape& s);

@@ -11,6 +11,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tile_transpose.cuh"
 
 namespace moe {
 namespace {
@@ -158,33 +159,38 @@ cudaError_t launch_pack_w13(const moe_shape& s, const void* w1, const void* w3, 
   return cudaGetLastError();
 }
 
-// [B, R, C] bf16 -> [B, C, R]: 32x32 tiles through shared memory (padded
-// against bank conflicts), block (32, 8).
+// [B, R, C] bf16 -> [B, C, R] in 64 x 64 tiles (tile_transpose.cuh); R and
+// C are multiples of 64 (the bf16 shape rules make d, f and 2f so).
 namespace {
-__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src,
-                                      __nv_bfloat16* __restrict__ dst, int R, int C) {
-  __shared__ __nv_bfloat16 tile[32][33];
+__global__ void __launch_bounds__(kTileThreads) transpose_tiles_kernel(
+    const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int R, int C) {
+  __shared__ alignas(16) uint8_t sm[kTileBytes];
   const size_t b = blockIdx.z;
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < R && c < C) tile[i][threadIdx.x] = src[(b * R + r) * C + c];
+  const int r0 = blockIdx.y * kTile, c0 = blockIdx.x * kTile;
+  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
+    const int i = it >> 3, p = it & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 + i < R && c0 + p * 8 + 8 <= C)
+      v = __ldg(reinterpret_cast<const uint4*>(src + (b * R + r0 + i) * C + c0 + p * 8));
+    tile_put(sm, i, p, v);
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (c < C && r < R) dst[(b * C + c) * R + r] = tile[threadIdx.x][i];
+  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
+    const int c = it >> 3, q = it & 7;
+    if (c0 + c < C && r0 + q * 8 + 8 <= R)
+      *reinterpret_cast<uint4*>(dst + (b * C + c0 + c) * R + r0 + q * 8) = tile_get(sm, c, q);
   }
 }
 }  // namespace
 
 cudaError_t launch_transpose_weights(const moe_shape& s, const void* w13, const void* w2,
                                      void* w13t, void* w2t, cudaStream_t st) {
-  const dim3 blk(32, 8);
+  if (s.d % kTile != 0 || (2 * s.f) % kTile != 0 || s.f % kTile != 0)
+    return cudaErrorInvalidValue;
   const unsigned E = (unsigned)(s.N + 1);
-  transpose_bf16_kernel<<<dim3((s.d + 31) / 32, (2 * s.f + 31) / 32, E), blk, 0, st>>>(
+  transpose_tiles_kernel<<<dim3(s.d / kTile, 2 * s.f / kTile, E), kTileThreads, 0, st>>>(
       static_cast<const __nv_bfloat16*>(w13), static_cast<__nv_bfloat16*>(w13t), 2 * s.f, s.d);
-  transpose_bf16_kernel<<<dim3((s.f + 31) / 32, (s.d + 31) / 32, E), blk, 0, st>>>(
+  transpose_tiles_kernel<<<dim3(s.f / kTile, s.d / kTile, E), kTileThreads, 0, st>>>(
       static_cast<const __nv_bfloat16*>(w2), static_cast<__nv_bfloat16*>(w2t), s.d, s.f);
   return cudaGetLastError();
 }
