@@ -544,6 +544,8 @@ def run_backward(cfg, dev, calls=10, warmup=3):
             "weight_gradients": {"ms": ms_dw, "achieved": achieved_dw, "unit": "TFLOP/s",
                                  "frac": achieved_dw / pk, "flops_per_call": fl_dw,
                                  "gpu_launches_per_call": 7,
+                                 "kernel": ("one CTA" if os.environ.get("MOE_WGRAD") == "single"
+                                            else "CTA pair"),
                                  "note": "dW2 and dW13 of every expert (6 d f FLOP per row), "
                                          "including the transposes into per-expert blocks"},
             "weight_transpose": {"ms": ms_wt, "bytes": wt_bytes,

@@ -91,30 +91,8 @@ __device__ __forceinline__ void unit_split(int rows, int& size, int& count) {
 }
 
 // Cluster-scope acquire: the arrivals come from both CTAs of the pair.
-__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  if (mbar_try_wait_cl(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cl(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*reinterpret_cast<volatile uint32_t*>(err) != 0u) return false;
-      if (globaltimer_ns() - t0 > PTimeoutNs) {
-        atomicOr(err, kErrWaitTimeout);
-        return false;
-      }
-    }
-  }
+  return mbar_wait_cluster_bounded(bar, parity, err, PTimeoutNs);
 }
 
 // One unit as every role sees it.

@@ -20,6 +20,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
+
 #include "epilogue.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -180,13 +183,14 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_gemm_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  // unit -> group g, right tile n, left tile m (m fastest: neighbours share the
-  // 256-row right tile); K blocks of the group's column block
+  // unit -> group g, left tile m, right tile n (n fastest: units running at the
+  // same time write whole rows of the gradient, and an expert's operands stay
+  // in L2 while its units run); K blocks of the group's column block
   auto decode = [&](int u, int& g, int& n, int& m, int& kb0, int& kcnt) {
     g = u / per_group;
     const int local = u - g * per_group;
-    n = local / MT;
-    m = local - n * MT;
+    m = local / NT;
+    n = local - m * NT;
     kb0 = args.colbase[g] / WBK;
     kcnt = (args.colbase[g + 1] - args.colbase[g]) / WBK;
   };
@@ -337,6 +341,256 @@ cudaError_t launch_wgrad(const WgradArgs& a, cudaStream_t st) {
   return note_cuda(cudaGetLastError(), "weight-gradient GEMM launch");
 }
 
+// ---- the same products on CTA pairs -----------------------------------------------
+// A unit is one 256 x 256 output tile of one expert, one tcgen05.mma
+// cta_group::2 (M=256, N=256, K=16) per K step: CTA r of the pair stages rows
+// 128r..128r+127 of the tile's left operand and rows 128r..128r+127 of its
+// right operand, so per K block a CTA stages 32 KB instead of 48 KB for the
+// same 128 x 256 outputs, and each CTA's TMEM holds its 128 rows of the tile.
+// The gradient rows are multiples of 256 (d and 2f are), so no unit is ragged.
+// Barriers: full (leader; both CTAs' copies land on it), empty and tfull (each
+// CTA; the leader's commits are multicast), tempty (leader; the 16 epilogue
+// warps of the pair).  Both CTAs reach the final cluster barrier, so neither
+// exits while its peer may still signal it.
+constexpr int QStages = 5;
+constexpr int QHalfBytes = WBM * WBK * 2;     // 16 KB: 128 rows x 64 K
+constexpr int QStageBytes = 2 * QHalfBytes;   // left rows + right rows
+// two staging buffers per epilogue warp: a piece is staged while the store of
+// the previous one may still be reading its buffer
+constexpr int QSmemBytes = 1024 + QStages * QStageBytes + 16 * WStgBytes + 256;
+static_assert(QSmemBytes <= 232448, "pair weight-gradient kernel exceeds the shared-memory opt-in");
+
+__global__ void __launch_bounds__(WThreads, 1) wgrad_pair_kernel(
+    const __grid_constant__ WgradArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* staging = base + (size_t)QStages * QStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + 16 * WStgBytes);
+  uint64_t* full = bars;               // [QStages] leader
+  uint64_t* empty = full + QStages;    // [QStages] each CTA
+  uint64_t* tfull = empty + QStages;   // [2] each CTA
+  uint64_t* tempty = tfull + 2;        // [2] leader
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int MT = args.M_total / (2 * WBM), NT = args.N_total / WBN;
+  const int per_group = MT * NT;
+  const int total = args.G1 * per_group;
+
+  if (tid == 0) {
+    for (int st = 0; st < QStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 16);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_2sm(tmem_holder, 2 * WBN);
+    tmem_relinquish_2sm();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either signals the other
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  auto decode = [&](int u, int& g, int& n, int& m, int& kb0, int& kcnt) {
+    g = u / per_group;
+    const int local = u - g * per_group;
+    m = local / NT;
+    n = local - m * NT;
+    kb0 = args.colbase[g] / WBK;
+    kcnt = (args.colbase[g + 1] - args.colbase[g]) / WBK;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&args.tmL);
+      tma_prefetch_desc(&args.tmR);
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int u = pair; u < total && ok; u += npairs) {
+        int g, n, m, kb0, kcnt;
+        decode(u, g, n, m, kb0, kcnt);
+        for (int kb = 0; kb < kcnt; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, WTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = base + (size_t)stage * QStageBytes;
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * QStageBytes);
+          tma_load_2d_2sm(sa, &args.tmL, (kb0 + kb) * WBK, m * 2 * WBM + (int)rank * WBM, fbar);
+          tma_load_2d_2sm(sa + QHalfBytes, &args.tmR, (kb0 + kb) * WBK,
+                          n * WBN + (int)rank * WBM, fbar);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == QStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {  // the copies already issued complete on these barriers
+        for (int st = 0; st < QStages; ++st)
+          if ((issued >> st) & 1u)
+            mbar_wait_bounded(&full[st], (issued_parity >> st) & 1u, args.status,
+                              WTimeoutNs / 8);
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * WBM, WBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int u = pair; u < total && ok; u += npairs, ++local) {
+        int g, n, m, kb0, kcnt;
+        decode(u, g, n, m, kb0, kcnt);
+        const int acc = local & 1;
+        if (!mbar_wait_cluster_bounded(&tempty[acc], ((local >> 1) & 1) ^ 1u, args.status,
+                                       WTimeoutNs))
+          break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * WBN;
+        for (int kb = 0; kb < kcnt; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, args.status, WTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(base + (size_t)stage * QStageBytes);
+          const uint32_t b0 = a0 + QHalfBytes;
+#pragma unroll
+          for (int k = 0; k < WBK / 16; ++k)
+            mma_bf16_2sm(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32),
+                         idesc, (kb | k) != 0);
+          mma_commit_2sm_mc(&empty[stage], 0x3);
+          if (++stage == QStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit_2sm_mc(&tfull[acc], 0x3);  // with no K blocks: arrives at once
+      }
+      mma_commit_2sm(drain);
+      mbar_wait_bounded(drain, 0, args.status, WTimeoutNs / 8);
+    }
+  } else {
+    // each CTA drains its 128 rows of the tile exactly as the one-CTA kernel
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    uint8_t* stg0 = staging + (size_t)(warp - 2) * 2 * WStgBytes;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    int local = 0;
+    for (int u = pair; u < total; u += npairs, ++local) {
+      int g, n, m, kb0, kcnt;
+      decode(u, g, n, m, kb0, kcnt);
+      const int acc = local & 1;
+      if (!mbar_wait_bounded(&tfull[acc], (local >> 1) & 1, args.status, WTimeoutNs)) break;
+      tc_fence_after();
+      const int grow = g * args.M_total + m * 2 * WBM + (int)rank * WBM + q * 32;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * WBN;
+#pragma unroll 1
+      for (int c = half * (WBN / 2); c < (half + 1) * (WBN / 2); c += 64) {
+        uint32_t packed[32];
+        if (kcnt > 0) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(taddr + c, v0);
+          tmem_ld32(taddr + c + 32, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            packed[i] = bf16x2_bits(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+            packed[16 + i] =
+                bf16x2_bits(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) packed[i] = 0u;
+        }
+        uint8_t* stg = stg0 + (c & 64 ? WStgBytes : 0);  // pieces alternate buffers
+        if (lane == 0) bulk_wait_read_but_one();  // this buffer's last store has read it
+        __syncwarp();
+        uint8_t* my_row = stg + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(my_row + ((j ^ (lane & 7)) << 4)) =
+              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&args.tmOut, stg, n * WBN + c, grow);
+          bulk_commit_group();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_2sm(tmem_base, 2 * WBN);
+  }
+}
+
+cudaError_t launch_wgrad_pair(const WgradArgs& a, cudaStream_t st) {
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(wgrad_pair_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 QSmemBytes),
+                            "pair weight-gradient GEMM: set shared-memory size");
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(WThreads, 1, 1);
+  cfg.dynamicSmemBytes = QSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)(num_sms() & ~1), 1, 1);
+  // as many pairs as can be resident at once, so no pair waits for a second wave
+  static int max_pairs = 0;
+  if (max_pairs == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, wgrad_pair_kernel, &cfg) != cudaSuccess || n <= 0)
+      n = num_sms() / 2;
+    max_pairs = n;
+  }
+  cfg.gridDim = dim3((unsigned)(2 * max_pairs), 1, 1);
+  return note_cuda(cudaLaunchKernelEx(&cfg, wgrad_pair_kernel, a),
+                   "pair weight-gradient GEMM launch");
+}
+
+// MOE_WGRAD=single selects the one-CTA kernel (read once per process).
+bool use_pair_wgrad() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("MOE_WGRAD");
+    v = (e != nullptr && std::strcmp(e, "single") == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+
 }  // namespace
 
 // Columns of the transposed layouts: all rows plus up to 63 of padding per group.
@@ -379,14 +633,16 @@ int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t
     return MOE_ERR_CUDA;
 
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const bool pair = use_pair_wgrad();
+  const uint32_t rbox = pair ? WBM : WBN;  // right-operand rows per CTA
   // dW2_e [d, f] = dYT_e HT_e^T
   WgradArgs a2{};
   bool ok = make_map(&a2.tmL, dYT, BF, 2, R, s.d, WBK, WBM) &&
-            make_map(&a2.tmR, HT, BF, 2, R, s.f, WBK, WBN);
+            make_map(&a2.tmR, HT, BF, 2, R, s.f, WBK, rbox);
   // dW13_e [2f, d] = dGUT_e AT_e^T (rows in the packed W13 order)
   WgradArgs a13{};
   ok = ok && make_map(&a13.tmL, dGUT, BF, 2, R, twof, WBK, WBM) &&
-       make_map(&a13.tmR, AT, BF, 2, R, s.d, WBK, WBN);
+       make_map(&a13.tmR, AT, BF, 2, R, s.d, WBK, rbox);
   const uint64_t G1 = (uint64_t)s.N + 1;
   ok = ok && make_map(&a2.tmOut, dw2, BF, 2, s.f, G1 * s.d, 64, 32) &&
        make_map(&a13.tmOut, dw13, BF, 2, s.d, G1 * twof, 64, 32);
@@ -401,8 +657,8 @@ int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t
   a2.N_total = s.f;
   a13.M_total = twof;
   a13.N_total = s.d;
-  if (launch_wgrad(a2, st) != cudaSuccess || launch_wgrad(a13, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  const auto run = pair ? launch_wgrad_pair : launch_wgrad;
+  if (run(a2, st) != cudaSuccess || run(a13, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

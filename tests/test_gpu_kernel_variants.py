@@ -1,10 +1,12 @@
-"""The opt-in bf16 expert GEMM kernels against the oracle.
+"""The opt-in bf16 GEMM kernels against the oracle.
 
 The library picks its expert GEMM kernel once per process from MOE_BF16_GEMM
 ("dual": two token tiles per weight tile, "pair": CTA pairs); the default
 one-tile kernel is covered by the other GPU tests.  Each variant reruns the
 bf16 layer parity tests (routing and dispatch bit-exact, expert outputs and
 the layer within the bf16 tolerance) in a child process with the variable set.
+Likewise MOE_WGRAD=single selects the one-CTA weight-gradient kernel instead
+of the default CTA-pair one; the weight-gradient parity tests rerun with it.
 """
 import os
 import subprocess
@@ -24,6 +26,16 @@ def test_bf16_expert_gemm_variant(kind):
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
            os.path.join(HERE, "test_gpu_parity.py"),
            "-k", "small_bf16 or mid_bf16 or all_experts or idle"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    tail = (r.stdout + r.stderr)[-3000:]
+    assert r.returncode == 0, tail
+    assert " passed" in r.stdout and "failed" not in r.stdout, tail
+
+
+def test_one_cta_weight_gradient_kernel():
+    env = dict(os.environ, MOE_WGRAD="single")
+    cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+           os.path.join(HERE, "test_gpu_backward.py"), "-k", "dw"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
     tail = (r.stdout + r.stderr)[-3000:]
     assert r.returncode == 0, tail
