@@ -38,7 +38,7 @@ from .moe import (  # noqa: F401
     affinity, biased_scores, group_scores, kept_groups, route, route_margins,
     route_softmax, route_softmax_margins, balance_loss,
     dispatch, swiglu_expert, swiglu_expert_backward, expert_outputs, combine, bias_update,
-    moe_forward,
+    moe_forward, combine_backward, route_backward, dispatch_backward, moe_backward,
     round_bf16, silu,
 )
 from .fp8 import (  # noqa: F401

@@ -323,6 +323,83 @@ def bias_update(bias, counts, T: int, K: int, gamma: float) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# backward of COMBINE, of the gates and of DISPATCH
+# ---------------------------------------------------------------------------
+
+def combine_backward(dy, y_perm, slot, gate) -> dict:
+    """Backward of y_t = y_shared_t + sum_k gate[t,k] * y_perm[slot[t,k]].
+
+    [P1] §2.2 runs the backward pass COMBINE -> MLP_B -> MLP_W -> DISPATCH;
+    this is its first step.  For each (t, k):
+        dy_perm[slot[t,k]] = gate[t,k] * dy_t      (the routed expert's output gradient)
+        dgate[t,k]         = dy_t . y_perm[slot[t,k]]
+    and the shared expert's output gradient is dy itself.  float64.
+    Returns dict(dy_perm [T*K, d], dgate [T, K])."""
+    dy = np.asarray(dy, dtype=np.float64)
+    y_perm = np.asarray(y_perm, dtype=np.float64)
+    slot = np.asarray(slot)
+    gate = np.asarray(gate, dtype=np.float64)
+    T, K = slot.shape
+    dy_perm = np.zeros((T * K, dy.shape[1]), dtype=np.float64)
+    dgate = np.empty((T, K), dtype=np.float64)
+    for t in range(T):
+        for k in range(K):
+            r = slot[t, k]
+            dy_perm[r] = gate[t, k] * dy[t]
+            dgate[t, k] = float(np.dot(dy[t], y_perm[r]))
+    return dict(dy_perm=dy_perm, dgate=dgate)
+
+
+def route_backward(x, router, idx, dgate) -> dict:
+    """Gradient of the gates with respect to the router logits, the layer
+    input and the router weights, the selection held fixed (the bias enters
+    only the selection, [P2] Q3, so it receives no gradient).
+
+    With z = x e_i (the logits), s = sigmoid(z) ([P4]: sigmoid affinity) and,
+    over the K selected experts, gate_k = s_k / S with S = sum_j s_j ([P4]:
+    normalisation over the selected affinities):
+        ds_k = (dgate_k - sum_j gate_j dgate_j) / S
+        dz_k = ds_k * s_k (1 - s_k)
+        dx_t += sum_k dz_k e_{idx_k},    de_i += sum over (t, k) with idx = i of dz_k x_t
+    Returns dict(dz [T, K], dx [T, d], drouter [N, d], s [T, K], gate [T, K])."""
+    x = np.asarray(x, dtype=np.float64)
+    R = np.asarray(router, dtype=np.float64)
+    idx = np.asarray(idx)
+    dgate = np.asarray(dgate, dtype=np.float64)
+    T, K = idx.shape
+    z = np.einsum("td,tkd->tk", x, R[idx])
+    s = 1.0 / (1.0 + np.exp(-z))
+    S = s.sum(axis=1, keepdims=True)
+    gate = s / S
+    ds = (dgate - (gate * dgate).sum(axis=1, keepdims=True)) / S
+    dz = ds * s * (1.0 - s)
+    dx = np.einsum("tk,tkd->td", dz, R[idx])
+    drouter = np.zeros_like(R)
+    for t in range(T):
+        for k in range(K):
+            drouter[idx[t, k]] += dz[t, k] * x[t]
+    return dict(dz=dz, dx=dx, drouter=drouter, s=s, gate=gate)
+
+
+def dispatch_backward(dx_perm, dx_shared, slot, dx_route=None) -> np.ndarray:
+    """Last step of the backward order ([P1] §2.2): every copy of token t
+    that DISPATCH made sends its input gradient back,
+        dx_t = dx_shared_t + sum_k dx_perm[slot[t,k]] (+ dx_route_t),
+    where dx_shared is the shared expert's input gradient and dx_route the
+    gradient through the router logits.  float64, [T, d]."""
+    dx = np.array(dx_shared, dtype=np.float64, copy=True)
+    dx_perm = np.asarray(dx_perm, dtype=np.float64)
+    slot = np.asarray(slot)
+    T, K = slot.shape
+    for t in range(T):
+        for k in range(K):
+            dx[t] += dx_perm[slot[t, k]]
+    if dx_route is not None:
+        dx += np.asarray(dx_route, dtype=np.float64)
+    return dx
+
+
+# ---------------------------------------------------------------------------
 # the whole layer
 # ---------------------------------------------------------------------------
 
@@ -338,3 +415,45 @@ def moe_forward(x, router, bias, get_weights, G: int, topG: int, K: int,
     y = combine(ex["shared"], ex["routed"], r["idx"], r["gate"], ex["tokens"])
     return dict(route=r, dispatch=d, y=y, tokens=ex["tokens"], shared=ex["shared"],
                 routed=ex["routed"])
+
+
+def moe_backward(x, router, bias, get_weights, G: int, topG: int, K: int, dy,
+                 h_round: str = "none") -> dict:
+    """The layer backward for every token, in the order of [P1] §2.2:
+    COMBINE backward, MLP_B and MLP_W of every expert (routed and shared),
+    then DISPATCH backward with the router path added.  The routing is the
+    forward's and held fixed.  float64.
+    Returns dict(dx [T, d], drouter [N, d], dw {e: (dW1, dW3, dW2)}, dgate,
+    dz, route, dispatch)."""
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    N = np.asarray(router).shape[0]
+    T, d = x.shape
+    r = route(x, router, bias, G, topG, K)
+    dsp = dispatch(r["idx"], N)
+    offs, perm_tok, slot = dsp["offsets"], dsp["perm_tok"], dsp["slot"]
+    y_perm = np.zeros((T * K, d), dtype=np.float64)
+    for e in range(N):
+        rows = np.arange(offs[e], offs[e + 1])
+        if rows.size:
+            w1, w3, w2 = get_weights(e)
+            y_perm[rows] = swiglu_expert(x[perm_tok[rows]], w1, w3, w2, h_round)
+    cb = combine_backward(dy, y_perm, slot, r["gate"])
+    dx_perm = np.zeros((T * K, d), dtype=np.float64)
+    dw = {}
+    for e in range(N):
+        rows = np.arange(offs[e], offs[e + 1])
+        w1, w3, w2 = get_weights(e)
+        if rows.size:
+            b = swiglu_expert_backward(x[perm_tok[rows]], w1, w3, w2, cb["dy_perm"][rows])
+            dx_perm[rows] = b["da"]
+            dw[e] = (b["dw1"], b["dw3"], b["dw2"])
+        else:
+            dw[e] = tuple(np.zeros_like(np.asarray(w, np.float64)) for w in (w1, w3, w2))
+    w1, w3, w2 = get_weights(N)
+    bs = swiglu_expert_backward(x, w1, w3, w2, dy)
+    dw[N] = (bs["dw1"], bs["dw3"], bs["dw2"])
+    rb = route_backward(x, router, r["idx"], cb["dgate"])
+    dx = dispatch_backward(dx_perm, bs["da"], slot, rb["dx"])
+    return dict(dx=dx, drouter=rb["drouter"], dw=dw, dgate=cb["dgate"], dz=rb["dz"],
+                route=r, dispatch=dsp)
