@@ -197,8 +197,9 @@ int moe_expert_ffn(const moe_shape* shape, const void* x_perm, const float* x_pe
 
 /* moe_expert_ffn_gathered (BF16 mode only): moe_expert_ffn without the
  * permuted copy of x.  GEMM1 reads each routed row straight from x, row
- * perm_tok[r] for row r of the expert-major order (four rows per TMA
- * tile::gather4 copy), so moe_dispatch may be called with x_perm = NULL.
+ * perm_tok[r] for row r of the expert-major order (the producer warp's
+ * 16-byte cp.async copies, written in the 128-byte-swizzled operand layout),
+ * so moe_dispatch may be called with x_perm = NULL.
  *   x          [T, d] bf16 layer input
  *   perm_tok   [T*K] int32, offsets [N+1] int32   from moe_dispatch
  *   w13, w2, y_perm, y_shared, ws   as at moe_expert_ffn
@@ -252,6 +253,49 @@ int moe_expert_ffn_backward_dw(const moe_shape* shape, const void* x_perm,
  * output dtype (fp32 in FP32 mode, else bf16).  No atomics: deterministic. */
 int moe_combine(const moe_shape* shape, const void* y_perm, const void* y_shared,
                 const int32_t* slot, const float* topk_gate, void* y, void* stream);
+
+/* ---- backward of COMBINE, of the gates and of DISPATCH --------------------
+ * [P1] §2.2 orders the backward pass COMBINE -> MLP_B -> MLP_W -> DISPATCH.
+ * These three calls are the steps around the expert backward
+ * (moe_expert_ffn_backward_dx/_dw).  The routing of the forward is held
+ * fixed; the bias receives no gradient ([P2] Q3: it only selects).
+ * Activations are fp32 in FP32 mode and bf16 otherwise (E4M3 mode keeps its
+ * layer input and outputs in bf16); gradients of the gates and of the router
+ * are fp32.  Every sum runs in fp32 in a fixed order: deterministic, no
+ * atomics.  All pointers are device pointers owned by the caller, 16-byte
+ * aligned; a NULL or misaligned pointer gives MOE_ERR_ARG.
+ *
+ * moe_combine_backward: for y[t] = y_shared[t] + sum_k gate[t,k] y_perm[slot[t,k]]
+ * and dy = dL/dy [T, d]:
+ *   dy_perm[slot[t,k]] = gate[t,k] * dy[t]          [T*K, d], one rounding
+ *   dgate[t,k]         = dy[t] . y_perm[slot[t,k]]   [T, K] fp32
+ * The shared expert's output gradient is dy itself.  Rows that no slot names
+ * are not written; a slot outside [0, T*K) gives dgate 0. */
+int moe_combine_backward(const moe_shape* shape, const void* dy, const void* y_perm,
+                         const int32_t* slot, const float* topk_gate, void* dy_perm,
+                         float* dgate, void* stream);
+
+/* moe_route_backward: the gates gate_k = s_k / S (S = sum over the K selected
+ * experts, s = sigmoid(x . e_i), [P4]) given dgate [T, K]:
+ *   dlogit[t,k] = s_k (1 - s_k) (dgate_k - sum_j gate_j dgate_j) / S   [T, K] fp32
+ *   dx_route[t] = sum_k dlogit[t,k] e_{idx[t,k]}                      [T, d] fp32
+ *   drouter[i]  = sum over expert i's dispatched rows r (in row order)
+ *                 of dlogit * x[perm_tok[r]]                          [N, d] fp32
+ * The logits are recomputed in fp32 from x and router_w [N, d] fp32.
+ *   topk_idx [T, K] int32 from moe_route; offsets, perm_tok, slot from
+ *   moe_dispatch.  An expert with no rows gets a zero row of drouter. */
+int moe_route_backward(const moe_shape* shape, const void* x, const float* router_w,
+                       const int32_t* topk_idx, const float* dgate, const int32_t* offsets,
+                       const int32_t* perm_tok, const int32_t* slot, float* dlogit,
+                       float* dx_route, float* drouter, void* stream);
+
+/* moe_dispatch_backward: each copy that DISPATCH made returns its gradient,
+ *   dx[t] = dx_shared[t] + sum_k dx_perm[slot[t,k]] (+ dx_route[t])
+ * accumulated in fp32 in that order and rounded once to the activation type.
+ *   dx_perm [T*K, d], dx_shared [T, d]   from moe_expert_ffn_backward_dx
+ *   dx_route [T, d] fp32 from moe_route_backward, or NULL to leave it out */
+int moe_dispatch_backward(const moe_shape* shape, const void* dx_perm, const void* dx_shared,
+                          const int32_t* slot, const float* dx_route, void* dx, void* stream);
 
 /* Auxiliary-loss-free bias update ([P4]; [P1] §1.2): for every expert,
  * bias[i] -= gamma if counts[i] * N > T * K, += gamma if counts[i] * N < T * K,

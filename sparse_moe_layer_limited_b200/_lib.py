@@ -51,6 +51,9 @@ _SIGS = {
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
     "moe_expert_ffn_gathered": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
+    "moe_combine_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
+    "moe_route_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 11),
+    "moe_dispatch_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
     "moe_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
     "moe_transpose_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 5),
     "moe_expert_ffn_backward_dx": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
@@ -247,6 +250,29 @@ def moe_combine(s, y_perm, y_shared, slot, topk_gate, y, stream=None):
     _expect(y, x_torch_dtype(s), s.T * s.d, "y")
     _call("moe_combine", ctypes.byref(s), _ptr(y_perm), _ptr(y_shared), _ptr(slot),
           _ptr(topk_gate), _ptr(y), _stream(stream))
+
+
+def moe_combine_backward(s, dy, y_perm, slot, topk_gate, dy_perm, dgate, stream=None):
+    _expect(dy_perm, x_torch_dtype(s), s.T * s.K * s.d, "dy_perm")
+    _expect(dgate, torch.float32, s.T * s.K, "dgate")
+    _call("moe_combine_backward", ctypes.byref(s), _ptr(dy), _ptr(y_perm), _ptr(slot),
+          _ptr(topk_gate), _ptr(dy_perm), _ptr(dgate), _stream(stream))
+
+
+def moe_route_backward(s, x, router_w, topk_idx, dgate, offsets, perm_tok, slot, dlogit,
+                       dx_route, drouter, stream=None):
+    _expect(dlogit, torch.float32, s.T * s.K, "dlogit")
+    _expect(dx_route, torch.float32, s.T * s.d, "dx_route")
+    _expect(drouter, torch.float32, s.N * s.d, "drouter")
+    _call("moe_route_backward", ctypes.byref(s), _ptr(x), _ptr(router_w), _ptr(topk_idx),
+          _ptr(dgate), _ptr(offsets), _ptr(perm_tok), _ptr(slot), _ptr(dlogit), _ptr(dx_route),
+          _ptr(drouter), _stream(stream))
+
+
+def moe_dispatch_backward(s, dx_perm, dx_shared, slot, dx_route, dx, stream=None):
+    _expect(dx, x_torch_dtype(s), s.T * s.d, "dx")
+    _call("moe_dispatch_backward", ctypes.byref(s), _ptr(dx_perm), _ptr(dx_shared), _ptr(slot),
+          _ptr(dx_route), _ptr(dx), _stream(stream))
 
 
 def moe_bias_update(s, counts, bias, gamma, stream=None):

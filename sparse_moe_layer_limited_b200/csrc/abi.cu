@@ -269,6 +269,44 @@ int moe_combine(const moe_shape* shape, const void* y_perm, const void* y_shared
                                     static_cast<cudaStream_t>(stream)));
 }
 
+int moe_combine_backward(const moe_shape* shape, const void* dy, const void* y_perm,
+                         const int32_t* slot, const float* topk_gate, void* dy_perm,
+                         float* dgate, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (!ptr_ok(dy) || !ptr_ok(y_perm) || !ptr_ok(slot) || !ptr_ok(topk_gate) ||
+      !ptr_ok(dy_perm) || !ptr_ok(dgate))
+    return MOE_ERR_ARG;
+  return cuda_status(launch_combine_backward(*shape, dy, y_perm, slot, topk_gate, dy_perm, dgate,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route_backward(const moe_shape* shape, const void* x, const float* router_w,
+                       const int32_t* topk_idx, const float* dgate, const int32_t* offsets,
+                       const int32_t* perm_tok, const int32_t* slot, float* dlogit,
+                       float* dx_route, float* drouter, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (!ptr_ok(x) || !ptr_ok(router_w) || !ptr_ok(topk_idx) || !ptr_ok(dgate) ||
+      !ptr_ok(offsets) || !ptr_ok(perm_tok) || !ptr_ok(slot) || !ptr_ok(dlogit) ||
+      !ptr_ok(dx_route) || !ptr_ok(drouter))
+    return MOE_ERR_ARG;
+  return cuda_status(launch_route_backward(*shape, x, router_w, topk_idx, dgate, offsets,
+                                           perm_tok, slot, dlogit, dx_route, drouter,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int moe_dispatch_backward(const moe_shape* shape, const void* dx_perm, const void* dx_shared,
+                          const int32_t* slot, const float* dx_route, void* dx, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (!ptr_ok(dx_perm) || !ptr_ok(dx_shared) || !ptr_ok(slot) || !ptr_ok(dx) ||
+      (dx_route != nullptr && !ptr_ok(dx_route)))
+    return MOE_ERR_ARG;
+  return cuda_status(launch_dispatch_backward(*shape, dx_perm, dx_shared, slot, dx_route, dx,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 int moe_bias_update(const moe_shape* shape, const int32_t* counts, float* bias, float gamma,
                     void* stream) {
   int rc = check(shape);

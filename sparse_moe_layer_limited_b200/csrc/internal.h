@@ -109,6 +109,16 @@ int launch_ffn_bwd_dx_bf16(const moe_shape& s, const void* x_perm, const int32_t
                            const void* x, const void* w13, const void* w13t, const void* w2t,
                            const void* dy_perm, const void* dy_shared, void* dx_perm,
                            void* dx_shared, void* ws_bwd, cudaStream_t st);
+cudaError_t launch_combine_backward(const moe_shape& s, const void* dy, const void* y_perm,
+                                    const int32_t* slot, const float* gate, void* dy_perm,
+                                    float* dgate, cudaStream_t st);
+cudaError_t launch_route_backward(const moe_shape& s, const void* x, const float* router_w,
+                                  const int32_t* idx, const float* dgate, const int32_t* offsets,
+                                  const int32_t* perm_tok, const int32_t* slot, float* dlogit,
+                                  float* dx_route, float* drouter, cudaStream_t st);
+cudaError_t launch_dispatch_backward(const moe_shape& s, const void* dx_perm,
+                                     const void* dx_shared, const int32_t* slot,
+                                     const float* dx_route, void* dx, cudaStream_t st);
 cudaError_t launch_transpose_weights(const moe_shape& s, const void* w13, const void* w2,
                                      void* w13t, void* w2t, cudaStream_t st);
 // bf16 expert GEMMs; with perm_tok set, GEMM1 gathers the routed rows from x

@@ -1,5 +1,6 @@
 """MoELayer: owns the device buffers of one layer shape and runs the forward
-through the C-ABI calls (route -> dispatch -> experts -> combine -> bias update)."""
+through the C-ABI calls (route -> dispatch -> experts -> combine -> bias update)
+and, in BF16 mode, the layer backward."""
 from __future__ import annotations
 
 import torch
@@ -78,6 +79,55 @@ class MoELayer:
             L.moe_expert_ffn(s, self.x_perm, self.x_perm_scales, self.offsets, x, self.w13,
                              self.w2, self.w13_scales, self.w2_scales, self.y_perm,
                              self.y_shared, self.ws, stream)
+
+    def backward(self, x, dy, w13t, w2t, weight_grads: bool = True, stream=None):
+        """Gradients of the last forward (its routing held fixed) given
+        dy = dL/dy [T, d], BF16 mode without gather, in the backward order
+        COMBINE -> MLP_B -> MLP_W -> DISPATCH:
+          moe_combine_backward -> moe_expert_ffn_backward_dx (-> _dw)
+          -> moe_route_backward -> moe_dispatch_backward.
+        w13t, w2t: the transposed weights (moe_transpose_weights).  Returns
+        dict(dx [T, d] bf16, drouter [N, d] fp32, dgate [T, K] fp32, and with
+        weight_grads dw13, dw2 laid out like w13, w2).  The bias gets no
+        gradient (it only selects experts)."""
+        s = self.shape
+        if s.dtype != L.DTYPE_BF16 or self.gather:
+            raise ValueError("the layer backward runs in BF16 mode on the x_perm path")
+        dev, xdt = x.device, L.x_torch_dtype(s)
+        if getattr(self, "_bwd", None) is None:
+            self._bwd = dict(
+                ws=torch.zeros(L.backward_workspace_size(s), dtype=torch.uint8, device=dev),
+                dy_perm=torch.empty(s.T * s.K, s.d, dtype=xdt, device=dev),
+                dgate=torch.empty(s.T, s.K, dtype=torch.float32, device=dev),
+                dx_perm=torch.empty(s.T * s.K, s.d, dtype=xdt, device=dev),
+                dx_shared=torch.empty(s.T, s.d, dtype=xdt, device=dev),
+                dlogit=torch.empty(s.T, s.K, dtype=torch.float32, device=dev),
+                dx_route=torch.empty(s.T, s.d, dtype=torch.float32, device=dev))
+        B = self._bwd
+        dx = torch.empty(s.T, s.d, dtype=xdt, device=dev)
+        drouter = torch.empty(s.N, s.d, dtype=torch.float32, device=dev)
+        L.moe_combine_backward(s, dy, self.y_perm, self.slot, self.topk_gate, B["dy_perm"],
+                               B["dgate"], stream)
+        L.moe_expert_ffn_backward_dx(s, self.x_perm, self.offsets, x, self.w13, w13t, w2t,
+                                     B["dy_perm"], dy, B["dx_perm"], B["dx_shared"], B["ws"],
+                                     stream)
+        out = dict(dx=dx, drouter=drouter, dgate=B["dgate"])
+        if weight_grads:
+            out["dw13"] = torch.empty_like(self.w13)
+            out["dw2"] = torch.empty_like(self.w2)
+            L.moe_expert_ffn_backward_dw(s, self.x_perm, self.offsets, x, B["dy_perm"], dy,
+                                         out["dw13"], out["dw2"], B["ws"], stream)
+        L.moe_route_backward(s, x, self.router_w, self.topk_idx, B["dgate"], self.offsets,
+                             self.perm_tok, self.slot, B["dlogit"], B["dx_route"], drouter,
+                             stream)
+        L.moe_dispatch_backward(s, B["dx_perm"], B["dx_shared"], self.slot, B["dx_route"], dx,
+                                stream)
+        return out
+
+    def backward_status(self, clear: bool = False) -> int:
+        """Status word of the backward workspace (0 = no device-side problem)."""
+        B = getattr(self, "_bwd", None)
+        return 0 if B is None else L.moe_read_device_status(B["ws"], None, clear)
 
     def device_status(self, clear: bool = False) -> int:
         return L.moe_read_device_status(self.ws, None, clear)
