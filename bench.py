@@ -42,7 +42,8 @@ def parse():
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--cpu-sample", type=int, default=2, help="tokens per oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak", "mma", "backward"],
+    p.add_argument("--probe", choices=["uniform", "cublas", "fp8peak", "mma", "backward",
+                                       "layer_backward"],
                    default=None,
                    help="measurement probes behind the profiles: expert GEMMs on uniform "
                         "expert loads, cuBLAS batched GEMM at the expert shapes, FP8 GEMM peak")
@@ -266,7 +267,14 @@ def run_probe(args, cfg):
              ideal grouped problem, routed part only), and a dense GEMM;
     fp8peak: torch._scaled_mm E4M3 8192^3, best of 10;
     mma:     the tcgen05.mma issue-rate probe (SM cycles per instruction shape);
-    backward: the expert backward (input and weight gradients) alone."""
+    backward: the expert backward (input and weight gradients) alone;
+    layer_backward: combine, gate/router and dispatch backward, and the whole
+             MoELayer.backward."""
+    if args.probe == "layer_backward":
+        import torch
+        out = run_layer_backward(cfg, torch.device("cuda"))
+        print(json.dumps(out), flush=True)
+        return out
     if args.probe == "backward":
         import torch
         out = run_backward(cfg, torch.device("cuda"))
@@ -555,6 +563,83 @@ def run_backward(cfg, dev, calls=10, warmup=3):
                                          "once per weight update, outside the timed steps"},
             "note": "expert FFN input gradients: GEMM1 recomputed, dh with the SwiGLU-backward "
                     "epilogue, dx (3 launches); weight gradients beside them"}
+
+
+def run_layer_backward(cfg, dev, calls=10, warmup=3):
+    """The backward steps around the experts on the layer's routing of one
+    synthetic batch (BF16): moe_combine_backward, moe_route_backward,
+    moe_dispatch_backward, each against the HBM roofline of its algorithmic
+    bytes, and the whole MoELayer.backward (14 launches).  dy is seeded
+    N(0, 1) bf16.  CUDA events over `calls` calls after `warmup`."""
+    import torch
+    import sparse_moe_layer_limited_b200 as M
+    from synth import device as sdev
+    s = M.shape(cfg.T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f, M.DTYPE_BF16)
+    w1 = sdev.expert_weights_bf16(cfg, 0, "w1", dev)
+    w3 = sdev.expert_weights_bf16(cfg, 0, "w3", dev)
+    w13 = torch.empty(cfg.N + 1, 2 * cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
+    M.moe_pack_w13(s, w1, w3, w13)
+    del w1, w3
+    w2 = sdev.expert_weights_bf16(cfg, 0, "w2", dev)
+    w13t = torch.empty(cfg.N + 1, cfg.d, 2 * cfg.f, dtype=torch.bfloat16, device=dev)
+    w2t = torch.empty(cfg.N + 1, cfg.f, cfg.d, dtype=torch.bfloat16, device=dev)
+    M.moe_transpose_weights(s, w13, w2, w13t, w2t)
+    router = torch.from_numpy(gen.make_router(cfg)).to(dev)
+    bias = torch.from_numpy(gen.make_bias(cfg)).to(dev)
+    layer = M.MoELayer(s, router, bias, w13, w2, gamma=cfg.gamma)
+    x = sdev.x_bf16(cfg, 0, device=dev)
+    layer.forward(x, update_bias=False)
+    g = torch.Generator(device=dev).manual_seed(11)
+    T, K, d, N = cfg.T, cfg.K, cfg.d, cfg.N
+    dy = torch.randn(T, d, generator=g, device=dev).to(torch.bfloat16)
+    dyp = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
+    dgate = torch.empty(T, K, dtype=torch.float32, device=dev)
+    dl = torch.empty(T, K, dtype=torch.float32, device=dev)
+    dxr = torch.empty(T, d, dtype=torch.float32, device=dev)
+    dR = torch.empty(N, d, dtype=torch.float32, device=dev)
+    dxp = torch.randn(T * K, d, generator=g, device=dev).to(torch.bfloat16)
+    dx = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(calls):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / calls
+
+    P = peaks()
+    steps = {
+        "combine_backward": (
+            lambda: M.moe_combine_backward(s, dy, layer.y_perm, layer.slot, layer.topk_gate, dyp,
+                                           dgate),
+            2.0 * (T * d + 2 * T * K * d), "dy + y_perm read, dy_perm written (bf16)"),
+        "route_backward": (
+            lambda: M.moe_route_backward(s, x, router, layer.topk_idx, dgate, layer.offsets,
+                                         layer.perm_tok, layer.slot, dl, dxr, dR),
+            2.0 * T * d + 4.0 * (N * d + T * d + N * d),
+            "x and the router read once, dx_route and drouter written (fp32)"),
+        "dispatch_backward": (
+            lambda: M.moe_dispatch_backward(s, dxp, dy, layer.slot, dxr, dx),
+            2.0 * (T * K * d + 2 * T * d) + 4.0 * T * d,
+            "dx_perm, dx_shared, dx_route read, dx written"),
+    }
+    out = {"workload": workload_name(cfg)}
+    for name, (fn, nbytes, what) in steps.items():
+        ms = timed(fn)
+        out[name] = {"ms": ms, "bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                     "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / P["hbm"], "bytes_note": what}
+    ms_all = timed(lambda: layer.backward(x, dy, w13t, w2t))
+    out["layer_backward"] = {"ms": ms_all, "tokens_per_s": T / (ms_all / 1e3),
+                             "gpu_launches_per_call": 14,
+                             "note": "combine, expert input and weight gradients, gate and "
+                                     "router, dispatch"}
+    out["device_status"] = layer.backward_status()
+    return out
 
 
 def softmax_route_baseline(M, s, x, router, layer, cfg, stream, reps=20):
