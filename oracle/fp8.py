@@ -14,6 +14,15 @@ E4M3(float32(v * inverse)); dequantised value = code * scale; a tile whose
 amax is 0 gets scale 1 and all-zero codes.  The block-scaled GEMM keeps one
 float64 partial sum per 128-wide K slice and applies both scales to it, which
 is the exact value of sum_k (qa*sa)(qb*sb).
+
+E5M2 (the same OCP definition, "E5M2") is the gradient format: [P3] (the
+10100.com article on the V3 report, FP8 paragraph) has the forward pass in
+E4M3 and the backward pass in E5M2.  1 sign bit, 5 exponent bits with bias
+15, 2 mantissa bits; exponent field 0 encodes subnormals (m/4 * 2^-14);
+S.11111.00 is infinity and S.11111.{01,10,11} NaN, so the largest finite
+magnitude is 1.75 * 2^15 = 57344.  Readings taken: encoding is
+round-to-nearest-even with saturation to +-57344 (like E4M3 here), and a
+gradient tile is scaled like an activation tile with 57344 in place of 448.
 """
 from __future__ import annotations
 
@@ -54,16 +63,54 @@ def e4m3_encode(v) -> np.ndarray:
     return np.where(np.isnan(v), np.uint8(0x7F), code).astype(np.uint8)
 
 
-def _quant_tiles(tiles32: np.ndarray):
+def e5m2_decode(codes) -> np.ndarray:
+    """E5M2 bit patterns (uint8) -> float64 values (+-inf for S.11111.00,
+    NaN for S.11111.{01,10,11})."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    E = (c >> 2) & 0x1F
+    M = c & 0x3
+    mag = np.where(E == 0, (M / 4.0) * 2.0 ** -14, (1.0 + M / 4.0) * np.exp2(E - 15.0))
+    mag = np.where(E == 31, np.where(M == 0, np.inf, np.nan), mag)
+    return sign * mag
+
+
+def e5m2_all_values() -> np.ndarray:
+    """Values of all 256 E5M2 codes, index = code."""
+    return e5m2_decode(np.arange(256, dtype=np.uint8))
+
+
+_POS_VALUES_E5M2 = e5m2_all_values()[:124]     # codes 0x00..0x7B: 0 .. 57344, increasing
+
+
+def e5m2_encode(v) -> np.ndarray:
+    """float -> E5M2 code, round to nearest (ties to even mantissa),
+    saturating overflow (infinities included) to +-57344; NaN -> 0x7F."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.nan_to_num(np.abs(v), nan=0.0, posinf=np.inf)
+    fin = np.isfinite(a)
+    _, e = np.frexp(np.where(fin, a, 0.0))     # a = m * 2**e, 0.5 <= m < 1
+    step_exp = np.maximum(e - 3, -16)          # 2 mantissa bits; subnormal step 2^-16
+    r = np.ldexp(np.rint(np.ldexp(np.where(fin, a, 0.0), -step_exp)), step_exp)
+    r = np.where(fin, np.minimum(r, 57344.0), 57344.0)
+    code = np.searchsorted(_POS_VALUES_E5M2, r).astype(np.uint8)
+    assert np.all(_POS_VALUES_E5M2[np.minimum(code, 123)] == r)
+    code = np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+    return np.where(np.isnan(v), np.uint8(0x7F), code).astype(np.uint8)
+
+
+def _quant_tiles(tiles32: np.ndarray, fmax: float = 448.0, encode=None):
     """Quantise tiles [..., n] (float32 values), each with its own online
-    scale from its max-abs.  Returns (codes [..., n], scales [...])."""
+    scale from its max-abs (scale = amax / fmax).  ``encode`` defaults to
+    E4M3.  Returns (codes [..., n], scales [...])."""
+    encode = e4m3_encode if encode is None else encode
     amax = np.max(np.abs(tiles32), axis=-1).astype(np.float32)
     zero = amax == 0
     safe = np.where(zero, np.float32(1.0), amax).astype(np.float32)
-    scale = np.where(zero, np.float32(1.0), safe / np.float32(448.0)).astype(np.float32)
-    inv = (np.float32(448.0) / safe).astype(np.float32)
+    scale = np.where(zero, np.float32(1.0), safe / np.float32(fmax)).astype(np.float32)
+    inv = (np.float32(fmax) / safe).astype(np.float32)
     prod = (tiles32 * inv[..., None]).astype(np.float32)
-    codes = np.where(zero[..., None], np.uint8(0), e4m3_encode(prod)).astype(np.uint8)
+    codes = np.where(zero[..., None], np.uint8(0), encode(prod)).astype(np.uint8)
     return codes, scale
 
 
@@ -73,6 +120,16 @@ def quant_rows_1x128(a):
     a32 = np.asarray(a, dtype=np.float32)
     M, K = a32.shape
     codes, scales = _quant_tiles(a32.reshape(M, K // 128, 128))
+    return codes.reshape(M, K), scales
+
+
+def quant_rows_1x128_e5m2(g):
+    """Per-row, per-128-column E5M2 quantisation of gradients [M, K]
+    (K % 128 == 0), scale = amax / 57344.  Returns (codes uint8 [M, K],
+    scales float32 [M, K/128])."""
+    g32 = np.asarray(g, dtype=np.float32)
+    M, K = g32.shape
+    codes, scales = _quant_tiles(g32.reshape(M, K // 128, 128), 57344.0, e5m2_encode)
     return codes.reshape(M, K), scales
 
 

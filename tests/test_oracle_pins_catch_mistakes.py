@@ -12,6 +12,7 @@ import oracle.fp8
 import oracle.moe
 from tests import test_oracle_backward as PB
 from tests import test_oracle_dispatch_expert as PD
+from tests import test_oracle_e5m2 as PE
 from tests import test_oracle_fp8 as PF
 from tests import test_oracle_layer_backward as PL
 from tests import test_oracle_route as PR
@@ -21,6 +22,7 @@ ORIG = {name: getattr(oracle.moe, name) for name in (
     "dispatch", "swiglu_expert_backward", "route_backward", "dispatch_backward",
     "combine_backward", "round_bf16", "affinity")}
 ORIG_E4M3 = oracle.fp8.e4m3_encode
+ORIG_E5M2 = oracle.fp8.e5m2_encode
 
 
 # ---- the planted mistakes -------------------------------------------------------------
@@ -172,6 +174,25 @@ def test_planted_e4m3_rounding_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "e4m3_encode", e4m3_ties_away)
     assert _fails([PF.test_exhaustive_code_table, PF.test_midpoints_round_to_even_and_saturate,
                    PF.test_encode_matches_torch_in_range])
+
+
+def e5m2_ties_away(v):
+    v = np.asarray(v, dtype=np.float64)
+    return ORIG_E5M2(v * (1.0 + 1e-9))
+
+
+def e5m2_overflow_to_inf(v):
+    c = ORIG_E5M2(v)
+    big = np.abs(np.asarray(v, dtype=np.float64)) > 57344.0
+    return np.where(big, (c & 0x80) | 0x7C, c).astype(np.uint8)
+
+
+@pytest.mark.parametrize("mutant", [e5m2_ties_away, e5m2_overflow_to_inf])
+def test_planted_e5m2_mistake_is_caught(monkeypatch, mutant):
+    monkeypatch.setattr(oracle.fp8, "e5m2_encode", mutant)
+    monkeypatch.setattr(oracle, "e5m2_encode", mutant)
+    assert _fails([PE.test_exhaustive_code_table, PE.test_midpoints_round_to_even_and_saturate,
+                   PE.test_encode_matches_torch_in_range])
 
 
 def test_the_unmodified_oracle_passes_the_same_pins():
