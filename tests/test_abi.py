@@ -90,3 +90,32 @@ def test_workspace_layout_grows_with_shape(L):
     b = L.workspace_size(L.shape(2048, 256, 8, 2, 2, 1, 256, L.DTYPE_BF16))
     assert 0 < a < b
     assert a % 256 == 0
+
+
+def test_backward_entry_points_reject_bad_arguments_before_any_launch(L):
+    f = L.lib()
+    fp32 = ctypes.byref(L.shape(128, 64, 16, 4, 1, 1, 32, L.DTYPE_FP32))
+    bf16 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 256, L.DTYPE_BF16))
+    bf16_f128 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 128, L.DTYPE_BF16))
+    mis = ctypes.c_void_p(0x1001)
+    ok = ctypes.c_void_p(0x1000)   # aligned, never dereferenced: the checks fail first
+    # layer backward steps: every pointer is required (dx_route may be NULL)
+    for s in (fp32, bf16):
+        assert f.moe_combine_backward(s, *([None] * 7)) == L.ERR_ARG
+        assert f.moe_route_backward(s, *([None] * 11)) == L.ERR_ARG
+        assert f.moe_dispatch_backward(s, *([None] * 6)) == L.ERR_ARG
+        assert f.moe_combine_backward(s, ok, ok, ok, ok, ok, mis, None) == L.ERR_ARG
+        assert f.moe_route_backward(s, *([ok] * 9), mis, ok, None) == L.ERR_ARG
+        # a misaligned optional dx_route is still rejected
+        assert f.moe_dispatch_backward(s, ok, ok, ok, mis, ok, None) == L.ERR_ARG
+        assert f.moe_dispatch_backward(s, ok, None, ok, None, ok, None) == L.ERR_ARG
+    assert f.moe_combine_backward(None, *([ok] * 6), None) == L.ERR_ARG
+    # expert backward and weight transposes: BF16 only; weight gradients need f % 256
+    assert f.moe_transpose_weights(fp32, ok, ok, ok, ok, None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dx(fp32, *([ok] * 11), None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dw(fp32, *([ok] * 8), None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dw(bf16_f128, *([ok] * 8), None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dx(bf16, *([None] * 11), None) == L.ERR_ARG
+    assert f.moe_expert_ffn_backward_dw(bf16, *([None] * 8), None) == L.ERR_ARG
+    assert f.moe_backward_workspace_size(fp32) == 0
+    assert f.moe_backward_workspace_size(bf16) > 0
