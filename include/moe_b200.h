@@ -297,6 +297,20 @@ int moe_route_backward(const moe_shape* shape, const void* x, const float* route
 int moe_dispatch_backward(const moe_shape* shape, const void* dx_perm, const void* dx_shared,
                           const int32_t* slot, const float* dx_route, void* dx, void* stream);
 
+/* moe_quantize_rows_e5m2: fine-grained quantisation of gradient rows to
+ * FP8-E5M2, the backward pass's format ([P3]: E4M3 forward, E5M2 backward;
+ * the 1x128 online scaling of [P1] §4.1).  Per 1x128 tile of each row:
+ *   scale = amax / 57344 and inverse = 57344 / amax (fp32, IEEE division),
+ *   code  = E5M2 round-to-nearest-even with saturation of v * inverse;
+ * an all-zero tile gets scale 1 and zero codes.
+ *   g       [rows, cols] bf16 row-major, cols % 128 == 0
+ *   codes   [rows, cols] uint8 E5M2 bit patterns
+ *   scales  block-major [cols/128, sc_ld] fp32, sc_ld >= rows (scales of one
+ *           128-column block contiguous over rows, like x_perm_scales)
+ * MOE_ERR_ARG for a bad size or a NULL / misaligned pointer. */
+int moe_quantize_rows_e5m2(const void* g, int64_t rows, int cols, uint8_t* codes,
+                           float* scales, int64_t sc_ld, void* stream);
+
 /* Auxiliary-loss-free bias update ([P4]; [P1] §1.2): for every expert,
  * bias[i] -= gamma if counts[i] * N > T * K, += gamma if counts[i] * N < T * K,
  * unchanged otherwise; fp32, in place. */

@@ -54,6 +54,8 @@ _SIGS = {
     "moe_combine_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
     "moe_route_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 11),
     "moe_dispatch_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
+    "moe_quantize_rows_e5m2": (ctypes.c_int, [_c_p, ctypes.c_int64, ctypes.c_int, _c_p, _c_p,
+                                              ctypes.c_int64, _c_p]),
     "moe_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
     "moe_transpose_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 5),
     "moe_expert_ffn_backward_dx": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
@@ -273,6 +275,18 @@ def moe_dispatch_backward(s, dx_perm, dx_shared, slot, dx_route, dx, stream=None
     _expect(dx, x_torch_dtype(s), s.T * s.d, "dx")
     _call("moe_dispatch_backward", ctypes.byref(s), _ptr(dx_perm), _ptr(dx_shared), _ptr(slot),
           _ptr(dx_route), _ptr(dx), _stream(stream))
+
+
+def moe_quantize_rows_e5m2(g, codes, scales, stream=None):
+    """g [rows, cols] bf16 -> codes [rows, cols] uint8 (E5M2 bits) and scales
+    [cols/128, sc_ld] fp32 (sc_ld = scales.shape[1] >= rows)."""
+    rows, cols = g.shape
+    _expect(g, torch.bfloat16, rows * cols, "g")
+    _expect(codes, torch.uint8, rows * cols, "codes")
+    if scales.dtype != torch.float32 or scales.dim() != 2 or scales.shape[0] != cols // 128:
+        raise ValueError("scales: expected float32 [cols/128, sc_ld]")
+    _call("moe_quantize_rows_e5m2", _ptr(g), ctypes.c_int64(rows), ctypes.c_int(cols),
+          _ptr(codes), _ptr(scales), ctypes.c_int64(scales.shape[1]), _stream(stream))
 
 
 def moe_bias_update(s, counts, bias, gamma, stream=None):

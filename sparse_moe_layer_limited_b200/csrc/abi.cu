@@ -307,6 +307,15 @@ int moe_dispatch_backward(const moe_shape* shape, const void* dx_perm, const voi
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int moe_quantize_rows_e5m2(const void* g, int64_t rows, int cols, uint8_t* codes,
+                           float* scales, int64_t sc_ld, void* stream) {
+  if (rows <= 0 || cols <= 0 || cols % 128 != 0 || sc_ld < rows) return MOE_ERR_ARG;
+  if (rows > (int64_t{1} << 40) / cols) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(g) || !ptr_ok(codes) || !ptr_ok(scales)) return MOE_ERR_ARG;
+  return cuda_status(launch_quant_rows_e5m2(g, rows, cols, codes, scales, sc_ld,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 int moe_bias_update(const moe_shape* shape, const int32_t* counts, float* bias, float gamma,
                     void* stream) {
   int rc = check(shape);

@@ -66,7 +66,8 @@ constexpr uint64_t FTimeoutNs = 2000000000ull;
 enum FEpi { kFEpiSwiGLUQuant = 0, kFEpiStore = 1 };
 
 // x [rows, d] bf16 -> codes [rows, d], scales block-major [d/128][sc_ld]; one
-// half-warp per tile.
+// half-warp per tile.  kE5M2: gradient rows in E5M2 instead of E4M3.
+template <bool kE5M2>
 __global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ x, long long rows, int d,
                                   uint8_t* __restrict__ q, float* __restrict__ sc,
                                   long long sc_ld) {
@@ -87,7 +88,7 @@ __global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ x, long long
     if (live)
       bf16x8_to_f32(*reinterpret_cast<const uint4*>(x + r * d + tc * QB + 8 * l16), v);
     uint2 codes;
-    const float s = quant_tile_16lanes(v, codes);
+    const float s = quant_tile_16lanes<kE5M2>(v, codes);
     if (live) {
       *reinterpret_cast<uint2*>(q + r * d + tc * QB + 8 * l16) = codes;
       if (l16 == 0) sc[(long long)tc * sc_ld + r] = s;
@@ -536,15 +537,28 @@ cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
-                              long long sc_ld, cudaStream_t st) {
+namespace {
+template <bool kE5M2>
+cudaError_t quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
+                       long long sc_ld, cudaStream_t st) {
   const long long tiles = rows * (d / QB);
   long long blocks = (tiles * 16 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  quant_rows_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rows, d,
-                                                 q, sc, sc_ld);
+  quant_rows_kernel<kE5M2><<<(int)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                        rows, d, q, sc, sc_ld);
   return note_cuda(cudaGetLastError(), "1x128 quantisation launch");
+}
+}  // namespace
+
+cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
+                              long long sc_ld, cudaStream_t st) {
+  return quant_rows<false>(x, rows, d, q, sc, sc_ld, st);
+}
+
+cudaError_t launch_quant_rows_e5m2(const void* g, long long rows, int d, uint8_t* q, float* sc,
+                                   long long sc_ld, cudaStream_t st) {
+  return quant_rows<true>(g, rows, d, q, sc, sc_ld, st);
 }
 
 cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const void* w2,

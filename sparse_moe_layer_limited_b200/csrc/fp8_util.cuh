@@ -14,8 +14,12 @@ namespace moe {
 constexpr int QB = 128;  // quantisation tile / K slice
 
 // A half-warp (16 lanes) holds one 128-wide tile, 8 consecutive elements per
-// lane.  Returns the tile scale; writes this lane's 8 codes.
+// lane.  Returns the tile scale; writes this lane's 8 codes.  kE5M2: the
+// gradient format of the backward pass (largest finite 57344) instead of
+// E4M3 (448), with the same scaling rule.
+template <bool kE5M2 = false>
 static __device__ __forceinline__ float quant_tile_16lanes(const float (&v)[8], uint2& codes) {
+  constexpr float kMax = kE5M2 ? 57344.f : 448.f;
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
@@ -25,8 +29,8 @@ static __device__ __forceinline__ float quant_tile_16lanes(const float (&v)[8], 
     codes = make_uint2(0u, 0u);
     return 1.f;
   }
-  const float scale = __fdiv_rn(amax, 448.f);
-  const float inv = __fdiv_rn(448.f, amax);
+  const float scale = __fdiv_rn(amax, kMax);
+  const float inv = __fdiv_rn(kMax, amax);
   uint32_t w[2];
 #pragma unroll
   for (int p = 0; p < 2; ++p) {
@@ -35,7 +39,8 @@ static __device__ __forceinline__ float quant_tile_16lanes(const float (&v)[8], 
     for (int q = 0; q < 2; ++q) {
       const int i = 4 * p + 2 * q;
       const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fmul_rn(v[i], inv), __fmul_rn(v[i + 1], inv)), __NV_SATFINITE, __NV_E4M3);
+          make_float2(__fmul_rn(v[i], inv), __fmul_rn(v[i + 1], inv)), __NV_SATFINITE,
+          kE5M2 ? __NV_E5M2 : __NV_E4M3);
       word |= (uint32_t)c2 << (16 * q);
     }
     w[p] = word;

@@ -138,6 +138,8 @@ int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_pe
                        const float* w13_scales, const float* w2_scales, void* y_perm,
                        void* y_shared, void* ws, cudaStream_t st);
 // x [rows, d] bf16 -> E4M3 codes [rows, d] and fp32 scales [rows, d/128].
+cudaError_t launch_quant_rows_e5m2(const void* g, long long rows, int d, uint8_t* q, float* sc,
+                                   long long sc_ld, cudaStream_t st);
 cudaError_t launch_quant_rows(const void* x, long long rows, int d, uint8_t* q, float* sc,
                               long long sc_ld,
                               cudaStream_t st);

@@ -119,3 +119,14 @@ def test_backward_entry_points_reject_bad_arguments_before_any_launch(L):
     assert f.moe_expert_ffn_backward_dw(bf16, *([None] * 8), None) == L.ERR_ARG
     assert f.moe_backward_workspace_size(fp32) == 0
     assert f.moe_backward_workspace_size(bf16) > 0
+
+
+def test_e5m2_quantiser_rejects_bad_sizes_before_any_launch(L):
+    f = L.lib()
+    ok = ctypes.c_void_p(0x1000)
+    mis = ctypes.c_void_p(0x1008)
+    assert f.moe_quantize_rows_e5m2(ok, 0, 128, ok, ok, 1, None) == L.ERR_ARG      # no rows
+    assert f.moe_quantize_rows_e5m2(ok, 4, 200, ok, ok, 4, None) == L.ERR_ARG      # cols % 128
+    assert f.moe_quantize_rows_e5m2(ok, 4, 128, ok, ok, 3, None) == L.ERR_ARG      # sc_ld < rows
+    assert f.moe_quantize_rows_e5m2(None, 4, 128, ok, ok, 4, None) == L.ERR_ARG
+    assert f.moe_quantize_rows_e5m2(ok, 4, 128, mis, ok, 4, None) == L.ERR_ARG
