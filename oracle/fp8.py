@@ -144,11 +144,17 @@ def quant_blocks_128(w):
     return codes, scales
 
 
-def fp8_gemm_ref(codes_a, sa, codes_b, sb) -> np.ndarray:
+_DECODE = {"e4m3": e4m3_decode, "e5m2": e5m2_decode}
+
+
+def fp8_gemm_ref(codes_a, sa, codes_b, sb, a_format: str = "e4m3",
+                 b_format: str = "e4m3") -> np.ndarray:
     """out[m, n] = sum_k (qa[m,k] sa[m,k/128]) (qb[n,k] sb[n/128,k/128]) in
-    float64, for A [M, K] (1x128 scales) and B [Nn, K] (128x128 scales)."""
-    qa = e4m3_decode(codes_a)
-    qb = e4m3_decode(codes_b)
+    float64, for A [M, K] (1x128 scales) and B [Nn, K] (128x128 scales).
+    ``a_format`` / ``b_format`` name each operand's FP8 format ("e4m3", or
+    "e5m2" for a gradient operand of the backward pass, [P3])."""
+    qa = _DECODE[a_format](codes_a)
+    qb = _DECODE[b_format](codes_b)
     M, K = qa.shape
     Nn = qb.shape[0]
     out = np.zeros((M, Nn), dtype=np.float64)

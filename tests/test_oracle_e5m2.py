@@ -95,3 +95,21 @@ def test_gradient_quantisation_error_bound(scale_exp):
             assert scales[r, t] == np.float32(np.float32(np.abs(tile).max()) / np.float32(57344))
             top = codes[r, 128 * t + int(np.argmax(np.abs(tile)))]
             assert abs(oracle.e5m2_decode(top)) == 57344.0
+
+
+def test_mixed_format_block_gemm_equals_the_dequantised_product():
+    """An E5M2 gradient operand (1x128 scales) against E4M3 weights (128x128
+    blocks): the block-scaled product equals the plain matmul of the two
+    dequantised matrices, and naming the wrong format changes it."""
+    rng = np.random.default_rng(21)
+    dy = rng.normal(size=(5, 256)) * 1e-3
+    w = rng.normal(size=(256, 256)) / 16
+    qa, sa = oracle.quant_rows_1x128_e5m2(dy)
+    qb, sb = oracle.quant_blocks_128(w)
+    got = oracle.fp8_gemm_ref(qa, sa, qb, sb, a_format="e5m2", b_format="e4m3")
+    a = oracle.e5m2_decode(qa) * np.repeat(sa.astype(np.float64), 128, axis=1)
+    b = oracle.e4m3_decode(qb) * np.kron(sb.astype(np.float64), np.ones((128, 128)))
+    np.testing.assert_allclose(got, a @ b.T, rtol=1e-12, atol=1e-18)
+    assert not np.allclose(oracle.fp8_gemm_ref(qa, sa, qb, sb), got)
+    # and it stays within the E5M2/E4M3 rounding of the exact product
+    assert np.linalg.norm(got - dy @ w.T) <= 0.15 * np.linalg.norm(dy @ w.T)
