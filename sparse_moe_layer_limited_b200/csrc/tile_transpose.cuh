@@ -22,7 +22,7 @@ constexpr int kTile = 64;
 constexpr int kTileThreads = 256;
 constexpr int kTileBytes = kTile * kTile * 2;
 
-__device__ __forceinline__ uint32_t tile_chunk(int c, int q) {
+__host__ __device__ __forceinline__ uint32_t tile_chunk(int c, int q) {
   return (uint32_t)c * 128u + ((uint32_t)((q ^ c ^ (c >> 3)) & 7) << 4);
 }
 
