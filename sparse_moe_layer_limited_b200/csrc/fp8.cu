@@ -44,6 +44,9 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <cstdlib>
+#include <cstring>
+
 #include "fp8_util.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -56,8 +59,11 @@ constexpr int FStages = 4;
 constexpr int FABytes = FBM * FBK;      // 16 KB
 constexpr int FBBytes = FBN * FBK;      // 32 KB
 constexpr int FStageBytes = FABytes + FBBytes;
-constexpr int FThreads = 576;   // warp 0 TMA, warp 1 MMA, warps 2..17 epilogue
-constexpr int FEpiWarps = 16;   // four per TMEM lane quadrant
+// warp 0 TMA, warp 1 MMA, then kEpiW epilogue warps (kEpiW / 4 per TMEM lane
+// quadrant): 16 by default; 8 (MOE_FP8_EPI=wide) gives each thread 128 running
+// sums and two TMEM loads in flight within the larger per-thread register
+// budget of a 10-warp CTA
+__host__ __device__ constexpr int fp8_threads(int epi_warps) { return 64 + 32 * epi_warps; }
 constexpr int FScaleSlots = 8;      // ring of per-slice activation-scale boxes
 constexpr int FScaleBox = 132;      // floats per box: 128 rows + up to 3 of alignment
 constexpr int FScaleSlotBytes = 640;
@@ -191,9 +197,16 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float x0, float x1, 
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
-template <int kEpi>
-__global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
+template <int kEpi, int kEpiW>
+__global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel(
     const __grid_constant__ Fp8Args args) {
+  static_assert(kEpiW == 16 || kEpiW == 8, "four or two epilogue warps per lane quadrant");
+  constexpr int FThreads = fp8_threads(kEpiW);
+  constexpr int FEpiWarps = kEpiW;
+  constexpr int kSub = kEpiW / 4;          // epilogue warps per TMEM lane quadrant
+  constexpr int kCols = FBN / kSub;        // accumulator columns per warp
+  constexpr int kFeat = (FBN / 2) / kSub;  // GEMM1: hidden features per warp
+  constexpr int kInFlight = kSub == 2 ? 2 : 1;  // 16-column TMEM loads per wait
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -379,11 +392,12 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       mbar_wait_bounded(drain, 0, args.status, FTimeoutNs / 8);
     }
   } else {
-    // ---- epilogue: warps 2..17 ----
-    // Warp w may read TMEM lanes 32*(w%4)..+31 (its row quadrant); the four
+    // ---- epilogue: warps 2 .. kEpiW+1 ----
+    // Warp w may read TMEM lanes 32*(w%4)..+31 (its row quadrant); the kSub
     // warps of a quadrant split the 256 columns: in GEMM1 warp `sub` owns the
-    // gate columns 32*sub.. and the up columns 128+32*sub.. (hidden features
-    // 32*sub..+31 of the tile), in GEMM2 the 64 columns 64*sub..
+    // gate columns kFeat*sub.. and the up columns 128+kFeat*sub.. (hidden
+    // features kFeat*sub..+kFeat-1 of the tile), in GEMM2 the kCols columns
+    // kCols*sub..
     const int q = warp & 3;
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
@@ -403,11 +417,11 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       // the slot's two weight-block scales follow the activation box: GEMM1
       // uses the gate block for its first 32 columns and the up block for the
       // rest, GEMM2 the block of its 64 columns
-      const int wA = (kEpi == kFEpiSwiGLUQuant) ? 0 : (sub >> 1);
-      const int wB = (kEpi == kFEpiSwiGLUQuant) ? 1 : (sub >> 1);
-      float acc[64];
+      const int wA = (kEpi == kFEpiSwiGLUQuant) ? 0 : (sub * kCols) / FBM;
+      const int wB = (kEpi == kFEpiSwiGLUQuant) ? 1 : (sub * kCols) / FBM;
+      float acc[kCols];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
       for (int kb = 0; kb < KB; ++kb, ++slice) {
         const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
         const uint32_t cs = slice % FScaleSlots, cph = (slice / FScaleSlots) & 1u;
@@ -426,21 +440,32 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * FBN;
+        // load c (16 columns) of this warp: GEMM1 gate loads first, then up
+        constexpr int kLoads = kCols / 16;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          int col;
-          if constexpr (kEpi == kFEpiSwiGLUQuant)
-            col = (c < 2) ? 32 * sub + 16 * c : 128 + 32 * sub + 16 * (c - 2);
-          else
-            col = 64 * sub + 16 * c;
-          const float sc = (c < 2) ? sA : sB;
-          uint32_t p[16];
-          tmem_ld16(taddr + col, p);
+        for (int c0 = 0; c0 < kLoads; c0 += kInFlight) {
+          uint32_t p[kInFlight][16];
+#pragma unroll
+          for (int j = 0; j < kInFlight; ++j) {
+            const int c = c0 + j;
+            int col;
+            if constexpr (kEpi == kFEpiSwiGLUQuant)
+              col = (c < kLoads / 2) ? kFeat * sub + 16 * c
+                                     : 128 + kFeat * sub + 16 * (c - kLoads / 2);
+            else
+              col = kCols * sub + 16 * c;
+            tmem_ld16(taddr + col, p[j]);
+          }
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; i += 2)
-            ffma2(acc[c * 16 + i], acc[c * 16 + i + 1], __uint_as_float(p[i]),
-                  __uint_as_float(p[i + 1]), sc);
+          for (int j = 0; j < kInFlight; ++j) {
+            const int c = c0 + j;
+            const float sc = (c < kLoads / 2) ? sA : sB;
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+              ffma2(acc[c * 16 + i], acc[c * 16 + i + 1], __uint_as_float(p[j][i]),
+                    __uint_as_float(p[j][i + 1]), sc);
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -449,29 +474,31 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
       if (!ok) break;
 
       if constexpr (kEpi == kFEpiSwiGLUQuant) {
-        // h for hidden features n*128 + 32*sub + i, i < 32
+        // h for hidden features n*128 + kFeat*sub + i, i < kFeat
         float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc[i] = silu_f(acc[i]) * acc[32 + i];
+        for (int i = 0; i < kFeat; ++i) {
+          acc[i] = silu_f(acc[i]) * acc[kFeat + i];
           amax = fmaxf(amax, fabsf(acc[i]));
         }
-        // the row's 1x128 tile spans the four warps of this quadrant
+        // the row's 1x128 tile spans the kSub warps of this quadrant
         float* xb = xchg + (local & 1) * 4 * FBM;
         xb[sub * FBM + row] = amax;
         __syncwarp();
         if (lane == 0) mbar_arrive(&xbar[local & 1]);
         if (!mbar_wait_bounded(&xbar[local & 1], (local >> 1) & 1, args.status, FTimeoutNs)) break;
-        amax = fmaxf(fmaxf(xb[row], xb[FBM + row]), fmaxf(xb[2 * FBM + row], xb[3 * FBM + row]));
+        amax = (kSub == 4) ? fmaxf(fmaxf(xb[row], xb[FBM + row]),
+                                   fmaxf(xb[2 * FBM + row], xb[3 * FBM + row]))
+                           : fmaxf(xb[row], xb[FBM + row]);
         const bool zero = amax == 0.f;
         const float scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
         const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
         if (valid) {
           uint8_t* qrow = ((g < args.N) ? args.q_routed + (long long)args.offsets[g] * args.out_ld
                                         : args.q_shared) +
-                          (long long)r * args.out_ld + n * QB + 32 * sub;
+                          (long long)r * args.out_ld + n * QB + kFeat * sub;
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
+          for (int v = 0; v < kFeat / 16; ++v) {
             uint32_t w4[4];
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {
@@ -500,9 +527,9 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
           __nv_bfloat16* yrow =
               ((g < args.N) ? args.y_routed + ((long long)args.offsets[g] + r) * args.out_ld
                             : args.y_shared + (long long)r * args.out_ld) +
-              n * FBN + 64 * sub;
+              n * FBN + kCols * sub;
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+          for (int v = 0; v < kCols / 8; ++v) {
             uint4 w;
             __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&w);
 #pragma unroll
@@ -523,16 +550,32 @@ __global__ void __launch_bounds__(FThreads, 1) grouped_gemm_fp8_kernel(
   }
 }
 
-template <int kEpi>
-cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
+template <int kEpi, int kEpiW>
+cudaError_t launch_fp8_gemm_w(const Fp8Args& a, cudaStream_t st) {
   const size_t smem = fp8_smem_bytes(a.N + 1);
-  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kEpi>,
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kEpi, kEpiW>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem),
                             "fp8 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
-  grouped_gemm_fp8_kernel<kEpi><<<num_sms(), FThreads, smem, st>>>(a);
+  grouped_gemm_fp8_kernel<kEpi, kEpiW><<<num_sms(), fp8_threads(kEpiW), smem, st>>>(a);
   return note_cuda(cudaGetLastError(), "fp8 GEMM launch");
+}
+
+// MOE_FP8_EPI=wide selects eight epilogue warps (read once per process).
+bool fp8_wide_epilogue() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("MOE_FP8_EPI");
+    v = (e != nullptr && std::strcmp(e, "wide") == 0) ? 1 : 0;
+  }
+  return v == 1;
+}
+
+template <int kEpi>
+cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
+  return fp8_wide_epilogue() ? launch_fp8_gemm_w<kEpi, 8>(a, st)
+                             : launch_fp8_gemm_w<kEpi, 16>(a, st);
 }
 
 }  // namespace
