@@ -179,3 +179,44 @@ def fp8_swiglu_expert(a, w1, w3, w2) -> np.ndarray:
     h = silu(fp8_gemm_ref(qa, sa, q1, s1)) * fp8_gemm_ref(qa, sa, q3, s3)
     qh, sh = quant_rows_1x128(h.astype(np.float32))
     return fp8_gemm_ref(qh, sh, q2, s2)
+
+
+def fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant: bool = True) -> dict:
+    """Input gradient of one SwiGLU expert with the FP8 recipe of the pages:
+    E4M3 operands in the forward pass and E5M2 gradients in the backward pass
+    ([P3]), each scaled per 1x128 tile (activations, gradients) or 128x128
+    block (weights) from its online max-abs ([P1] §4.1).  Steps:
+      1. g = a W1^T, u = a W3^T recomputed from the E4M3 operands of the
+         forward (a per 1x128 along d, W1 and W3 per block) and rounded to
+         bf16 (the values the recompute stores);
+      2. dy quantised to E5M2 per 1x128 along d; dh = dy W2 against the
+         E4M3 blocks of W2 (its 128x128 blocks read transposed);
+      3. dg = dh * u * silu'(g), du = dh * silu(g) from the bf16 g, u;
+      4. dg and du quantised to E5M2 per 1x128 along f (each 128-feature tile
+         is all gate or all up, as in the packed layout);
+      5. da = dg W1 + du W3 against the E4M3 blocks of W1 and W3.
+    ``quant=False`` skips every quantisation (float64 operands): the same
+    steps then give the exact backward with bf16 g and u.
+    Returns dict(da [M, d], dh [M, f], dg, du, g, u)."""
+    from .moe import round_bf16
+    a = np.asarray(a, dtype=np.float64)
+    w1, w3, w2 = (np.asarray(w, np.float64) for w in (w1, w3, w2))
+    dy = np.asarray(dy, dtype=np.float64)
+
+    def mm(x, w, x_format):
+        """x [M, K] (rows scaled per 1x128) times w [N, K]^T (128x128 blocks)."""
+        if not quant:
+            return x @ w.T
+        qx, sx = (quant_rows_1x128(x) if x_format == "e4m3"
+                  else quant_rows_1x128_e5m2(x))
+        qw, sw = quant_blocks_128(w)
+        return fp8_gemm_ref(qx, sx, qw, sw, a_format=x_format, b_format="e4m3")
+
+    g = round_bf16(mm(a, w1, "e4m3"))
+    u = round_bf16(mm(a, w3, "e4m3"))
+    dh = mm(dy, w2.T, "e5m2")
+    sig = 1.0 / (1.0 + np.exp(-g))
+    dg = dh * u * sig * (1.0 + g * (1.0 - sig))
+    du = dh * g * sig
+    da = mm(dg, w1.T, "e5m2") + mm(du, w3.T, "e5m2")
+    return dict(da=da, dh=dh, dg=dg, du=du, g=g, u=u)

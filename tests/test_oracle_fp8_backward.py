@@ -1,0 +1,72 @@
+"""Pins for oracle.fp8_swiglu_expert_backward_dx, the FP8 input gradient of
+one expert (E4M3 forward operands, E5M2 gradients).
+
+With the quantisation switched off the same steps must give the exact
+backward (pinned separately by finite differences), which checks the wiring:
+which weight, which transpose, which rounding of g and u.  With it switched
+on, the result must stay within the precision of the two formats, keep rows
+independent (every scale belongs to one row), and map a zero gradient to an
+exactly zero one."""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _case(seed, M=4, d=256, f=256):
+    rng = np.random.default_rng(seed)
+    a = oracle.round_bf16(rng.normal(size=(M, d)))
+    w1 = oracle.round_bf16(rng.normal(size=(f, d)) / np.sqrt(d))
+    w3 = oracle.round_bf16(rng.normal(size=(f, d)) / np.sqrt(d))
+    w2 = oracle.round_bf16(rng.normal(size=(d, f)) / np.sqrt(f))
+    dy = oracle.round_bf16(rng.normal(size=(M, d)) * 1e-2)
+    return a, w1, w3, w2, dy
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_without_quantisation_it_is_the_exact_backward(seed):
+    a, w1, w3, w2, dy = _case(seed)
+    got = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant=False)
+    want = oracle.swiglu_expert_backward(a, w1, w3, w2, dy, gu_round="bf16")
+    np.testing.assert_allclose(got["da"], want["da"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(got["dg"], want["dg"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(got["du"], want["du"], rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("seed", [2, 3])
+def test_fp8_error_stays_within_the_formats_precision(seed):
+    """E5M2 keeps 2 mantissa bits (half-step 2^-3 relative), E4M3 3 bits
+    (2^-4); summed over 256-long contractions the errors average, so the
+    gradient lands within 20% in norm, but it is not exact."""
+    a, w1, w3, w2, dy = _case(seed)
+    got = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy)
+    exact = oracle.swiglu_expert_backward(a, w1, w3, w2, dy)
+    def rel(x, y):
+        return np.linalg.norm(x - y) / np.linalg.norm(y)
+    assert rel(got["dh"], exact["dh"]) <= 0.1
+    assert rel(got["g"], a @ w1.T) <= 0.06
+    assert 1e-3 <= rel(got["da"], exact["da"]) <= 0.2
+
+
+def test_rows_are_independent():
+    a, w1, w3, w2, dy = _case(4, M=6)
+    whole = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy)["da"]
+    for r in range(6):
+        one = oracle.fp8_swiglu_expert_backward_dx(a[r:r + 1], w1, w3, w2, dy[r:r + 1])["da"]
+        np.testing.assert_array_equal(one[0], whole[r])
+
+
+def test_zero_gradient_gives_exact_zero():
+    a, w1, w3, w2, dy = _case(5)
+    got = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, np.zeros_like(dy))
+    assert np.all(got["dh"] == 0.0) and np.all(got["da"] == 0.0)
+
+
+def test_gradient_scale_invariance():
+    """Scaling dy by a power of two scales every E5M2 tile scale by the same
+    power and leaves the codes unchanged, so dh and da scale exactly."""
+    a, w1, w3, w2, dy = _case(6)
+    base = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy)
+    big = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy * 2.0 ** 20)
+    np.testing.assert_array_equal(big["dh"], base["dh"] * 2.0 ** 20)
+    np.testing.assert_array_equal(big["da"], base["da"] * 2.0 ** 20)

@@ -14,6 +14,7 @@ from tests import test_oracle_backward as PB
 from tests import test_oracle_dispatch_expert as PD
 from tests import test_oracle_e5m2 as PE
 from tests import test_oracle_fp8 as PF
+from tests import test_oracle_fp8_backward as PFB
 from tests import test_oracle_layer_backward as PL
 from tests import test_oracle_route as PR
 
@@ -193,6 +194,20 @@ def test_planted_e5m2_mistake_is_caught(monkeypatch, mutant):
     monkeypatch.setattr(oracle, "e5m2_encode", mutant)
     assert _fails([PE.test_exhaustive_code_table, PE.test_midpoints_round_to_even_and_saturate,
                    PE.test_encode_matches_torch_in_range])
+
+
+ORIG_FP8_BWD = oracle.fp8.fp8_swiglu_expert_backward_dx
+
+
+def fp8_backward_weights_swapped(a, w1, w3, w2, dy, quant=True):
+    return ORIG_FP8_BWD(a, w3, w1, w2, dy, quant)
+
+
+def test_planted_fp8_backward_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(oracle.fp8, "fp8_swiglu_expert_backward_dx", fp8_backward_weights_swapped)
+    monkeypatch.setattr(oracle, "fp8_swiglu_expert_backward_dx", fp8_backward_weights_swapped)
+    assert _fails([lambda: PFB.test_without_quantisation_it_is_the_exact_backward(0),
+                   lambda: PFB.test_fp8_error_stays_within_the_formats_precision(2)])
 
 
 def test_the_unmodified_oracle_passes_the_same_pins():
