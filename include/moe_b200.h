@@ -223,7 +223,9 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
  *              dispatched row and for the shared expert's rows
  *   ws_bwd     moe_backward_workspace_size(shape) bytes; its first 256 bytes
  *              are a status word like the forward workspace's (zero them once)
- * MOE_ERR_UNSUPPORTED for other dtypes. */
+ * MOE_ERR_UNSUPPORTED for other dtypes.  moe_transpose_weights takes the
+ * bf16 weights of a BF16 or E4M3 shape (MOE_ERR_UNSUPPORTED for FP32);
+ * moe_backward_workspace_size is 0 for an FP32 shape. */
 size_t moe_backward_workspace_size(const moe_shape* shape);
 int moe_transpose_weights(const moe_shape* shape, const void* w13, const void* w2, void* w13t,
                           void* w2t, void* stream);
@@ -232,6 +234,37 @@ int moe_expert_ffn_backward_dx(const moe_shape* shape, const void* x_perm,
                                const void* w13t, const void* w2t, const void* dy_perm,
                                const void* dy_shared, void* dx_perm, void* dx_shared,
                                void* ws_bwd, void* stream);
+
+/* FP8 input gradients of the experts, E4M3 mode with f % 256 == 0: E4M3
+ * operands in the forward and E5M2 gradients in the backward ([P3]), each
+ * scaled per 1x128 tile or 128x128 block from its online max-abs ([P1] §4.1):
+ *   1. g, u recomputed from the forward's E4M3 operands, stored bf16;
+ *   2. dy quantised to E5M2 per 1x128 along d;
+ *   3. dh = dy W2 against W2^T's E4M3 blocks, fp32 with per-slice promotion;
+ *      dg = dh * u * silu'(g), du = dh * silu(g), stored bf16;
+ *   4. [dg du] quantised to E5M2 per 1x128 along 2f;
+ *   5. da = [dg du] W13 against W13^T's E4M3 blocks -> bf16.
+ *   x_perm, x_perm_scales, offsets   E4M3 dispatch outputs (moe_dispatch)
+ *   x          [T, d] bf16 layer input (the shared expert's rows)
+ *   w13, w13_scales   the forward's E4M3 weights (moe_quantize_weights)
+ *   w13t, w13t_scales, w2t, w2t_scales   E4M3 codes [N+1, d, 2f], [N+1, f, d]
+ *              and block scales [N+1, d/128, 2f/128], [N+1, f/128, d/128]
+ *              from moe_quantize_weights_transposed
+ *   dy_perm, dy_shared, dx_perm, dx_shared   bf16, as at moe_expert_ffn_backward_dx
+ *   ws_bwd     moe_backward_workspace_size(shape) bytes (status word first)
+ * moe_quantize_weights_transposed quantises the bf16 transposes (from
+ * moe_transpose_weights) per 128x128 block: the blocks are the forward's
+ * blocks transposed, so codes and scales are the forward's, transposed. */
+int moe_quantize_weights_transposed(const moe_shape* shape, const void* w13t, const void* w2t,
+                                    void* w13t_q, float* w13t_scales, void* w2t_q,
+                                    float* w2t_scales, void* stream);
+int moe_expert_ffn_backward_dx_fp8(const moe_shape* shape, const void* x_perm,
+                                   const float* x_perm_scales, const int32_t* offsets,
+                                   const void* x, const void* w13, const float* w13_scales,
+                                   const void* w13t, const float* w13t_scales, const void* w2t,
+                                   const float* w2t_scales, const void* dy_perm,
+                                   const void* dy_shared, void* dx_perm, void* dx_shared,
+                                   void* ws_bwd, void* stream);
 
 /* moe_expert_ffn_backward_dw: the weight gradients ([P1] §2.2 MLP_W), BF16
  * mode with f % 256 == 0, to be called after moe_expert_ffn_backward_dx with

@@ -181,7 +181,8 @@ def fp8_swiglu_expert(a, w1, w3, w2) -> np.ndarray:
     return fp8_gemm_ref(qh, sh, q2, s2)
 
 
-def fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant: bool = True) -> dict:
+def fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant: bool = True,
+                                  dgu_round: str = "none") -> dict:
     """Input gradient of one SwiGLU expert with the FP8 recipe of the pages:
     E4M3 operands in the forward pass and E5M2 gradients in the backward pass
     ([P3]), each scaled per 1x128 tile (activations, gradients) or 128x128
@@ -196,7 +197,9 @@ def fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant: bool = True) -> dict
          is all gate or all up, as in the packed layout);
       5. da = dg W1 + du W3 against the E4M3 blocks of W1 and W3.
     ``quant=False`` skips every quantisation (float64 operands): the same
-    steps then give the exact backward with bf16 g and u.
+    steps then give the exact backward with bf16 g and u.  ``dgu_round=
+    'bf16'`` rounds dg and du to bf16 first (where an implementation stores
+    them before quantising).
     Returns dict(da [M, d], dh [M, f], dg, du, g, u)."""
     from .moe import round_bf16
     a = np.asarray(a, dtype=np.float64)
@@ -218,5 +221,7 @@ def fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant: bool = True) -> dict
     sig = 1.0 / (1.0 + np.exp(-g))
     dg = dh * u * sig * (1.0 + g * (1.0 - sig))
     du = dh * g * sig
+    if dgu_round == "bf16":
+        dg, du = round_bf16(dg), round_bf16(du)
     da = mm(dg, w1.T, "e5m2") + mm(du, w3.T, "e5m2")
     return dict(da=da, dh=dh, dg=dg, du=du, g=g, u=u)

@@ -56,6 +56,8 @@ _SIGS = {
     "moe_dispatch_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
     "moe_quantize_rows_e5m2": (ctypes.c_int, [_c_p, ctypes.c_int64, ctypes.c_int, _c_p, _c_p,
                                               ctypes.c_int64, _c_p]),
+    "moe_quantize_weights_transposed": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
+    "moe_expert_ffn_backward_dx_fp8": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 16),
     "moe_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
     "moe_transpose_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 5),
     "moe_expert_ffn_backward_dx": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
@@ -225,8 +227,8 @@ def backward_workspace_size(s) -> int:
 
 
 def moe_transpose_weights(s, w13, w2, w13t, w2t, stream=None):
-    _expect(w13t, w_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "w13t")
-    _expect(w2t, w_torch_dtype(s), (s.N + 1) * s.d * s.f, "w2t")
+    _expect(w13t, x_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "w13t")   # bf16 weights
+    _expect(w2t, x_torch_dtype(s), (s.N + 1) * s.d * s.f, "w2t")
     _call("moe_transpose_weights", ctypes.byref(s), _ptr(w13), _ptr(w2), _ptr(w13t), _ptr(w2t),
           _stream(stream))
 
@@ -237,6 +239,28 @@ def moe_expert_ffn_backward_dx(s, x_perm, offsets, x, w13, w13t, w2t, dy_perm, d
     _expect(dx_shared, x_torch_dtype(s), s.T * s.d, "dx_shared")
     _call("moe_expert_ffn_backward_dx", ctypes.byref(s), _ptr(x_perm), _ptr(offsets), _ptr(x),
           _ptr(w13), _ptr(w13t), _ptr(w2t), _ptr(dy_perm), _ptr(dy_shared), _ptr(dx_perm),
+          _ptr(dx_shared), _ptr(ws_bwd), _stream(stream))
+
+
+def moe_quantize_weights_transposed(s, w13t, w2t, w13t_q, w13t_scales, w2t_q, w2t_scales,
+                                    stream=None):
+    _expect(w13t_q, torch.float8_e4m3fn, (s.N + 1) * s.d * 2 * s.f, "w13t_q")
+    _expect(w2t_q, torch.float8_e4m3fn, (s.N + 1) * s.f * s.d, "w2t_q")
+    _expect(w13t_scales, torch.float32, (s.N + 1) * (s.d // 128) * (2 * s.f // 128),
+            "w13t_scales")
+    _expect(w2t_scales, torch.float32, (s.N + 1) * (s.f // 128) * (s.d // 128), "w2t_scales")
+    _call("moe_quantize_weights_transposed", ctypes.byref(s), _ptr(w13t), _ptr(w2t),
+          _ptr(w13t_q), _ptr(w13t_scales), _ptr(w2t_q), _ptr(w2t_scales), _stream(stream))
+
+
+def moe_expert_ffn_backward_dx_fp8(s, x_perm, x_perm_scales, offsets, x, w13, w13_scales, w13t,
+                                   w13t_scales, w2t, w2t_scales, dy_perm, dy_shared, dx_perm,
+                                   dx_shared, ws_bwd, stream=None):
+    _expect(dx_perm, torch.bfloat16, s.T * s.K * s.d, "dx_perm")
+    _expect(dx_shared, torch.bfloat16, s.T * s.d, "dx_shared")
+    _call("moe_expert_ffn_backward_dx_fp8", ctypes.byref(s), _ptr(x_perm), _ptr(x_perm_scales),
+          _ptr(offsets), _ptr(x), _ptr(w13), _ptr(w13_scales), _ptr(w13t), _ptr(w13t_scales),
+          _ptr(w2t), _ptr(w2t_scales), _ptr(dy_perm), _ptr(dy_shared), _ptr(dx_perm),
           _ptr(dx_shared), _ptr(ws_bwd), _stream(stream))
 
 

@@ -214,15 +214,51 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
 }
 
 size_t moe_backward_workspace_size(const moe_shape* shape) {
-  if (check(shape) != MOE_OK || shape->dtype != MOE_DTYPE_BF16) return 0;
-  return backward_ws_bytes(*shape);
+  if (check(shape) != MOE_OK) return 0;
+  if (shape->dtype == MOE_DTYPE_BF16) return backward_ws_bytes(*shape);
+  if (shape->dtype == MOE_DTYPE_E4M3) return bwd_layout_fp8(*shape).total;
+  return 0;
+}
+
+int moe_quantize_weights_transposed(const moe_shape* shape, const void* w13t, const void* w2t,
+                                    void* w13t_q, float* w13t_scales, void* w2t_q,
+                                    float* w2t_scales, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(w13t) || !ptr_ok(w2t) || !ptr_ok(w13t_q) || !ptr_ok(w13t_scales) ||
+      !ptr_ok(w2t_q) || !ptr_ok(w2t_scales))
+    return MOE_ERR_ARG;
+  return cuda_status(launch_quantize_weights_transposed(*shape, w13t, w2t, w13t_q, w13t_scales,
+                                                        w2t_q, w2t_scales,
+                                                        static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_ffn_backward_dx_fp8(const moe_shape* shape, const void* x_perm,
+                                   const float* x_perm_scales, const int32_t* offsets,
+                                   const void* x, const void* w13, const float* w13_scales,
+                                   const void* w13t, const float* w13t_scales, const void* w2t,
+                                   const float* w2t_scales, const void* dy_perm,
+                                   const void* dy_shared, void* dx_perm, void* dx_shared,
+                                   void* ws_bwd, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_E4M3 || shape->f % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(x_perm) || !ptr_ok(x_perm_scales) || !ptr_ok(offsets) || !ptr_ok(x) ||
+      !ptr_ok(w13) || !ptr_ok(w13_scales) || !ptr_ok(w13t) || !ptr_ok(w13t_scales) ||
+      !ptr_ok(w2t) || !ptr_ok(w2t_scales) || !ptr_ok(dy_perm) || !ptr_ok(dy_shared) ||
+      !ptr_ok(dx_perm) || !ptr_ok(dx_shared) || ws_check(shape, ws_bwd) != MOE_OK)
+    return MOE_ERR_ARG;
+  return launch_ffn_bwd_dx_e4m3(*shape, x_perm, x_perm_scales, offsets, x, w13, w13_scales, w13t,
+                                w13t_scales, w2t, w2t_scales, dy_perm, dy_shared, dx_perm,
+                                dx_shared, ws_bwd, static_cast<cudaStream_t>(stream));
 }
 
 int moe_transpose_weights(const moe_shape* shape, const void* w13, const void* w2, void* w13t,
                           void* w2t, void* stream) {
   int rc = check(shape);
   if (rc) return rc;
-  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (shape->dtype == MOE_DTYPE_FP32) return MOE_ERR_UNSUPPORTED;  // bf16 weights
   if (!ptr_ok(w13) || !ptr_ok(w2) || !ptr_ok(w13t) || !ptr_ok(w2t)) return MOE_ERR_ARG;
   return cuda_status(launch_transpose_weights(*shape, w13, w2, w13t, w2t,
                                               static_cast<cudaStream_t>(stream)));

@@ -7,6 +7,15 @@ namespace moe {
 
 __device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
+// SwiGLU backward for one hidden feature: with dh the gradient of
+// h = silu(g) * u, dg = dh * u * silu'(g) (silu'(g) = s (1 + g (1 - s)),
+// s = sigmoid(g)) and du = dh * silu(g).
+__device__ __forceinline__ void swiglu_bwd(float dh, float g, float u, float& dg, float& du) {
+  const float sg = 1.f / (1.f + expf(-g));
+  dg = dh * u * (sg * (1.f + g * (1.f - sg)));
+  du = dh * (g * sg);
+}
+
 // 32 fp32 values -> 32 bf16 (round to nearest even), four 16-byte stores.
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) {
   uint4 w[4];

@@ -47,6 +47,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "epilogue.cuh"
 #include "fp8_util.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -69,7 +70,7 @@ constexpr int FScaleBox = 132;      // floats per box: 128 rows + up to 3 of ali
 constexpr int FScaleSlotBytes = 640;
 constexpr uint64_t FTimeoutNs = 2000000000ull;
 
-enum FEpi { kFEpiSwiGLUQuant = 0, kFEpiStore = 1 };
+enum FEpi { kFEpiSwiGLUQuant = 0, kFEpiStore = 1, kFEpiSwiGLUBwd = 2 };
 
 // x [rows, d] bf16 -> codes [rows, d], scales block-major [d/128][sc_ld]; one
 // half-warp per tile.  kE5M2: gradient rows in E5M2 instead of E4M3.
@@ -170,8 +171,11 @@ struct alignas(64) Fp8Args {
   float* qs_routed;        // GEMM1: h scales, block-major [out_ld/128][qs_ld], routed rows
   float* qs_shared;        // ... shared-expert rows (same array, column TK onwards)
   long long qs_ld;
-  __nv_bfloat16* y_routed;  // GEMM2 outputs
-  __nv_bfloat16* y_shared;
+  __nv_bfloat16* y_routed;  // Store / SwiGLU-backward outputs, row (offsets[g] + r)
+  __nv_bfloat16* y_shared;  // ... shared-expert row r
+  const __nv_bfloat16* aux_routed;  // SwiGLU backward: the stored g, u [rows, 2f], packed
+  const __nv_bfloat16* aux_shared;
+  int a_format;             // A operand: kF8E4M3 (forward) or kF8E5M2 (gradients)
   uint32_t* status;
   int N, T;
   int rows_routed;
@@ -195,7 +199,6 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float x0, float x1, 
       : "f"(x0), "f"(x1), "f"(s));
 }
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
 template <int kEpi, int kEpiW>
 __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel(
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
   } else if (warp == 1) {
     // ---- MMA issuer: one TMEM slice buffer per 128-wide K slice ----
     if (lane == 0) {
-      const uint32_t idesc = idesc_e4m3_f32(FBM, FBN);
+      const uint32_t idesc = idesc_f8_f32(FBM, FBN, (uint32_t)args.a_format, kF8E4M3);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t slice = 0;
@@ -522,6 +525,36 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
             qs[(long long)n * args.qs_ld + r] = scale;
           }
         }
+      } else if constexpr (kEpi == kFEpiSwiGLUBwd) {
+        // acc holds dh for hidden features n*256 + kCols*sub + i; g, u and the
+        // outputs dg, du sit in the packed [rows, 2f] layout (gate block of
+        // 128 features, then their up block)
+        if (valid) {
+          const long long orow = (g < args.N) ? (long long)args.offsets[g] + r : (long long)r;
+          const __nv_bfloat16* arow =
+              ((g < args.N) ? args.aux_routed : args.aux_shared) + orow * args.out_ld;
+          __nv_bfloat16* drow = ((g < args.N) ? args.y_routed : args.y_shared) + orow * args.out_ld;
+#pragma unroll
+          for (int i0 = 0; i0 < kCols; i0 += 8) {
+            const int j0 = n * FBN + kCols * sub + i0;       // first feature of the 8
+            const int col = (j0 / 128) * 256 + (j0 % 128);   // its gate column; up at +128
+            float gt[8], up[8], dg[8], du[8];
+            bf16x8_load(arow + col, gt);
+            bf16x8_load(arow + col + 128, up);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) swiglu_bwd(acc[i0 + i], gt[i], up[i], dg[i], du[i]);
+            uint4 wg, wu;
+            __nv_bfloat162* hg = reinterpret_cast<__nv_bfloat162*>(&wg);
+            __nv_bfloat162* hu = reinterpret_cast<__nv_bfloat162*>(&wu);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              hg[i] = __floats2bfloat162_rn(dg[2 * i], dg[2 * i + 1]);
+              hu[i] = __floats2bfloat162_rn(du[2 * i], du[2 * i + 1]);
+            }
+            *reinterpret_cast<uint4*>(drow + col) = wg;
+            *reinterpret_cast<uint4*>(drow + col + 128) = wu;
+          }
+        }
       } else {
         if (valid) {
           __nv_bfloat16* yrow =
@@ -620,6 +653,162 @@ cudaError_t launch_quantize_weights(const moe_shape& s, const void* w13, const v
       static_cast<const __nv_bfloat16*>(w2), s.f, br2, bc2, static_cast<uint8_t*>(w2_q),
       w2_scales);
   return cudaGetLastError();
+}
+
+// The transposed weights W13^T [N+1, d, 2f] and W2^T [N+1, f, d] (bf16, from
+// moe_transpose_weights) quantised per 128x128 block like the forward's: the
+// blocks are the forward's blocks transposed, so codes and scales are theirs.
+cudaError_t launch_quantize_weights_transposed(const moe_shape& s, const void* w13t,
+                                               const void* w2t, void* w13t_q, float* w13t_scales,
+                                               void* w2t_q, float* w2t_scales, cudaStream_t st) {
+  const long long E = s.N + 1;
+  const long long br13 = E * s.d / QB;
+  const int bc13 = 2 * s.f / QB;
+  quant_blocks_kernel<<<(unsigned)(br13 * bc13), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w13t), 2 * s.f, br13, bc13,
+      static_cast<uint8_t*>(w13t_q), w13t_scales);
+  const long long br2 = E * s.f / QB;
+  const int bc2 = s.d / QB;
+  quant_blocks_kernel<<<(unsigned)(br2 * bc2), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w2t), s.d, br2, bc2, static_cast<uint8_t*>(w2t_q),
+      w2t_scales);
+  return cudaGetLastError();
+}
+
+BwdLayoutFp8 bwd_layout_fp8(const moe_shape& s) {
+  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
+  const size_t TK = (size_t)s.T * s.K, rows = TK + s.T;
+  const size_t ld_rows = (size_t)scale_ld((long long)rows), ld_x = (size_t)scale_ld(s.T);
+  const size_t twof = 2 * (size_t)s.f;
+  BwdLayoutFp8 B;
+  size_t off = 256;
+  B.gu = off;
+  off = al(off + rows * twof * 2);
+  B.dgu = off;
+  off = al(off + rows * twof * 2);
+  B.xq = off;
+  off = al(off + (size_t)s.T * s.d);
+  B.xs = off;
+  off = al(off + (size_t)(s.d / QB) * ld_x * 4);
+  B.dyq = off;
+  off = al(off + rows * s.d);
+  B.dys = off;
+  off = al(off + (size_t)(s.d / QB) * ld_rows * 4);
+  B.dguq = off;
+  off = al(off + rows * twof);
+  B.dgus = off;
+  off = al(off + (twof / QB) * ld_rows * 4);
+  B.total = off;
+  return B;
+}
+
+// The experts' input gradients in FP8 (E5M2 gradients against E4M3 weights):
+//   1. g, u recomputed from the forward's E4M3 operands, stored bf16 (Store);
+//   2. dY quantised to E5M2 per 1x128 along d;
+//   3. dH = dY W2 against W2^T's E4M3 blocks, SwiGLU-backward epilogue -> dg, du bf16;
+//   4. dG U quantised to E5M2 per 1x128 along 2f;
+//   5. dX = dGU W13 against W13^T's E4M3 blocks (Store).
+int launch_ffn_bwd_dx_e4m3(const moe_shape& s, const void* x_perm, const float* x_perm_scales,
+                           const int32_t* offsets, const void* x, const void* w13q,
+                           const float* w13_scales, const void* w13tq, const float* w13t_scales,
+                           const void* w2tq, const float* w2t_scales, const void* dy_perm,
+                           const void* dy_shared, void* dx_perm, void* dx_shared, void* ws_bwd,
+                           cudaStream_t st) {
+  const BwdLayoutFp8 B = bwd_layout_fp8(s);
+  uint8_t* w = static_cast<uint8_t*>(ws_bwd);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w);
+  __nv_bfloat16* GU = reinterpret_cast<__nv_bfloat16*>(w + B.gu);
+  __nv_bfloat16* dGU = reinterpret_cast<__nv_bfloat16*>(w + B.dgu);
+  uint8_t* xq = w + B.xq;
+  float* xs = reinterpret_cast<float*>(w + B.xs);
+  uint8_t* dyq = w + B.dyq;
+  float* dys = reinterpret_cast<float*>(w + B.dys);
+  uint8_t* dguq = w + B.dguq;
+  float* dgus = reinterpret_cast<float*>(w + B.dgus);
+  const uint64_t TK = (uint64_t)s.T * s.K, rows = TK + s.T;
+  const uint64_t twof = 2ull * s.f;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const long long ld_routed = scale_ld((long long)TK), ld_x = scale_ld(s.T);
+  const long long ld_rows = scale_ld((long long)rows);
+  auto common = [&](Fp8Args& a, int n_acc, int k_dim, int out_ld, int a_format,
+                    int a_shared_row0) {
+    a.offsets = offsets;
+    a.status = status;
+    a.N = s.N;
+    a.T = s.T;
+    a.rows_routed = (int)TK;
+    a.a_shared_row0 = a_shared_row0;
+    a.n_acc = n_acc;
+    a.k_dim = k_dim;
+    a.out_ld = out_ld;
+    a.a_format = a_format;
+  };
+
+  // 1. g, u = A W13^T in E4M3, stored bf16 [rows, 2f]
+  if (launch_quant_rows(x, s.T, s.d, xq, xs, ld_x, st) != cudaSuccess) return MOE_ERR_CUDA;
+  Fp8Args g1{};
+  bool ok = make_map(&g1.tmA_routed, x_perm, U8, 1, s.d, TK, FBK, FBM) &&
+            make_map(&g1.tmA_shared, xq, U8, 1, s.d, s.T, FBK, FBM) &&
+            make_map(&g1.tmB, w13q, U8, 1, s.d, (uint64_t)(s.N + 1) * twof, FBK, FBN) &&
+            make_map_f32_rows(&g1.tmS_routed, x_perm_scales, ld_routed, s.d / QB, FScaleBox) &&
+            make_map_f32_rows(&g1.tmS_shared, xs, ld_x, s.d / QB, FScaleBox);
+  if (!ok) {
+    note_text("fp8 backward GEMM1: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
+  common(g1, (int)twof, s.d, (int)twof, kF8E4M3, 0);
+  g1.sw = w13_scales;
+  g1.y_routed = GU;
+  g1.y_shared = GU + TK * twof;
+  if (launch_fp8_gemm<kFEpiStore>(g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // 2. dY -> E5M2, routed rows then shared rows, one block-major scale array
+  if (launch_quant_rows_e5m2(dy_perm, (long long)TK, s.d, dyq, dys, ld_rows, st) != cudaSuccess ||
+      launch_quant_rows_e5m2(dy_shared, s.T, s.d, dyq + TK * s.d, dys + TK, ld_rows, st) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  // 3. dH = dY W2 (B = W2^T [(N+1) f, d]), SwiGLU backward into dGU
+  Fp8Args g2{};
+  ok = make_map(&g2.tmA_routed, dyq, U8, 1, s.d, rows, FBK, FBM) &&
+       make_map(&g2.tmA_shared, dyq, U8, 1, s.d, rows, FBK, FBM) &&
+       make_map(&g2.tmB, w2tq, U8, 1, s.d, (uint64_t)(s.N + 1) * s.f, FBK, FBN) &&
+       make_map_f32_rows(&g2.tmS_routed, dys, ld_rows, s.d / QB, FScaleBox) &&
+       make_map_f32_rows(&g2.tmS_shared, dys, ld_rows, s.d / QB, FScaleBox);
+  if (!ok) {
+    note_text("fp8 backward dH GEMM: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
+  common(g2, s.f, s.d, (int)twof, kF8E5M2, (int)TK);
+  g2.sw = w2t_scales;
+  g2.aux_routed = GU;
+  g2.aux_shared = GU + TK * twof;
+  g2.y_routed = dGU;
+  g2.y_shared = dGU + TK * twof;
+  if (launch_fp8_gemm<kFEpiSwiGLUBwd>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // 4. dGU -> E5M2 over all rows
+  if (launch_quant_rows_e5m2(dGU, (long long)rows, (int)twof, dguq, dgus, ld_rows, st) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  // 5. dX = dGU W13 (B = W13^T [(N+1) d, 2f])
+  Fp8Args g3{};
+  ok = make_map(&g3.tmA_routed, dguq, U8, 1, twof, rows, FBK, FBM) &&
+       make_map(&g3.tmA_shared, dguq, U8, 1, twof, rows, FBK, FBM) &&
+       make_map(&g3.tmB, w13tq, U8, 1, twof, (uint64_t)(s.N + 1) * s.d, FBK, FBN) &&
+       make_map_f32_rows(&g3.tmS_routed, dgus, ld_rows, (int)(twof / QB), FScaleBox) &&
+       make_map_f32_rows(&g3.tmS_shared, dgus, ld_rows, (int)(twof / QB), FScaleBox);
+  if (!ok) {
+    note_text("fp8 backward dX GEMM: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
+  common(g3, s.d, (int)twof, s.d, kF8E5M2, (int)TK);
+  g3.sw = w13t_scales;
+  g3.y_routed = static_cast<__nv_bfloat16*>(dx_perm);
+  g3.y_shared = static_cast<__nv_bfloat16*>(dx_shared);
+  if (launch_fp8_gemm<kFEpiStore>(g3, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 int launch_ffn_tc_e4m3(const moe_shape& s, const void* x_perm, const float* x_perm_scales,

@@ -430,12 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
               bf16x8_load(arow + col + 128 + 8 * q4, up + 8 * q4);
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float dh = __uint_as_float(v[i]);
-              const float sg = 1.f / (1.f + expf(-gt[i]));
-              dg[i] = dh * up[i] * (sg * (1.f + gt[i] * (1.f - sg)));
-              du[i] = dh * (gt[i] * sg);
-            }
+            for (int i = 0; i < 32; ++i)
+              swiglu_bwd(__uint_as_float(v[i]), gt[i], up[i], dg[i], du[i]);
             store_row32(orow + col, dg);
             store_row32(orow + col + 128, du);
           }

@@ -99,6 +99,24 @@ struct BwdLayout {
   size_t gu = 0, dgu = 0, colbase = 0, at = 0, dyt = 0, ht = 0, dgut = 0;
   size_t total = 0;
 };
+// Backward workspace of the FP8 (E4M3) mode: status word, then the stored g, u
+// and dg, du (bf16 [T*K + T, 2f], packed like W13), x in E4M3 for the shared
+// expert, and the E5M2 gradients dY [T*K + T, d] and dGU [T*K + T, 2f] with
+// their block-major 1x128 scales.
+struct BwdLayoutFp8 {
+  size_t gu = 0, dgu = 0, xq = 0, xs = 0, dyq = 0, dys = 0, dguq = 0, dgus = 0;
+  size_t total = 0;
+};
+BwdLayoutFp8 bwd_layout_fp8(const moe_shape& s);
+int launch_ffn_bwd_dx_e4m3(const moe_shape& s, const void* x_perm, const float* x_perm_scales,
+                           const int32_t* offsets, const void* x, const void* w13q,
+                           const float* w13_scales, const void* w13tq, const float* w13t_scales,
+                           const void* w2tq, const float* w2t_scales, const void* dy_perm,
+                           const void* dy_shared, void* dx_perm, void* dx_shared, void* ws_bwd,
+                           cudaStream_t st);
+cudaError_t launch_quantize_weights_transposed(const moe_shape& s, const void* w13t,
+                                               const void* w2t, void* w13t_q, float* w13t_scales,
+                                               void* w2t_q, float* w2t_scales, cudaStream_t st);
 long long wgrad_cols(const moe_shape& s);
 BwdLayout bwd_layout(const moe_shape& s);
 size_t backward_ws_bytes(const moe_shape& s);

@@ -209,10 +209,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
 }
-// Instruction descriptor, kind::f8f6f4 with E4M3 A/B, fp32 accumulate, K-major.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) |
+// Instruction descriptor, kind::f8f6f4, fp32 accumulate, K-major; operand
+// formats in bits 7-9 (A) and 10-12 (B): 0 = E4M3, 1 = E5M2.
+constexpr uint32_t kF8E4M3 = 0, kF8E5M2 = 1;
+__host__ __device__ constexpr uint32_t idesc_f8_f32(int M, int N, uint32_t a_fmt,
+                                                    uint32_t b_fmt) {
+  return (1u << 4) | ((a_fmt & 7u) << 7) | ((b_fmt & 7u) << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+// E4M3 A and B.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return idesc_f8_f32(M, N, kF8E4M3, kF8E4M3);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,

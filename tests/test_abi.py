@@ -130,3 +130,20 @@ def test_e5m2_quantiser_rejects_bad_sizes_before_any_launch(L):
     assert f.moe_quantize_rows_e5m2(ok, 4, 128, ok, ok, 3, None) == L.ERR_ARG      # sc_ld < rows
     assert f.moe_quantize_rows_e5m2(None, 4, 128, ok, ok, 4, None) == L.ERR_ARG
     assert f.moe_quantize_rows_e5m2(ok, 4, 128, mis, ok, 4, None) == L.ERR_ARG
+
+
+def test_fp8_backward_entry_points_reject_bad_arguments_before_any_launch(L):
+    f = L.lib()
+    ok = ctypes.c_void_p(0x1000)
+    e4m3 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 256, L.DTYPE_E4M3))
+    e4m3_f128 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 128, L.DTYPE_E4M3))
+    bf16 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 256, L.DTYPE_BF16))
+    fp32 = ctypes.byref(L.shape(128, 64, 16, 4, 1, 1, 32, L.DTYPE_FP32))
+    assert f.moe_expert_ffn_backward_dx_fp8(bf16, *([ok] * 15), None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dx_fp8(e4m3_f128, *([ok] * 15), None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dx_fp8(e4m3, *([None] * 15), None) == L.ERR_ARG
+    assert f.moe_quantize_weights_transposed(bf16, *([ok] * 6), None) == L.ERR_UNSUPPORTED
+    assert f.moe_quantize_weights_transposed(e4m3, *([None] * 6), None) == L.ERR_ARG
+    assert f.moe_transpose_weights(fp32, ok, ok, ok, ok, None) == L.ERR_UNSUPPORTED
+    assert f.moe_transpose_weights(e4m3, None, ok, ok, ok, None) == L.ERR_ARG
+    assert f.moe_backward_workspace_size(e4m3) > 0

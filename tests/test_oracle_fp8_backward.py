@@ -70,3 +70,12 @@ def test_gradient_scale_invariance():
     big = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy * 2.0 ** 20)
     np.testing.assert_array_equal(big["dh"], base["dh"] * 2.0 ** 20)
     np.testing.assert_array_equal(big["da"], base["da"] * 2.0 ** 20)
+
+
+def test_bf16_rounding_of_dg_du_is_the_stated_rounding():
+    a, w1, w3, w2, dy = _case(7)
+    got = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant=False, dgu_round="bf16")
+    want = oracle.swiglu_expert_backward(a, w1, w3, w2, dy, gu_round="bf16", dgu_round="bf16")
+    np.testing.assert_allclose(got["da"], want["da"], rtol=1e-12, atol=1e-15)
+    q = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, dgu_round="bf16")
+    assert np.all(oracle.round_bf16(q["dg"]) == q["dg"]) and np.all(oracle.round_bf16(q["du"]) == q["du"])
