@@ -44,5 +44,6 @@ from .moe import (  # noqa: F401
 from .fp8 import (  # noqa: F401
     e4m3_decode, e4m3_encode, e4m3_all_values, quant_rows_1x128, quant_blocks_128,
     e5m2_decode, e5m2_encode, e5m2_all_values, quant_rows_1x128_e5m2,
-    fp8_gemm_ref, fp8_swiglu_expert, fp8_swiglu_expert_backward_dx,
+    fp8_gemm_ref, fp8_swiglu_expert, fp8_swiglu_expert_backward_dx, quant_cols_1x128,
+    fp8_weight_grad,
 )

@@ -225,3 +225,48 @@ def fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, quant: bool = True,
         dg, du = round_bf16(dg), round_bf16(du)
     da = mm(dg, w1.T, "e5m2") + mm(du, w3.T, "e5m2")
     return dict(da=da, dh=dh, dg=dg, du=du, g=g, u=u)
+
+
+def quant_cols_1x128(m, fmt: str = "e4m3"):
+    """Quantise the columns of m [R, C] in 128-row tiles (the contraction
+    dimension of a weight-gradient product), zero-padding R up to a multiple
+    of 128: each (column, 128-row tile) gets its own max-abs scale.
+    Returns (codes uint8 [R, C], scales float32 [ceil(R/128), C])."""
+    m32 = np.asarray(m, dtype=np.float32)
+    R, C = m32.shape
+    Rp = (R + 127) // 128 * 128
+    pad = np.zeros((Rp, C), dtype=np.float32)
+    pad[:R] = m32
+    tiles = pad.reshape(Rp // 128, 128, C).transpose(0, 2, 1)          # [tiles, C, 128]
+    if fmt == "e4m3":
+        codes, scales = _quant_tiles(tiles)
+    else:
+        codes, scales = _quant_tiles(tiles, 57344.0, e5m2_encode)
+    codes = codes.transpose(0, 2, 1).reshape(Rp, C)[:R]
+    return codes, scales
+
+
+def fp8_weight_grad(dy, h, quant: bool = True) -> np.ndarray:
+    """dW = dy^T h for one expert's rows (dy [R, M] the output gradients, h
+    [R, N] the layer inputs of that GEMM), with both operands in FP8 along
+    the contraction over the R rows: dy in E5M2 and h in E4M3, each column
+    scaled per 128-row tile from the expert's first row ([P3] E5M2 in the
+    backward pass; [P1] §4.1 1x128 online scaling, the tile laid along the
+    contraction as for every other FP8 product here).  Per tile kb:
+        dW[i, j] += sdy[kb, i] sh[kb, j] sum_{r in kb} qdy[r, i] qh[r, j]
+    in float64.  ``quant=False`` gives dy^T h exactly.  [M, N]."""
+    dy = np.asarray(dy, dtype=np.float64)
+    h = np.asarray(h, dtype=np.float64)
+    if not quant:
+        return dy.T @ h
+    R = dy.shape[0]
+    qd, sd = quant_cols_1x128(dy, "e5m2")
+    qh, sh = quant_cols_1x128(h, "e4m3")
+    vd, vh = e5m2_decode(qd), e4m3_decode(qh)
+    out = np.zeros((dy.shape[1], h.shape[1]), dtype=np.float64)
+    for kb in range((R + 127) // 128):
+        rs = slice(128 * kb, min(R, 128 * (kb + 1)))
+        part = vd[rs].T @ vh[rs]
+        out += (part * np.asarray(sd[kb], np.float64)[:, None]
+                * np.asarray(sh[kb], np.float64)[None, :])
+    return out

@@ -79,3 +79,45 @@ def test_bf16_rounding_of_dg_du_is_the_stated_rounding():
     np.testing.assert_allclose(got["da"], want["da"], rtol=1e-12, atol=1e-15)
     q = oracle.fp8_swiglu_expert_backward_dx(a, w1, w3, w2, dy, dgu_round="bf16")
     assert np.all(oracle.round_bf16(q["dg"]) == q["dg"]) and np.all(oracle.round_bf16(q["du"]) == q["du"])
+
+
+@pytest.mark.parametrize("R", [1, 100, 300])
+def test_weight_gradient_without_quantisation_is_exact(R):
+    rng = np.random.default_rng(R)
+    dy, h = rng.normal(size=(R, 256)), rng.normal(size=(R, 128))
+    np.testing.assert_allclose(oracle.fp8_weight_grad(dy, h, quant=False), dy.T @ h, rtol=1e-13)
+
+
+@pytest.mark.parametrize("R", [100, 300])
+def test_weight_gradient_error_and_tiles(R):
+    """Tiles run along the rows (R = 300: two full tiles and one of 44): the
+    dequantised operands reproduce the product exactly in float64, the error
+    against the exact product stays within the formats' precision, and
+    scaling either operand by a power of two scales the result exactly."""
+    rng = np.random.default_rng(R + 1)
+    dy, h = rng.normal(size=(R, 256)) * 1e-3, rng.normal(size=(R, 128))
+    got = oracle.fp8_weight_grad(dy, h)
+    qd, sd = oracle.quant_cols_1x128(dy, "e5m2")
+    qh, sh = oracle.quant_cols_1x128(h, "e4m3")
+    assert sd.shape == ((R + 127) // 128, 256) and qd.shape == dy.shape
+    vd = oracle.e5m2_decode(qd) * np.repeat(sd.astype(np.float64), 128, axis=0)[:R]
+    vh = oracle.e4m3_decode(qh) * np.repeat(sh.astype(np.float64), 128, axis=0)[:R]
+    np.testing.assert_allclose(got, vd.T @ vh, rtol=1e-12, atol=1e-15)
+    exact = dy.T @ h
+    assert 1e-3 <= np.linalg.norm(got - exact) / np.linalg.norm(exact) <= 0.15
+    np.testing.assert_array_equal(oracle.fp8_weight_grad(dy * 2.0 ** 12, h), got * 2.0 ** 12)
+    np.testing.assert_array_equal(oracle.fp8_weight_grad(dy, h * 2.0 ** -7), got * 2.0 ** -7)
+
+
+def test_column_tiles_are_independent_of_other_columns():
+    """Each (column, 128-row tile) has its own scale: changing one column
+    changes no other column's codes or scales."""
+    rng = np.random.default_rng(9)
+    m = rng.normal(size=(200, 6))
+    q0, s0 = oracle.quant_cols_1x128(m)
+    m2 = m.copy()
+    m2[:, 3] *= 1000.0
+    q1, s1 = oracle.quant_cols_1x128(m2)
+    keep = [0, 1, 2, 4, 5]
+    np.testing.assert_array_equal(q0[:, keep], q1[:, keep])
+    np.testing.assert_array_equal(s0[:, keep], s1[:, keep])
