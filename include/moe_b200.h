@@ -266,6 +266,22 @@ int moe_expert_ffn_backward_dx_fp8(const moe_shape* shape, const void* x_perm,
                                    const void* dy_shared, void* dx_perm, void* dx_shared,
                                    void* ws_bwd, void* stream);
 
+/* moe_expert_ffn_backward_dw_fp8: FP8 weight gradients, E4M3 mode with
+ * f % 256 == 0, to be called after moe_expert_ffn_backward_dx_fp8 with the
+ * same ws_bwd (it reads the g, u and dg, du left there):
+ *   dW2_e = dY_e^T H_e,  dW13_e = [dg du]_e^T A_e  (packed like W13)
+ * with the gradient operand in E5M2 and the activation in E4M3, each column
+ * of each scaled per 128-row tile of the expert's rows ([P3]; [P1] §4.1),
+ * fp32 per-slice promotion, bf16 results.  A is the layer input x gathered
+ * through perm_tok (E4M3 mode keeps no bf16 copy of the dispatched rows).
+ *   perm_tok [T*K], offsets [N+1]   from moe_dispatch
+ *   x        [T, d] bf16;  dy_perm, dy_shared as at the _dx_fp8 call
+ *   dw13 [N+1, 2f, d], dw2 [N+1, d, f] bf16 out; an expert without rows gets zeros */
+int moe_expert_ffn_backward_dw_fp8(const moe_shape* shape, const int32_t* perm_tok,
+                                   const int32_t* offsets, const void* x, const void* dy_perm,
+                                   const void* dy_shared, void* dw13, void* dw2, void* ws_bwd,
+                                   void* stream);
+
 /* moe_expert_ffn_backward_dw: the weight gradients ([P1] §2.2 MLP_W), BF16
  * mode with f % 256 == 0, to be called after moe_expert_ffn_backward_dx with
  * the same ws_bwd (it reads the g, u and dg, du that call leaves there):

@@ -8,6 +8,7 @@ from ._lib import (  # noqa: F401
     backward_workspace_size, moe_expert_ffn_backward_dw, moe_expert_ffn_backward_dx,
     moe_transpose_weights, moe_combine_backward, moe_route_backward, moe_dispatch_backward,
     moe_quantize_rows_e5m2, moe_quantize_weights_transposed, moe_expert_ffn_backward_dx_fp8,
+    moe_expert_ffn_backward_dw_fp8,
     DTYPE_BF16, DTYPE_E4M3, DTYPE_FP32, MoEError, MoEShape, check_shape, lib, moe_bias_update,
     moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_expert_ffn, moe_expert_ffn_gathered,
     moe_forward, moe_pack_w13, moe_quantize_weights,

@@ -58,6 +58,7 @@ _SIGS = {
                                               ctypes.c_int64, _c_p]),
     "moe_quantize_weights_transposed": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
     "moe_expert_ffn_backward_dx_fp8": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 16),
+    "moe_expert_ffn_backward_dw_fp8": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(MoEShape)]),
     "moe_transpose_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 5),
     "moe_expert_ffn_backward_dx": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
@@ -262,6 +263,15 @@ def moe_expert_ffn_backward_dx_fp8(s, x_perm, x_perm_scales, offsets, x, w13, w1
           _ptr(offsets), _ptr(x), _ptr(w13), _ptr(w13_scales), _ptr(w13t), _ptr(w13t_scales),
           _ptr(w2t), _ptr(w2t_scales), _ptr(dy_perm), _ptr(dy_shared), _ptr(dx_perm),
           _ptr(dx_shared), _ptr(ws_bwd), _stream(stream))
+
+
+def moe_expert_ffn_backward_dw_fp8(s, perm_tok, offsets, x, dy_perm, dy_shared, dw13, dw2,
+                                   ws_bwd, stream=None):
+    _expect(dw13, torch.bfloat16, (s.N + 1) * 2 * s.f * s.d, "dw13")
+    _expect(dw2, torch.bfloat16, (s.N + 1) * s.d * s.f, "dw2")
+    _call("moe_expert_ffn_backward_dw_fp8", ctypes.byref(s), _ptr(perm_tok), _ptr(offsets),
+          _ptr(x), _ptr(dy_perm), _ptr(dy_shared), _ptr(dw13), _ptr(dw2), _ptr(ws_bwd),
+          _stream(stream))
 
 
 def moe_expert_ffn_backward_dw(s, x_perm, offsets, x, dy_perm, dy_shared, dw13, dw2, ws_bwd,

@@ -234,6 +234,20 @@ int moe_quantize_weights_transposed(const moe_shape* shape, const void* w13t, co
                                                         static_cast<cudaStream_t>(stream)));
 }
 
+int moe_expert_ffn_backward_dw_fp8(const moe_shape* shape, const int32_t* perm_tok,
+                                   const int32_t* offsets, const void* x, const void* dy_perm,
+                                   const void* dy_shared, void* dw13, void* dw2, void* ws_bwd,
+                                   void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_E4M3 || shape->f % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(perm_tok) || !ptr_ok(offsets) || !ptr_ok(x) || !ptr_ok(dy_perm) ||
+      !ptr_ok(dy_shared) || !ptr_ok(dw13) || !ptr_ok(dw2) || ws_check(shape, ws_bwd) != MOE_OK)
+    return MOE_ERR_ARG;
+  return launch_ffn_bwd_dw_e4m3(*shape, perm_tok, offsets, x, dy_perm, dy_shared, dw13, dw2,
+                                ws_bwd, static_cast<cudaStream_t>(stream));
+}
+
 int moe_expert_ffn_backward_dx_fp8(const moe_shape* shape, const void* x_perm,
                                    const float* x_perm_scales, const int32_t* offsets,
                                    const void* x, const void* w13, const float* w13_scales,

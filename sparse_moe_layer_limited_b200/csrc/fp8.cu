@@ -698,6 +698,36 @@ BwdLayoutFp8 bwd_layout_fp8(const moe_shape& s) {
   off = al(off + rows * twof);
   B.dgus = off;
   off = al(off + (twof / QB) * ld_rows * 4);
+  // weight-gradient pass
+  const size_t R = (size_t)wgrad_cols_fp8(s), KT = R / QB;
+  const size_t ld_d = (size_t)scale_ld(s.d), ld_f = (size_t)scale_ld(s.f);
+  const size_t ld_2f = (size_t)scale_ld((long long)twof);
+  B.colbase = off;
+  off = al(off + (size_t)(s.N + 2) * 4);
+  B.at = off;
+  off = al(off + (size_t)s.d * R * 2);
+  B.dyt = off;
+  off = al(off + (size_t)s.d * R * 2);
+  B.ht = off;
+  off = al(off + (size_t)s.f * R * 2);
+  B.dgut = off;
+  off = al(off + twof * R * 2);
+  B.atq = off;
+  off = al(off + (size_t)s.d * R);
+  B.dytq = off;
+  off = al(off + (size_t)s.d * R);
+  B.htq = off;
+  off = al(off + (size_t)s.f * R);
+  B.dgutq = off;
+  off = al(off + twof * R);
+  B.ats = off;
+  off = al(off + KT * ld_d * 4);
+  B.dyts = off;
+  off = al(off + KT * ld_d * 4);
+  B.hts = off;
+  off = al(off + KT * ld_f * 4);
+  B.dguts = off;
+  off = al(off + KT * ld_2f * 4);
   B.total = off;
   return B;
 }

@@ -1,0 +1,344 @@
+// FP8 weight gradients of the experts: E5M2 gradients against E4M3
+// activations (the 10100.com article on the V3 report, FP8 paragraph: E4M3
+// forward, E5M2 backward), each operand scaled per 128-row tile along the
+// contraction from its online max-abs (the mhpq.cn article §4.1 fine-grained
+// scaling, the tile laid along the contraction as in every FP8 product here).
+//
+// Per expert e (group N = the shared expert):
+//   dW2_e  [d, f]  = dY_e^T H_e        dW13_e [2f, d] = [dg du]_e^T A_e
+// Layout pass (gemm_wgrad.cu's transposes with 128-column padding, A gathered
+// from x through perm_tok), then each transposed operand [C, R] is quantised
+// per 1x128 tile of its rows, i.e. per 128 expert rows of one feature:
+// scales [R/128][C] block-major.  The GEMM is the K-grouped unit loop of the
+// bf16 weight-gradient kernel with the FP8 per-slice promotion of fp8.cu: a
+// unit is one 128 x 256 gradient tile of one expert, its K loop the expert's
+// column block in 128-row slices; every slice lands in one of two 256-column
+// TMEM buffers (tcgen05.mma kind::f8f6f4, E5M2 x E4M3, K=32 per MMA) and
+// sixteen epilogue warps (four per TMEM lane quadrant, 64 columns each) fold
+// it into fp32 register sums with the slice's scale product, a row scale
+// times a column scale.  The producer stages each slice's 128 row scales and
+// 256 column scales in a ring of shared-memory slots by TMA.
+// All waits are bounded (~2 s) and set the device status word on expiry.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int GBM = 128, GBN = 256, GBK = 128;  // gradient tile rows, columns; K slice
+constexpr int GStages = 4;
+constexpr int GABytes = GBM * GBK;              // 16 KB (one byte per element)
+constexpr int GBBytes = GBN * GBK;              // 32 KB
+constexpr int GStageBytes = GABytes + GBBytes;
+constexpr int GThreads = 576;                   // warp 0 TMA, warp 1 MMA, warps 2-17 epilogue
+constexpr int GEpiWarps = 16;
+constexpr int GScaleSlots = 8;
+constexpr int GScaleSlotBytes = (GBM + GBN) * 4;  // row scales, then column scales
+constexpr size_t GSmemBytes = 1024 + (size_t)GStages * GStageBytes +
+                              (size_t)GScaleSlots * GScaleSlotBytes + 512;
+static_assert(GSmemBytes <= 232448, "FP8 weight-gradient kernel exceeds the shared memory");
+constexpr uint64_t GTimeoutNs = 2000000000ull;
+
+struct alignas(64) Fp8WgradArgs {
+  CUtensorMap tmL;   // left codes [M_total, R] E5M2 (the gradient), box {128, 128}
+  CUtensorMap tmR;   // right codes [N_total, R] E4M3 (the activation), box {128, 256}
+  CUtensorMap tmSL;  // left scales [R/128, ld] fp32, box {128, 1}
+  CUtensorMap tmSR;  // right scales [R/128, ld] fp32, box {256, 1}
+  const int32_t* colbase;  // [G1 + 1] column block of each group, multiples of 128
+  __nv_bfloat16* out;      // [G1, M_total, N_total]
+  uint32_t* status;
+  int G1, M_total, N_total;
+};
+
+__global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
+    const __grid_constant__ Fp8WgradArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* sc_ring = reinterpret_cast<float*>(base + (size_t)GStages * GStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)GStages * GStageBytes +
+                                               (size_t)GScaleSlots * GScaleSlotBytes);
+  uint64_t* full = bars;                       // [GStages]
+  uint64_t* empty = full + GStages;            // [GStages]
+  uint64_t* sfull = empty + GStages;           // [2] slice buffer written
+  uint64_t* sempty = sfull + 2;                // [2] slice buffer drained (16 warps)
+  uint64_t* scfull = sempty + 2;               // [GScaleSlots] scale slot landed
+  uint64_t* scempty = scfull + GScaleSlots;    // [GScaleSlots] scale slot read (16 warps)
+  uint64_t* drain = scempty + GScaleSlots;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int MT = args.M_total / GBM, NT = args.N_total / GBN;
+  const int per_group = MT * NT;
+  const int total = args.G1 * per_group;
+
+  if (tid == 0) {
+    for (int s = 0; s < GStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sfull[a], 1);
+      mbar_init(&sempty[a], GEpiWarps);
+    }
+    for (int c = 0; c < GScaleSlots; ++c) {
+      mbar_init(&scfull[c], 1);
+      mbar_init(&scempty[c], GEpiWarps);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 2 * GBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  // unit -> group g, row tile m, column tile n (n fastest); K slices of the
+  // group's column block
+  auto decode = [&](int u, int& g, int& m, int& n, int& kb0, int& kcnt) {
+    g = u / per_group;
+    const int local = u - g * per_group;
+    m = local / NT;
+    n = local - m * NT;
+    kb0 = args.colbase[g] / GBK;
+    kcnt = (args.colbase[g + 1] - args.colbase[g]) / GBK;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&args.tmL);
+      tma_prefetch_desc(&args.tmR);
+      tma_prefetch_desc(&args.tmSL);
+      tma_prefetch_desc(&args.tmSR);
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      uint32_t sslice = 0, sc_issued = 0, sc_parity = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        int g, m, n, kb0, kcnt;
+        decode(u, g, m, n, kb0, kcnt);
+        for (int kb = 0; kb < kcnt; ++kb, ++sslice) {
+          const uint32_t cs = sslice % GScaleSlots, cph = (sslice / GScaleSlots) & 1u;
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, GTimeoutNs) ||
+              !mbar_wait_bounded(&scempty[cs], cph ^ 1u, args.status, GTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = base + (size_t)stage * GStageBytes;
+          const int k = (kb0 + kb) * GBK;
+          mbar_arrive_expect_tx(&full[stage], GStageBytes);
+          tma_load_2d(sa, &args.tmL, k, m * GBM, &full[stage]);
+          tma_load_2d(sa + GABytes, &args.tmR, k, n * GBN, &full[stage]);
+          float* slot = sc_ring + cs * (GScaleSlotBytes / 4);
+          mbar_arrive_expect_tx(&scfull[cs], GScaleSlotBytes);
+          tma_load_2d(slot, &args.tmSL, m * GBM, kb0 + kb, &scfull[cs]);
+          tma_load_2d(slot + GBM, &args.tmSR, n * GBN, kb0 + kb, &scfull[cs]);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          sc_issued |= 1u << cs;
+          sc_parity = (sc_parity & ~(1u << cs)) | (cph << cs);
+          if (++stage == GStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {  // the copies already issued complete on these barriers
+        for (int s = 0; s < GStages; ++s)
+          if ((issued >> s) & 1u)
+            mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.status, GTimeoutNs / 8);
+        for (int c = 0; c < GScaleSlots; ++c)
+          if ((sc_issued >> c) & 1u)
+            mbar_wait_bounded(&scfull[c], (sc_parity >> c) & 1u, args.status, GTimeoutNs / 8);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f8_f32(GBM, GBN, kF8E5M2, kF8E4M3);
+      int stage = 0;
+      uint32_t phase = 0, slice = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        int g, m, n, kb0, kcnt;
+        decode(u, g, m, n, kb0, kcnt);
+        for (int kb = 0; kb < kcnt; ++kb, ++slice) {
+          const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
+          if (!mbar_wait_bounded(&sempty[sb], sph ^ 1u, args.status, GTimeoutNs) ||
+              !mbar_wait_bounded(&full[stage], phase, args.status, GTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(base + (size_t)stage * GStageBytes);
+          const uint32_t b0 = a0 + GABytes;
+#pragma unroll
+          for (int k = 0; k < GBK / 32; ++k)
+            mma_e4m3(tmem_base + sb * GBN, smem_desc_sw128(a0 + k * 32),
+                     smem_desc_sw128(b0 + k * 32), idesc, k != 0);
+          mma_commit(&empty[stage]);
+          mma_commit(&sfull[sb]);
+          if (++stage == GStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0, args.status, GTimeoutNs / 8);
+    }
+  } else {
+    // warps 2..17: warp w reads TMEM lanes 32*(w%4)..+31; the four warps of a
+    // quadrant own the 64 columns 64*sub.. of the tile
+    const int q = warp & 3;
+    const int sub = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    uint32_t slice = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int g, m, n, kb0, kcnt;
+      decode(u, g, m, n, kb0, kcnt);
+      float acc[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      for (int kb = 0; kb < kcnt; ++kb, ++slice) {
+        const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
+        const uint32_t cs = slice % GScaleSlots, cph = (slice / GScaleSlots) & 1u;
+        if (!mbar_wait_bounded(&scfull[cs], cph, args.status, GTimeoutNs) ||
+            !mbar_wait_bounded(&sfull[sb], sph, args.status, GTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float* slot = sc_ring + cs * (GScaleSlotBytes / 4);
+        const float s_row = slot[row];
+        const float* s_col = slot + GBM + 64 * sub;
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * GBN + 64 * sub;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t p[16];
+          tmem_ld16(taddr + 16 * c, p);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            acc[16 * c + i] = fmaf(__uint_as_float(p[i]), s_row * s_col[16 * c + i],
+                                   acc[16 * c + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sempty[sb]);
+          mbar_arrive(&scempty[cs]);
+        }
+      }
+      if (!ok) break;
+      // an expert without rows stores zeros
+      __nv_bfloat16* orow = args.out +
+                            ((size_t)g * args.M_total + (size_t)m * GBM + row) * args.N_total +
+                            (size_t)n * GBN + 64 * sub;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        uint4 w;
+        __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          hb[i] = __floats2bfloat162_rn(acc[8 * v + 2 * i], acc[8 * v + 2 * i + 1]);
+        reinterpret_cast<uint4*>(orow)[v] = w;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * GBN);
+  }
+}
+
+cudaError_t launch_fp8_wgrad(const Fp8WgradArgs& a, cudaStream_t st) {
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(fp8_wgrad_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)GSmemBytes),
+                            "fp8 weight-gradient GEMM: set shared-memory size");
+  if (e != cudaSuccess) return e;
+  fp8_wgrad_kernel<<<num_sms(), GThreads, GSmemBytes, st>>>(a);
+  return note_cuda(cudaGetLastError(), "fp8 weight-gradient GEMM launch");
+}
+
+}  // namespace
+
+// Columns of the FP8 transposed layouts: all rows plus up to 127 of padding
+// per group (blocks padded to one 128-row scale tile).
+long long wgrad_cols_fp8(const moe_shape& s) {
+  const long long rows = (long long)s.T * s.K + s.T;
+  return (rows + (long long)(s.N + 1) * 127 + 127) / 128 * 128;
+}
+
+int launch_ffn_bwd_dw_e4m3(const moe_shape& s, const int32_t* perm_tok, const int32_t* offsets,
+                           const void* x, const void* dy_perm, const void* dy_shared, void* dw13,
+                           void* dw2, void* ws_bwd, cudaStream_t st) {
+  const BwdLayoutFp8 B = bwd_layout_fp8(s);
+  uint8_t* w = static_cast<uint8_t*>(ws_bwd);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w);
+  const __nv_bfloat16* GU = reinterpret_cast<const __nv_bfloat16*>(w + B.gu);
+  const __nv_bfloat16* dGU = reinterpret_cast<const __nv_bfloat16*>(w + B.dgu);
+  int32_t* colbase = reinterpret_cast<int32_t*>(w + B.colbase);
+  auto bfp = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(w + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(w + off); };
+  const long long R = wgrad_cols_fp8(s);
+  const int twof = 2 * s.f;
+  // A: the layer input rows, gathered from x through perm_tok (E4M3 mode keeps
+  // no bf16 copy of the dispatched rows)
+  if (launch_group_transposes(s, GBK, x, perm_tok, x, dy_perm, dy_shared, GU, dGU, offsets,
+                              colbase, R, bfp(B.at), bfp(B.dyt), bfp(B.ht), bfp(B.dgut),
+                              st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // each transposed operand [C, R] per 1x128 tile of its rows
+  const long long ld_d = scale_ld(s.d), ld_f = scale_ld(s.f), ld_2f = scale_ld(twof);
+  if (launch_quant_rows_e5m2(bfp(B.dyt), s.d, (int)R, w + B.dytq, f32(B.dyts), ld_d, st) !=
+          cudaSuccess ||
+      launch_quant_rows(bfp(B.ht), s.f, (int)R, w + B.htq, f32(B.hts), ld_f, st) !=
+          cudaSuccess ||
+      launch_quant_rows_e5m2(bfp(B.dgut), twof, (int)R, w + B.dgutq, f32(B.dguts), ld_2f, st) !=
+          cudaSuccess ||
+      launch_quant_rows(bfp(B.at), s.d, (int)R, w + B.atq, f32(B.ats), ld_d, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint64_t KT = (uint64_t)(R / GBK);
+  // dW2_e [d, f] = dYT_e HT_e^T
+  Fp8WgradArgs a2{};
+  bool ok = make_map(&a2.tmL, w + B.dytq, U8, 1, R, s.d, GBK, GBM) &&
+            make_map(&a2.tmR, w + B.htq, U8, 1, R, s.f, GBK, GBN) &&
+            make_map_f32_rows(&a2.tmSL, f32(B.dyts), ld_d, KT, GBM) &&
+            make_map_f32_rows(&a2.tmSR, f32(B.hts), ld_f, KT, GBN);
+  // dW13_e [2f, d] = dGUT_e AT_e^T (rows in the packed W13 order)
+  Fp8WgradArgs a13{};
+  ok = ok && make_map(&a13.tmL, w + B.dgutq, U8, 1, R, twof, GBK, GBM) &&
+       make_map(&a13.tmR, w + B.atq, U8, 1, R, s.d, GBK, GBN) &&
+       make_map_f32_rows(&a13.tmSL, f32(B.dguts), ld_2f, KT, GBM) &&
+       make_map_f32_rows(&a13.tmSR, f32(B.ats), ld_d, KT, GBN);
+  if (!ok) {
+    note_text("fp8 weight-gradient GEMM: tensor-map encoding failed");
+    return MOE_ERR_CUDA;
+  }
+  a2.colbase = a13.colbase = colbase;
+  a2.status = a13.status = status;
+  a2.G1 = a13.G1 = s.N + 1;
+  a2.out = static_cast<__nv_bfloat16*>(dw2);
+  a2.M_total = s.d;
+  a2.N_total = s.f;
+  a13.out = static_cast<__nv_bfloat16*>(dw13);
+  a13.M_total = twof;
+  a13.N_total = s.d;
+  if (launch_fp8_wgrad(a2, st) != cudaSuccess || launch_fp8_wgrad(a13, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -44,8 +44,8 @@ constexpr uint64_t WTimeoutNs = 2000000000ull;
 
 // ---- layout: column blocks per group --------------------------------------------
 
-// colbase[g] = sum over g' < g of round_up(rows_g', 64); colbase[N+1] = R.
-__global__ void colbase_kernel(const int32_t* __restrict__ offsets, int N, int T,
+// colbase[g] = sum over g' < g of round_up(rows_g', pad); colbase[N+1] = R.
+__global__ void colbase_kernel(const int32_t* __restrict__ offsets, int N, int T, int pad,
                                int32_t* __restrict__ colbase) {
   const int lane = threadIdx.x;
   const int G1 = N + 1;
@@ -53,7 +53,7 @@ __global__ void colbase_kernel(const int32_t* __restrict__ offsets, int N, int T
   const int g0 = min(G1, lane * per), g1 = min(G1, g0 + per);
   auto padded = [&](int g) {
     const int rows = (g < N) ? offsets[g + 1] - offsets[g] : T;
-    return (max(rows, 0) + WBK - 1) / WBK * WBK;
+    return (max(rows, 0) + pad - 1) / pad * pad;
   };
   int sum = 0;
   for (int g = g0; g < g1; ++g) sum += padded(g);
@@ -72,17 +72,20 @@ __global__ void colbase_kernel(const int32_t* __restrict__ offsets, int N, int T
 }
 
 // Rows [rows, C] (dispatched rows from `routed`, then the shared expert's
-// from `shared`) -> dst [C, R]: group g's rows go, in order, to its columns
+// from `shared`; with `perm_tok`, dispatched row r is row perm_tok[r] of
+// `routed`) -> dst [C, R]: group g's rows go, in order, to its columns
 // colbase[g] .. colbase[g] + rows_g - 1, and its padding columns up to
 // colbase[g + 1] get zeros.  One 64 x 64 tile per CTA (tile_transpose.cuh);
-// the colbase values are multiples of 64, so a column tile lies in one group.
+// the colbase values are multiples of 64 (the padding is 64 or 128), so a
+// column tile lies in one group.
 // kSwiGLUH: the source holds the packed gate/up products [rows, 2f] and the
 // value moved is h = silu(g) * u of feature c (C = f), rounded to bf16.
 template <bool kSwiGLUH>
 __global__ void __launch_bounds__(kTileThreads) transpose_groups_kernel(
     const __nv_bfloat16* __restrict__ routed, const __nv_bfloat16* __restrict__ shared, int TK,
     int T, int N, int C, int src_ld, const int32_t* __restrict__ offsets,
-    const int32_t* __restrict__ colbase, long long ld, __nv_bfloat16* __restrict__ dst) {
+    const int32_t* __restrict__ perm_tok, const int32_t* __restrict__ colbase, long long ld,
+    __nv_bfloat16* __restrict__ dst) {
   __shared__ alignas(16) uint8_t sm[kTileBytes];
   __shared__ int s_group;
   const long long col0 = (long long)blockIdx.y * kTile;
@@ -107,9 +110,11 @@ __global__ void __launch_bounds__(kTileThreads) transpose_groups_kernel(
     const int i = it >> 3, p = it & 7;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     const long long r = first + local0 + i;
-    if (local0 + i < count && r >= 0 && r < limit && f0 + p * 8 + 8 <= C) {
+    const long long src = (perm_tok != nullptr && r >= 0 && r < TK) ? perm_tok[r] : r;
+    const bool src_ok = perm_tok == nullptr || r >= TK || (src >= 0 && src < T);
+    if (local0 + i < count && r >= 0 && r < limit && src_ok && f0 + p * 8 + 8 <= C) {
       const __nv_bfloat16* row =
-          r < TK ? routed + (size_t)r * src_ld : shared + (size_t)(r - TK) * src_ld;
+          r < TK ? routed + (size_t)src * src_ld : shared + (size_t)(r - TK) * src_ld;
       if constexpr (kSwiGLUH) {
         const int col = (f0 / 128) * 256 + (f0 % 128) + p * 8;
         float gt[8], up[8];
@@ -599,6 +604,36 @@ long long wgrad_cols(const moe_shape& s) {
   return (rows + (long long)(s.N + 1) * (WBK - 1) + WBK - 1) / WBK * WBK;
 }
 
+// The activations of every product laid out transposed in per-group column
+// blocks padded to `pad` (64 for the bf16 MMA's K step, 128 for an FP8 scale
+// tile): AT = [A; x]^T (A the dispatched rows, or x gathered through
+// perm_tok), dYT = [dy_perm; dy_shared]^T, HT from the stored g, u, and
+// dGUT = dGU^T.  colbase [N+2] receives the blocks' first columns.
+cudaError_t launch_group_transposes(const moe_shape& s, int pad, const void* a_routed,
+                                    const int32_t* a_perm, const void* x, const void* dy_perm,
+                                    const void* dy_shared, const __nv_bfloat16* GU,
+                                    const __nv_bfloat16* dGU, const int32_t* offsets,
+                                    int32_t* colbase, long long R, __nv_bfloat16* AT,
+                                    __nv_bfloat16* dYT, __nv_bfloat16* HT, __nv_bfloat16* dGUT,
+                                    cudaStream_t st) {
+  const int TK = s.T * s.K;
+  const int twof = 2 * s.f;
+  const auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
+  colbase_kernel<<<1, 32, 0, st>>>(offsets, s.N, s.T, pad, colbase);
+  const unsigned col_tiles = (unsigned)(R / kTile);
+  auto layout = [&](auto kernel, const __nv_bfloat16* routed, const int32_t* perm,
+                    const __nv_bfloat16* shared, int C, int src_ld, __nv_bfloat16* dst) {
+    kernel<<<dim3(C / kTile, col_tiles), kTileThreads, 0, st>>>(
+        routed, shared, TK, s.T, s.N, C, src_ld, offsets, perm, colbase, R, dst);
+  };
+  layout(transpose_groups_kernel<false>, bf(a_routed), a_perm, bf(x), s.d, s.d, AT);
+  layout(transpose_groups_kernel<false>, bf(dy_perm), nullptr, bf(dy_shared), s.d, s.d, dYT);
+  layout(transpose_groups_kernel<true>, GU, nullptr, GU + (size_t)TK * twof, s.f, twof, HT);
+  layout(transpose_groups_kernel<false>, dGU, nullptr, dGU + (size_t)TK * twof, twof, twof,
+         dGUT);
+  return note_cuda(cudaGetLastError(), "weight-gradient layout kernels");
+}
+
 int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                            const void* x, const void* dy_perm, const void* dy_shared,
                            void* dw13, void* dw2, void* ws_bwd, cudaStream_t st) {
@@ -612,24 +647,10 @@ int launch_ffn_bwd_dw_bf16(const moe_shape& s, const void* x_perm, const int32_t
   __nv_bfloat16* dYT = reinterpret_cast<__nv_bfloat16*>(w + B.dyt);
   __nv_bfloat16* HT = reinterpret_cast<__nv_bfloat16*>(w + B.ht);
   __nv_bfloat16* dGUT = reinterpret_cast<__nv_bfloat16*>(w + B.dgut);
-  const int TK = s.T * s.K;
   const long long R = wgrad_cols(s);
   const int twof = 2 * s.f;
-  const auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
-
-  colbase_kernel<<<1, 32, 0, st>>>(offsets, s.N, s.T, colbase);
-  // AT = [x_perm; x]^T, dYT = [dy_perm; dy_shared]^T, HT from GU, dGUT = dGU^T
-  const unsigned col_tiles = (unsigned)(R / kTile);
-  auto layout = [&](auto kernel, const __nv_bfloat16* routed, const __nv_bfloat16* shared, int C,
-                    int src_ld, __nv_bfloat16* dst) {
-    kernel<<<dim3(C / kTile, col_tiles), kTileThreads, 0, st>>>(routed, shared, TK, s.T, s.N, C,
-                                                                src_ld, offsets, colbase, R, dst);
-  };
-  layout(transpose_groups_kernel<false>, bf(x_perm), bf(x), s.d, s.d, AT);
-  layout(transpose_groups_kernel<false>, bf(dy_perm), bf(dy_shared), s.d, s.d, dYT);
-  layout(transpose_groups_kernel<true>, GU, GU + (size_t)TK * twof, s.f, twof, HT);
-  layout(transpose_groups_kernel<false>, dGU, dGU + (size_t)TK * twof, twof, twof, dGUT);
-  if (note_cuda(cudaGetLastError(), "weight-gradient layout kernels") != cudaSuccess)
+  if (launch_group_transposes(s, WBK, x_perm, nullptr, x, dy_perm, dy_shared, GU, dGU, offsets,
+                              colbase, R, AT, dYT, HT, dGUT, st) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

@@ -1,5 +1,6 @@
 // Internal declarations shared by the kernel files and the C-ABI layer.
 #pragma once
+#include <cuda_bf16.h>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -105,8 +106,16 @@ struct BwdLayout {
 // their block-major 1x128 scales.
 struct BwdLayoutFp8 {
   size_t gu = 0, dgu = 0, xq = 0, xs = 0, dyq = 0, dys = 0, dguq = 0, dgus = 0;
+  // weight-gradient pass: column blocks, the transposed operands (bf16), their
+  // codes (per 1x128 tile of each row) and block-major scales [R/128][C]
+  size_t colbase = 0, at = 0, dyt = 0, ht = 0, dgut = 0;
+  size_t atq = 0, dytq = 0, htq = 0, dgutq = 0, ats = 0, dyts = 0, hts = 0, dguts = 0;
   size_t total = 0;
 };
+long long wgrad_cols_fp8(const moe_shape& s);
+int launch_ffn_bwd_dw_e4m3(const moe_shape& s, const int32_t* perm_tok, const int32_t* offsets,
+                           const void* x, const void* dy_perm, const void* dy_shared, void* dw13,
+                           void* dw2, void* ws_bwd, cudaStream_t st);
 BwdLayoutFp8 bwd_layout_fp8(const moe_shape& s);
 int launch_ffn_bwd_dx_e4m3(const moe_shape& s, const void* x_perm, const float* x_perm_scales,
                            const int32_t* offsets, const void* x, const void* w13q,
@@ -117,6 +126,13 @@ int launch_ffn_bwd_dx_e4m3(const moe_shape& s, const void* x_perm, const float* 
 cudaError_t launch_quantize_weights_transposed(const moe_shape& s, const void* w13t,
                                                const void* w2t, void* w13t_q, float* w13t_scales,
                                                void* w2t_q, float* w2t_scales, cudaStream_t st);
+cudaError_t launch_group_transposes(const moe_shape& s, int pad, const void* a_routed,
+                                    const int32_t* a_perm, const void* x, const void* dy_perm,
+                                    const void* dy_shared, const __nv_bfloat16* GU,
+                                    const __nv_bfloat16* dGU, const int32_t* offsets,
+                                    int32_t* colbase, long long R, __nv_bfloat16* AT,
+                                    __nv_bfloat16* dYT, __nv_bfloat16* HT, __nv_bfloat16* dGUT,
+                                    cudaStream_t st);
 long long wgrad_cols(const moe_shape& s);
 BwdLayout bwd_layout(const moe_shape& s);
 size_t backward_ws_bytes(const moe_shape& s);

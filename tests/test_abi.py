@@ -147,3 +147,12 @@ def test_fp8_backward_entry_points_reject_bad_arguments_before_any_launch(L):
     assert f.moe_transpose_weights(fp32, ok, ok, ok, ok, None) == L.ERR_UNSUPPORTED
     assert f.moe_transpose_weights(e4m3, None, ok, ok, ok, None) == L.ERR_ARG
     assert f.moe_backward_workspace_size(e4m3) > 0
+
+
+def test_fp8_weight_gradient_entry_point_rejects_bad_arguments(L):
+    f = L.lib()
+    ok = ctypes.c_void_p(0x1000)
+    e4m3 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 256, L.DTYPE_E4M3))
+    bf16 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 256, L.DTYPE_BF16))
+    assert f.moe_expert_ffn_backward_dw_fp8(bf16, *([ok] * 8), None) == L.ERR_UNSUPPORTED
+    assert f.moe_expert_ffn_backward_dw_fp8(e4m3, *([None] * 8), None) == L.ERR_ARG
