@@ -165,13 +165,21 @@ def fp8_gemm_ref(codes_a, sa, codes_b, sb, a_format: str = "e4m3",
     return out
 
 
-def fp8_swiglu_expert(a, w1, w3, w2) -> np.ndarray:
+def fp8_swiglu_expert(a, w1, w3, w2, quant: bool = True) -> np.ndarray:
     """One SwiGLU expert with all three GEMMs in block-scaled E4M3 ([P1] §4.1):
     the rows ``a`` (bf16 values) are quantised per 1x128 tile along d, W1, W3
-    ([f, d]) and W2 ([d, f]) per 128x128 block; the hidden activation
+    ([f, d]) and W2 ([d, f]) per 128x128 block; the gate product a W1^T goes
+    through silu and multiplies the up product a W3^T; the hidden activation
     h = silu(a W1^T) * (a W3^T) is held in float32 (the accumulation
-    precision the pages name) and quantised per 1x128 tile along f before W2."""
+    precision the pages name) and quantised per 1x128 tile along f (each of
+    its rows separately) before W2.  ``quant=False`` skips every quantisation
+    and the float32 holding of h: the same steps then give the exact float64
+    expert."""
     from .moe import silu
+    if not quant:
+        a = np.asarray(a, dtype=np.float64)
+        h = silu(a @ np.asarray(w1, np.float64).T) * (a @ np.asarray(w3, np.float64).T)
+        return h @ np.asarray(w2, np.float64).T
     qa, sa = quant_rows_1x128(a)
     q1, s1 = quant_blocks_128(w1)
     q3, s3 = quant_blocks_128(w3)

@@ -216,3 +216,74 @@ def test_the_unmodified_oracle_passes_the_same_pins():
     for _, _, ps in CASES:
         pins.update(ps)
     assert not _fails(list(pins))
+
+
+# ---- FP8 forward expert: four plausible composition mistakes ----------------------------
+
+from tests import test_oracle_fp8_expert as PFX  # noqa: E402
+
+ORIG_FP8_FWD = oracle.fp8.fp8_swiglu_expert
+
+
+def fp8_gate_and_up_swapped(a, w1, w3, w2, quant=True):
+    return ORIG_FP8_FWD(a, w3, w1, w2, quant)
+
+
+def _fp8_expert_with(a, w1, w3, w2, h_quant, w2_scales=lambda s: s):
+    F = oracle.fp8
+    qa, sa = F.quant_rows_1x128(a)
+    q1, s1 = F.quant_blocks_128(w1)
+    q3, s3 = F.quant_blocks_128(w3)
+    q2, s2 = F.quant_blocks_128(w2)
+    h = oracle.moe.silu(F.fp8_gemm_ref(qa, sa, q1, s1)) * F.fp8_gemm_ref(qa, sa, q3, s3)
+    return h_quant(h.astype(np.float32), q2, w2_scales(s2))
+
+
+def fp8_h_not_quantised(a, w1, w3, w2, quant=True):
+    if not quant:
+        return ORIG_FP8_FWD(a, w1, w3, w2, quant)
+    def keep_h(h, q2, s2):
+        W2 = oracle.fp8.e4m3_decode(q2) * np.kron(s2.astype(np.float64), np.ones((128, 128)))
+        return h.astype(np.float64) @ W2.T
+    return _fp8_expert_with(a, w1, w3, w2, keep_h)
+
+
+def fp8_h_quantised_per_column(a, w1, w3, w2, quant=True):
+    if not quant:
+        return ORIG_FP8_FWD(a, w1, w3, w2, quant)
+    def h_by_columns(h, q2, s2):
+        qh, sh = oracle.fp8.quant_cols_1x128(h)                     # 128-row tiles along M
+        H = oracle.fp8.e4m3_decode(qh) * np.repeat(sh.astype(np.float64), 128, axis=0)[:h.shape[0]]
+        W2 = oracle.fp8.e4m3_decode(q2) * np.kron(s2.astype(np.float64), np.ones((128, 128)))
+        return H @ W2.T
+    return _fp8_expert_with(a, w1, w3, w2, h_by_columns)
+
+
+def fp8_w2_scales_transposed(a, w1, w3, w2, quant=True):
+    if not quant:
+        return ORIG_FP8_FWD(a, w1, w3, w2, quant)
+    def rows(h, q2, s2):
+        qh, sh = oracle.fp8.quant_rows_1x128(h)
+        return oracle.fp8.fp8_gemm_ref(qh, sh, q2, s2)
+    # W2 is [d, f]: its scale grid is [d/128, f/128]; read it the other way round
+    return _fp8_expert_with(a, w1, w3, w2, rows,
+                            lambda s: np.ascontiguousarray(s.T).reshape(s.shape))
+
+
+FP8_FWD_PINS = [lambda: PFX.test_without_quantisation_it_is_the_exact_expert(0),
+                PFX.test_lossless_operands_leave_the_1x128_quantisation_of_h_along_f,
+                lambda: PFX.test_error_stays_within_e4m3_precision(2),
+                PFX.test_rows_are_independent,
+                PFX.test_equals_swiglu_of_the_dequantised_operands]
+
+
+@pytest.mark.parametrize("mutant", [fp8_gate_and_up_swapped, fp8_h_not_quantised,
+                                    fp8_h_quantised_per_column, fp8_w2_scales_transposed])
+def test_planted_fp8_forward_mistake_is_caught(monkeypatch, mutant):
+    monkeypatch.setattr(oracle.fp8, "fp8_swiglu_expert", mutant)
+    monkeypatch.setattr(oracle, "fp8_swiglu_expert", mutant)
+    assert _fails(FP8_FWD_PINS), f"no pin caught {mutant.__name__}"
+
+
+def test_the_unmodified_fp8_forward_passes_its_pins():
+    assert not _fails(FP8_FWD_PINS)
