@@ -385,12 +385,14 @@ int moe_quantize_weights(const moe_shape* shape, const void* w13_bf16, const voi
  * forbids new allocations, or a host application that hands the library only
  * its input and output buffers -- and so cannot provide a workspace.  The
  * pages describe no such entry point; it has no counterpart there.
- * Arguments, layouts and results are those of moe_dispatch, without `ws`.
- * Scratch: a fixed 1 MiB static device array inside the library (held on
- * every GPU that loads the library until the process exits).  The dispatch
- * tables need 256 + 2 * ceil(T/32) * N * 4 bytes (each table rounded up to
- * 256 bytes); a shape that needs more than 1 MiB (e.g. T > 16384 at N = 256)
- * returns MOE_ERR_WORKSPACE before anything is enqueued.  E4M3 mode returns
+ * Arguments, layouts and results are those of moe_dispatch, without `ws`;
+ * as there, x_perm may be NULL (offsets, perm_tok and slot only).
+ * Scratch: a fixed static device array of 1 MiB + 256 bytes inside the
+ * library (held on every GPU that loads the library until the process
+ * exits).  The dispatch needs a 256-byte status word plus two tables of
+ * ceil(T/32) * N * 4 bytes each (each rounded up to 256 bytes); a shape that
+ * needs more than the array (at N = 256: T > 16384) returns
+ * MOE_ERR_WORKSPACE before anything is enqueued.  E4M3 mode returns
  * MOE_ERR_UNSUPPORTED.
  * The first call on a device looks up the array's device address (with
  * that device current) and caches it; make that first call before any

@@ -23,18 +23,5 @@ def build(verbose: bool = False, extra=()) -> str:
     return LIB_PATH
 
 
-PROBE_PATH = os.path.join(HERE, "mma_rate")
-
-
-def build_probe(verbose: bool = False) -> str:
-    """The standalone tcgen05.mma issue-rate probe (csrc/probe/mma_rate.cu)."""
-    cmd = ["nvcc", "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
-           "-o", PROBE_PATH, os.path.join(HERE, "csrc", "probe", "mma_rate.cu")]
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
-    return PROBE_PATH
-
-
 if __name__ == "__main__":
     build(verbose=True)

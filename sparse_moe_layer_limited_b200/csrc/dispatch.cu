@@ -245,17 +245,18 @@ cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* id
 // over only its input and output buffers), moe_dispatch_noalloc keeps the
 // three scratch regions of the dispatch (status word, per-chunk histograms,
 // per-chunk bases) in one fixed static device array of this file instead of
-// the caller's workspace.  The array is kNoAllocScratchBytes long and lives
-// on every GPU that loads the library until the process exits; shapes that
-// need more are rejected.  Host code cannot pass the array's name to a
+// the caller's workspace.  The array is kNoAllocScratchBytes long (1 MiB of
+// tables plus the 256-byte status word, so T = 16384 fits at N = 256) and
+// lives on every GPU that loads the library until the process exits; shapes
+// that need more are rejected.  Host code cannot pass the array's name to a
 // kernel (on the host it is only a stand-in symbol), so its device address
 // is looked up with cudaGetSymbolAddress once per device, with that device
 // current, on the first call there.
 namespace moe {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;  // 1 MiB
 constexpr size_t kNoAllocStatusBytes = 256;
+constexpr size_t kNoAllocScratchBytes = ((size_t)1 << 20) + kNoAllocStatusBytes;
 constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_dispatch_scratch[kNoAllocScratchBytes];
@@ -296,8 +297,10 @@ extern "C" int moe_dispatch_noalloc(const moe_shape* shape, const void* x,
     return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
   };
   if (!ok16(x) || !ok16(topk_idx) || !ok16(counts) || !ok16(offsets) || !ok16(perm_tok) ||
-      !ok16(slot) || !ok16(x_perm))
+      !ok16(slot))
     return MOE_ERR_ARG;
+  // as in moe_dispatch, x_perm may be NULL: offsets, perm_tok and slot only
+  if (x_perm != nullptr && !ok16(x_perm)) return MOE_ERR_ARG;
   if (s.dtype == MOE_DTYPE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (noalloc_scratch_need(s) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
   (void)x_perm_scales;

@@ -20,7 +20,6 @@ def M():
     return M
 
 
-@pytest.mark.skip(reason="awaits its first run on a GPU")
 @pytest.mark.parametrize("T", [300, 1])
 def test_fp8_backward_dx_matches_oracle(M, T):
     import torch
@@ -87,7 +86,6 @@ def _packed(dg, du):
     return out
 
 
-@pytest.mark.skip(reason="awaits its first run on a GPU")
 def test_fp8_backward_dw_matches_oracle(M):
     """moe_expert_ffn_backward_dw_fp8 after the _dx_fp8 call: dW2 and the
     packed dW13 of every expert against oracle.fp8_weight_grad on the

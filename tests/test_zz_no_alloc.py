@@ -23,11 +23,12 @@ from tests import support as S
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     import sparse_moe_layer_limited_b200 as M
     f = M.lib()
-    big = M.shape(20000, 256, 256, 8, 8, 4, 256, M.DTYPE_BF16)   # needs > 1 MiB of tables
     fake = ctypes.c_void_p(1 << 20)                                # never dereferenced
-    rc = f.moe_dispatch_noalloc(ctypes.byref(big), fake, fake, fake, fake, fake, fake, fake,
-                                None, None)
-    assert rc == M._lib.ERR_WORKSPACE
+    for T in (20000, 16385):       # at N = 256 the array holds the tables of T <= 16384
+        big = M.shape(T, 256, 256, 8, 8, 4, 256, M.DTYPE_BF16)
+        rc = f.moe_dispatch_noalloc(ctypes.byref(big), fake, fake, fake, fake, fake, fake, fake,
+                                    None, None)
+        assert rc == M._lib.ERR_WORKSPACE, T
     ok = M.shape(1000, 256, 8, 2, 2, 1, 256, M.DTYPE_BF16)
     assert f.moe_dispatch_noalloc(ctypes.byref(ok), None, fake, fake, fake, fake, fake, fake,
                                   None, None) == M._lib.ERR_ARG
@@ -40,7 +41,7 @@ def _inputs(cfg):
     return x, r
 
 
-def _dispatch_both(M, cfg, x, r):
+def _dispatch_both(M, cfg, x, r, slots_only=False):
     import torch
     s = S.moe_shape(cfg)
     xd = S.to_dev_x(x, cfg)
@@ -52,15 +53,16 @@ def _dispatch_both(M, cfg, x, r):
         perm = torch.full((s.T * s.K,), -7, dtype=torch.int32, device="cuda")
         slot = torch.full((s.T, s.K), -7, dtype=torch.int32, device="cuda")
         xp = torch.zeros(s.T * s.K, s.d, dtype=xd.dtype, device="cuda")
+        xp_arg = None if slots_only else xp
         if which == "ws":
             ws = torch.zeros(M.workspace_size(s), dtype=torch.uint8, device="cuda")
-            M.moe_dispatch(s, xd, idx, counts, off, perm, slot, xp, None, ws)
+            M.moe_dispatch(s, xd, idx, counts, off, perm, slot, xp_arg, None, ws)
         else:
             rc = M.lib().moe_dispatch_noalloc(
                 ctypes.byref(s), ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(idx.data_ptr()),
                 ctypes.c_void_p(counts.data_ptr()), ctypes.c_void_p(off.data_ptr()),
                 ctypes.c_void_p(perm.data_ptr()), ctypes.c_void_p(slot.data_ptr()),
-                ctypes.c_void_p(xp.data_ptr()), None,
+                None if slots_only else ctypes.c_void_p(xp.data_ptr()), None,
                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
             assert rc == 0, M.status_string(rc)
         torch.cuda.synchronize()
@@ -84,3 +86,26 @@ def test_noalloc_matches_workspace_dispatch_twice():
         d = oracle.dispatch(r["idx"], cfg.N)
         np.testing.assert_array_equal(o2, d["offsets"])
         np.testing.assert_array_equal(p2, d["perm_tok"])
+
+
+@pytest.mark.gpu
+def test_noalloc_at_its_largest_shape_and_slots_only():
+    """T = 16384 at N = 256 is the largest shape the array holds (1 MiB of
+    tables); and with x_perm NULL only offsets, perm_tok and slot are written,
+    as with moe_dispatch."""
+    import sparse_moe_layer_limited_b200 as M
+    big = CONFIGS[1].with_(T=16384, d=256, N=256, K=8, G=8, topG=4, f=256)
+    small = CONFIGS[1].with_(T=300, d=256, N=16, K=4, G=4, topG=2, f=256)
+    for cfg, slots_only in ((big, False), (small, True)):
+        x, r = _inputs(cfg)
+        (o1, p1, s1, x1), (o2, p2, s2, x2) = _dispatch_both(M, cfg, x, r, slots_only)
+        np.testing.assert_array_equal(o2, o1)
+        np.testing.assert_array_equal(p2, p1)
+        np.testing.assert_array_equal(s2, s1)
+        np.testing.assert_array_equal(x2, x1)
+        d = oracle.dispatch(r["idx"], cfg.N)
+        np.testing.assert_array_equal(o2, d["offsets"])
+        np.testing.assert_array_equal(p2, d["perm_tok"])
+        np.testing.assert_array_equal(s2, d["slot"])
+        if slots_only:
+            assert not x2.any()            # the rows were not copied
