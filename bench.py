@@ -59,8 +59,10 @@ def peaks():
             p = json.load(fh)
         return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
                     bf16_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    sustained_mhz=p.get("clocks_under_load", {}).get("sm_mhz_median"),
                     source="measured")
-    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, sustained_mhz=1300.0,
+                source="fallback")
 
 
 def workload_name(cfg):
@@ -254,10 +256,11 @@ def main():
         extra["fp8"] = run_layer(BY_NAME["v3_fp8"], dev, max(5, args.steps // 5), 3, pg, local)
         extra["decode"] = run_layer(BY_NAME["decode_zipf"], dev, max(20, args.steps), 3, pg,
                                     local)
-    bwd = layer_bwd = None
+    bwd = layer_bwd = bwd_fp8 = None
     if not args.no_extra and cfg.dtype == "bf16" and world == 1:
         bwd = run_backward(cfg, dev)
         layer_bwd = run_layer_backward(cfg, dev)
+        bwd_fp8 = run_backward_fp8(BY_NAME["v3_fp8"], dev)
 
     if rank == 0:
         P = peaks()
@@ -299,6 +302,8 @@ def main():
             line["backward_dx"] = bwd
         if layer_bwd is not None:
             line["layer_backward"] = layer_bwd
+        if bwd_fp8 is not None:
+            line["backward_fp8"] = bwd_fp8
         if world == 1 and not args.no_cpu_baseline:
             v, cores, note = cpu_oracle_baseline(cfg, args.cpu_sample)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
@@ -460,6 +465,98 @@ def run_backward(cfg, dev, calls=10, warmup=3):
                     "epilogue, dx (3 launches); weight gradients beside them"}
 
 
+def run_backward_fp8(cfg, dev, calls=5, warmup=2):
+    """The FP8 expert backward on the layer's routing of one synthetic batch
+    (E4M3 weights and activations, E5M2 gradients): input gradients
+    (moe_expert_ffn_backward_dx_fp8: GEMM1 recomputed, dY quantised, dY W2^T
+    with the SwiGLU-backward epilogue, dGU quantised, dGU W13; 10*d*f FLOP per
+    dispatched or shared row) and weight gradients
+    (moe_expert_ffn_backward_dw_fp8: layout, four quantisations, dW2 and
+    dW13; 6*d*f FLOP per row).  dY is seeded N(0, 1) bf16.  CUDA events over
+    `calls` calls after `warmup`; peak = the measured bf16 burst rate x 2."""
+    import torch
+    import sparse_moe_layer_limited_b200 as M
+    from synth import device as sdev
+    s = M.shape(cfg.T, cfg.d, cfg.N, cfg.K, cfg.G, cfg.topG, cfg.f, M.DTYPE_E4M3)
+    E, d, f = cfg.N + 1, cfg.d, cfg.f
+    w1 = sdev.expert_weights_bf16(cfg, 0, "w1", dev)
+    w3 = sdev.expert_weights_bf16(cfg, 0, "w3", dev)
+    w13 = torch.empty(E, 2 * f, d, dtype=torch.bfloat16, device=dev)
+    M.moe_pack_w13(s, w1, w3, w13)
+    del w1, w3
+    w2 = sdev.expert_weights_bf16(cfg, 0, "w2", dev)
+    q = lambda *shape: torch.empty(*shape, dtype=torch.float8_e4m3fn, device=dev)  # noqa: E731
+    f32 = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)  # noqa: E731
+    w13q, w2q = q(E, 2 * f, d), q(E, d, f)
+    s13, s2 = f32(E, 2 * f // 128, d // 128), f32(E, d // 128, f // 128)
+    M.moe_quantize_weights(s, w13, w2, w13q, s13, w2q, s2)
+    w13t = torch.empty(E, d, 2 * f, dtype=torch.bfloat16, device=dev)
+    w2t = torch.empty(E, f, d, dtype=torch.bfloat16, device=dev)
+    M.moe_transpose_weights(s, w13, w2, w13t, w2t)
+    del w13, w2
+    w13tq, w2tq = q(E, d, 2 * f), q(E, f, d)
+    s13t, s2t = f32(E, d // 128, 2 * f // 128), f32(E, f // 128, d // 128)
+    M.moe_quantize_weights_transposed(s, w13t, w2t, w13tq, s13t, w2tq, s2t)
+    torch.cuda.synchronize()
+    del w13t, w2t
+    router = torch.from_numpy(gen.make_router(cfg)).to(dev)
+    bias = torch.from_numpy(gen.make_bias(cfg)).to(dev)
+    layer = M.MoELayer(s, router, bias, w13q, w2q, s13, s2, gamma=cfg.gamma)
+    x = sdev.x_bf16(cfg, 0, device=dev)
+    layer.forward(x, update_bias=False)
+    g = torch.Generator(device=dev).manual_seed(7)
+    dyp = torch.randn(cfg.T * cfg.K, d, generator=g, device=dev).to(torch.bfloat16)
+    dys = torch.randn(cfg.T, d, generator=g, device=dev).to(torch.bfloat16)
+    dxp, dxs = torch.empty_like(dyp), torch.empty_like(dys)
+    ws = torch.zeros(M.backward_workspace_size(s), dtype=torch.uint8, device=dev)
+    dw13 = torch.empty(E, 2 * f, d, dtype=torch.bfloat16, device=dev)
+    dw2 = torch.empty(E, d, f, dtype=torch.bfloat16, device=dev)
+
+    def call_dx():
+        M.moe_expert_ffn_backward_dx_fp8(s, layer.x_perm, layer.x_perm_scales, layer.offsets, x,
+                                         w13q, s13, w13tq, s13t, w2tq, s2t, dyp, dys, dxp, dxs,
+                                         ws)
+
+    def call_dw():
+        M.moe_expert_ffn_backward_dw_fp8(s, layer.perm_tok, layer.offsets, x, dyp, dys, dw13,
+                                         dw2, ws)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(calls):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / calls
+
+    ms = timed(call_dx)
+    call_dx()                # the weight pass reads what the input pass leaves in ws
+    ms_dw = timed(call_dw)
+    status = M.moe_read_device_status(ws)
+    rows = cfg.T * cfg.K + cfg.T
+    fl, fl_dw = 10.0 * d * f * rows, 6.0 * d * f * rows
+    P = peaks()
+    pk = 2.0 * P["bf16"]
+    a, a_dw = fl / (ms / 1e3) / 1e12, fl_dw / (ms_dw / 1e3) / 1e12
+    return {"workload": workload_name(cfg), "ms": ms, "tokens_per_s": cfg.T / (ms / 1e3),
+            "roofline": {"bound": "tensor", "achieved": a, "unit": "TFLOP/s", "peak": pk,
+                         "frac": a / pk, "peak_source": P["source"] + " bf16 burst x nominal "
+                         "fp8/bf16 ratio 2", "flops_per_call": fl},
+            "gpu_launches_per_call": 7, "device_status": status,
+            "weight_gradients": {"ms": ms_dw, "achieved": a_dw, "unit": "TFLOP/s",
+                                 "frac": a_dw / pk, "flops_per_call": fl_dw,
+                                 "gpu_launches_per_call": 11,
+                                 "note": "dW2 and dW13 of every expert (6 d f FLOP per row), "
+                                         "including the layout pass and the four 1x128 "
+                                         "quantisations"},
+            "note": "E4M3 operands, E5M2 gradients: input gradients (GEMM1 recomputed, dY "
+                    "quantised, dh with the SwiGLU-backward epilogue, dGU quantised, dx)"}
+
+
 def run_layer_backward(cfg, dev, calls=10, warmup=3):
     """The backward steps around the experts on the layer's routing of one
     synthetic batch (BF16): moe_combine_backward, moe_route_backward,
@@ -569,27 +666,36 @@ _READ_GBS = {}
 
 
 def hbm_read_stream_gbs(dev, gib=4, reps=10):
-    """Read-only HBM bandwidth: a float32 sum over a `gib` GiB bf16 buffer
-    (larger than L2), best of `reps` CUDA-event timings, bytes read / time."""
+    """Read-only HBM bandwidth over a `gib` GiB bf16 buffer (larger than L2):
+    the better of a float32 sum over it and a matrix-vector product that
+    streams it as a [rows, 8192] matrix, each best of `reps` CUDA-event
+    timings; bytes read / time."""
     import torch
     if dev in _READ_GBS:
         return _READ_GBS[dev]
     n = gib * (1 << 30) // 2
     buf = torch.ones(n, dtype=torch.bfloat16, device=dev)
-    for _ in range(3):
-        buf.sum(dtype=torch.float32)
-    torch.cuda.synchronize()
-    best = 1e30
-    for _ in range(reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        buf.sum(dtype=torch.float32)
-        e1.record()
+    mat = buf.view(-1, 8192)
+    vec = torch.ones(8192, dtype=torch.bfloat16, device=dev)
+
+    def best(fn):
+        for _ in range(3):
+            fn()
         torch.cuda.synchronize()
-        best = min(best, e0.elapsed_time(e1))
-    del buf
+        out = 1e30
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            out = min(out, e0.elapsed_time(e1))
+        return out
+
+    ms = min(best(lambda: buf.sum(dtype=torch.float32)), best(lambda: torch.mv(mat, vec)))
+    del buf, mat, vec
     torch.cuda.empty_cache()
-    _READ_GBS[dev] = 2.0 * n / (best / 1e3) / 1e9
+    _READ_GBS[dev] = 2.0 * n / (ms / 1e3) / 1e9
     return _READ_GBS[dev]
 
 
@@ -661,6 +767,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
     if pg is not None:
         pg.barrier()
+    M.moe_read_gemm_clock(layer.ws, clear=True)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for k in range(steps):
@@ -668,6 +775,9 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
         torch.cuda.synchronize()
     if pg is not None:
         pg.barrier()
+    # the SM clock the expert GEMMs themselves ran at (their first CTA's
+    # cycle and nanosecond counters over the timed steps)
+    gclk = M.moe_read_gemm_clock(layer.ws)
     per_phase = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps)]
                  for i, p in enumerate(phases)}
     total_ms = evs[0][0].elapsed_time(evs[-1][5])
@@ -701,12 +811,20 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
     by = used * 3 * cfg.d * cfg.f * wbytes + 2 * cfg.T * cfg.d * 2 + cfg.N * cfg.d * 4
     roof_ms = max(fl / (peak * 1e12), by / (P["hbm"] * 1e9)) * 1e3
     ms_step = total_ms / steps
+    kmhz = gclk["fp8_mhz"] if fp8 else gclk["bf16_mhz"]
     if cfg.zipf_s is None:
         achieved = ffn_flops(cfg) / (ffn_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": "moe_expert_ffn (grouped GEMM1+SwiGLU, GEMM2)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": peak_src, "peak_sustained": peak_sus,
-                "frac_of_sustained": achieved / peak_sus, "traffic": None}
+                "frac_of_sustained": achieved / peak_sus, "traffic": None,
+                "kernel_sm_mhz": kmhz}
+        if kmhz and P.get("sustained_mhz"):
+            # the measured cuBLAS rate per MHz (its sustained run and that run's
+            # median clock) at the clock these kernels ran at
+            at_clk = peak_sus * kmhz / P["sustained_mhz"]
+            roof["peak_at_kernel_clock"] = at_clk
+            roof["frac_at_kernel_clock"] = achieved / at_clk
         if cfg.name == "v3_bf16" and cfg.T == 8192 and cfg.N == 256 and not pair_gemm():
             # DRAM bytes of one moe_expert_ffn call (GEMM1 + GEMM2), from the ncu
             # capture of the same kernels on the T=1024 / 32+1-expert case
@@ -737,7 +855,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
                                 else P["source"] + " copy"),
                 "peak_copy": P["hbm"], "peak_read_stream": rd, "nominal_gbs": 7700.0,
                 "frac_of_nominal": achieved / 7700.0,
-                "traffic": None, "experts_hit": used - 1}
+                "traffic": None, "experts_hit": used - 1, "kernel_sm_mhz": kmhz}
     return {"cfg": cfg, "steps": steps, "total_ms": total_ms, "e2e_ms": e2e_ms,
             "softmax_route": baseline,
             "phases_ms": {p: statistics.mean(v) for p, v in per_phase.items()},

@@ -122,6 +122,15 @@ int moe_workspace_init(void* ws, void* stream);
  * was non-zero. */
 int moe_read_device_status(void* ws, void* stream, uint32_t* status_out, int clear);
 
+/* Measurement aid, not a step of the method: the expert GEMM kernels add,
+ * on every launch, the SM cycles and wall-clock nanoseconds of their first
+ * CTA (start to end) to counters in the workspace head (bytes 128..159).
+ * This synchronises `stream` and copies them into counters_out[4] =
+ * {bf16 cycles, bf16 ns, FP8 cycles, FP8 ns}; cycles / ns is the average SM
+ * clock, in GHz, over the launches since the last clear.  `clear` non-zero
+ * zeroes them afterwards.  MOE_ERR_ARG for a NULL pointer. */
+int moe_read_gemm_clock(void* ws, void* stream, uint64_t* counters_out, int clear);
+
 /* Routing: affinity, biased group-limited top-K, gates and per-expert counts.
  * [P4] sigmoid affinity and gate normalisation; [P2] Q3 / [P1] §1.2 bias for
  * selection only; [P1] §3.1 group limit; [P5] top-K by affinity.
@@ -365,6 +374,20 @@ int moe_quantize_rows_e5m2(const void* g, int64_t rows, int cols, uint8_t* codes
  * unchanged otherwise; fp32, in place. */
 int moe_bias_update(const moe_shape* shape, const int32_t* counts, float* bias, float gamma,
                     void* stream);
+
+/* moe_gather_rows: dst[i] = src[idx[i]] for i < n, whole rows of row_bytes
+ * bytes (any element type).  Expert parallelism ([P1] §2.1: each GPU holds a
+ * contiguous share of the routed experts; §3.1: tokens reach them by
+ * all-to-all) receives rows grouped by source GPU, then by expert; this
+ * regroups them by expert for the grouped expert GEMM, and puts the results
+ * back in arrival order.
+ *   src  [src_rows, row_bytes] device, 16-byte aligned
+ *   idx  [n] int32 device; an index outside [0, src_rows) writes a zero row
+ *   dst  [n, row_bytes] device, 16-byte aligned, must not overlap src
+ * row_bytes % 16 == 0.  MOE_ERR_ARG for a bad size or pointer; n = 0 is a
+ * no-op. */
+int moe_gather_rows(const void* src, int64_t src_rows, const int32_t* idx, int64_t n,
+                    int row_bytes, void* dst, void* stream);
 
 /* Weight preparation (not part of the timed forward).
  * moe_pack_w13: w1, w3 [N+1, f, d] -> w13 [N+1, 2f, d] in the 128-row block

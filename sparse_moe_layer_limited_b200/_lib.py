@@ -45,6 +45,8 @@ _SIGS = {
     "moe_workspace_init": (ctypes.c_int, [_c_p, _c_p]),
     "moe_read_device_status": (ctypes.c_int, [_c_p, _c_p, ctypes.POINTER(ctypes.c_uint32),
                                               ctypes.c_int]),
+    "moe_read_gemm_clock": (ctypes.c_int, [_c_p, _c_p, ctypes.POINTER(ctypes.c_uint64),
+                                           ctypes.c_int]),
     "moe_route": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 8),
     "moe_route_softmax": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 8),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 10),
@@ -66,6 +68,8 @@ _SIGS = {
     "moe_dispatch_noalloc": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, ctypes.c_float,
                                        _c_p]),
+    "moe_gather_rows": (ctypes.c_int, [_c_p, ctypes.c_int64, _c_p, ctypes.c_int64, ctypes.c_int,
+                                       _c_p, _c_p]),
     "moe_pack_w13": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 4),
     "moe_quantize_weights": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
     "moe_forward": (ctypes.c_int, [ctypes.POINTER(MoEShape), _c_p, _c_p, _c_p, ctypes.c_float]
@@ -146,6 +150,17 @@ def w_torch_dtype(s: MoEShape):
 
 def moe_workspace_init(ws, stream=None):
     _call("moe_workspace_init", _ptr(ws), _stream(stream))
+
+
+def moe_read_gemm_clock(ws, stream=None, clear=False) -> dict:
+    """Average SM clock (MHz) of the bf16 and FP8 expert GEMM launches since
+    the last clear, from the kernels' own cycle and nanosecond counters
+    (None where no launch was recorded)."""
+    c = (ctypes.c_uint64 * 4)()
+    _call("moe_read_gemm_clock", _ptr(ws), _stream(stream), c, int(clear))
+    mhz = lambda cyc, ns: (1e3 * cyc / ns) if ns else None  # noqa: E731
+    return {"bf16_mhz": mhz(c[0], c[1]), "fp8_mhz": mhz(c[2], c[3]), "bf16_ns": c[1],
+            "fp8_ns": c[3]}
 
 
 def moe_read_device_status(ws, stream=None, clear=False) -> int:
@@ -328,6 +343,16 @@ def moe_bias_update(s, counts, bias, gamma, stream=None):
     _expect(bias, torch.float32, s.N, "bias")
     _call("moe_bias_update", ctypes.byref(s), _ptr(counts), _ptr(bias), ctypes.c_float(gamma),
           _stream(stream))
+
+
+def moe_gather_rows(src, idx, dst, stream=None):
+    """dst[i] = src[idx[i]] (whole rows); src and dst 2-D with equal row bytes."""
+    if src.dim() != 2 or dst.dim() != 2 or src.dtype != dst.dtype or src.shape[1] != dst.shape[1]:
+        raise ValueError("src and dst: 2-D tensors of one dtype and row length")
+    _expect(idx, torch.int32, dst.shape[0], "idx")
+    row_bytes = src.shape[1] * src.element_size()
+    _call("moe_gather_rows", _ptr(src), ctypes.c_int64(src.shape[0]), _ptr(idx),
+          ctypes.c_int64(dst.shape[0]), ctypes.c_int(row_bytes), _ptr(dst), _stream(stream))
 
 
 def moe_pack_w13(s, w1, w3, w13, stream=None):

@@ -124,6 +124,20 @@ int moe_read_device_status(void* ws, void* stream, uint32_t* status_out, int cle
   return v ? MOE_ERR_DEVICE : MOE_OK;
 }
 
+int moe_read_gemm_clock(void* ws, void* stream, uint64_t* counters_out, int clear) {
+  if (!ws || !counters_out) return MOE_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* rec = static_cast<uint8_t*>(ws) + kClockRecordOffset;
+  cudaError_t e = cudaMemcpyAsync(counters_out, rec, 4 * sizeof(uint64_t),
+                                  cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && clear) {
+    e = cudaMemsetAsync(rec, 0, 4 * sizeof(uint64_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  }
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int moe_route(const moe_shape* shape, const void* x, const float* router_w, const float* bias,
               int32_t* topk_idx, float* topk_gate, int32_t* counts, void* ws, void* stream) {
   int rc = check(shape);

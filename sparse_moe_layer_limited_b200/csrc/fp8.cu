@@ -61,9 +61,9 @@ constexpr int FABytes = FBM * FBK;      // 16 KB
 constexpr int FBBytes = FBN * FBK;      // 32 KB
 constexpr int FStageBytes = FABytes + FBBytes;
 // warp 0 TMA, warp 1 MMA, then kEpiW epilogue warps (kEpiW / 4 per TMEM lane
-// quadrant): 16 by default; 8 (MOE_FP8_EPI=wide) gives each thread 128 running
-// sums and two TMEM loads in flight within the larger per-thread register
-// budget of a 10-warp CTA
+// quadrant): 16 by default; 8 (MOE_FP8_EPI=wide or wide32) gives each thread
+// 128 running sums within the larger per-thread register budget of a 10-warp
+// CTA
 __host__ __device__ constexpr int fp8_threads(int epi_warps) { return 64 + 32 * epi_warps; }
 constexpr int FScaleSlots = 8;      // ring of per-slice activation-scale boxes
 constexpr int FScaleBox = 132;      // floats per box: 128 rows + up to 3 of alignment
@@ -200,16 +200,19 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float x0, float x1, 
 }
 
 
-template <int kEpi, int kEpiW>
+// kEpiW epilogue warps; each reads its slice columns kLd at a time (16 or 32
+// columns per tcgen05.ld), kInFlight loads per wait
+template <int kEpi, int kEpiW, int kLd, int kInFlight>
 __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel(
     const __grid_constant__ Fp8Args args) {
   static_assert(kEpiW == 16 || kEpiW == 8, "four or two epilogue warps per lane quadrant");
+  static_assert(kLd == 16 || kLd == 32, "16- or 32-column TMEM loads");
   constexpr int FThreads = fp8_threads(kEpiW);
   constexpr int FEpiWarps = kEpiW;
   constexpr int kSub = kEpiW / 4;          // epilogue warps per TMEM lane quadrant
   constexpr int kCols = FBN / kSub;        // accumulator columns per warp
   constexpr int kFeat = (FBN / 2) / kSub;  // GEMM1: hidden features per warp
-  constexpr int kInFlight = kSub == 2 ? 2 : 1;  // 16-column TMEM loads per wait
+  static_assert((kCols / kLd) % (2 * kInFlight) == 0, "gate and up halves split evenly");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -230,6 +233,9 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const bool clock_cta = blockIdx.x == 0 && tid == 0 && args.status;
+  ClockMark cm{};
+  if (clock_cta) cm = clock_start();
   const int G1 = args.N + 1;
   const int NT = args.n_acc / FBN;
   const int KB = args.k_dim / FBK;
@@ -443,21 +449,24 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * FBN;
-        // load c (16 columns) of this warp: GEMM1 gate loads first, then up
-        constexpr int kLoads = kCols / 16;
+        // load c (kLd columns) of this warp: GEMM1 gate loads first, then up
+        constexpr int kLoads = kCols / kLd;
 #pragma unroll
         for (int c0 = 0; c0 < kLoads; c0 += kInFlight) {
-          uint32_t p[kInFlight][16];
+          uint32_t p[kInFlight][kLd];
 #pragma unroll
           for (int j = 0; j < kInFlight; ++j) {
             const int c = c0 + j;
             int col;
             if constexpr (kEpi == kFEpiSwiGLUQuant)
-              col = (c < kLoads / 2) ? kFeat * sub + 16 * c
-                                     : 128 + kFeat * sub + 16 * (c - kLoads / 2);
+              col = (c < kLoads / 2) ? kFeat * sub + kLd * c
+                                     : 128 + kFeat * sub + kLd * (c - kLoads / 2);
             else
-              col = kCols * sub + 16 * c;
-            tmem_ld16(taddr + col, p[j]);
+              col = kCols * sub + kLd * c;
+            if constexpr (kLd == 32)
+              tmem_ld32(taddr + col, p[j]);
+            else
+              tmem_ld16(taddr + col, p[j]);
           }
           tmem_wait_ld();
 #pragma unroll
@@ -465,8 +474,8 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
             const int c = c0 + j;
             const float sc = (c < kLoads / 2) ? sA : sB;
 #pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              ffma2(acc[c * 16 + i], acc[c * 16 + i + 1], __uint_as_float(p[j][i]),
+            for (int i = 0; i < kLd; i += 2)
+              ffma2(acc[c * kLd + i], acc[c * kLd + i + 1], __uint_as_float(p[j][i]),
                     __uint_as_float(p[j][i + 1]), sc);
           }
         }
@@ -581,34 +590,49 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+  if (clock_cta)
+    clock_stop(cm, reinterpret_cast<unsigned long long*>(
+                       reinterpret_cast<uint8_t*>(args.status) + kClockRecordOffset + 16));
 }
 
-template <int kEpi, int kEpiW>
+template <int kEpi, int kEpiW, int kLd, int kInFlight>
 cudaError_t launch_fp8_gemm_w(const Fp8Args& a, cudaStream_t st) {
   const size_t smem = fp8_smem_bytes(a.N + 1);
-  cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kEpi, kEpiW>,
+  auto kernel = grouped_gemm_fp8_kernel<kEpi, kEpiW, kLd, kInFlight>;
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(kernel,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem),
                             "fp8 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
-  grouped_gemm_fp8_kernel<kEpi, kEpiW><<<num_sms(), fp8_threads(kEpiW), smem, st>>>(a);
+  kernel<<<num_sms(), fp8_threads(kEpiW), smem, st>>>(a);
   return note_cuda(cudaGetLastError(), "fp8 GEMM launch");
 }
 
-// MOE_FP8_EPI=wide selects eight epilogue warps (read once per process).
-bool fp8_wide_epilogue() {
+// The epilogue's TMEM read shape, chosen once per process by MOE_FP8_EPI:
+//   unset   16 warps, 16-column loads, one per wait (64 running sums per thread)
+//   x32     16 warps, 32-column loads, one per wait
+//   wide    8 warps, 16-column loads, two per wait (128 running sums per thread)
+//   wide32  8 warps, 32-column loads, one per wait
+int fp8_epilogue_kind() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("MOE_FP8_EPI");
-    v = (e != nullptr && std::strcmp(e, "wide") == 0) ? 1 : 0;
+    v = 0;
+    if (e != nullptr && std::strcmp(e, "x32") == 0) v = 1;
+    if (e != nullptr && std::strcmp(e, "wide") == 0) v = 2;
+    if (e != nullptr && std::strcmp(e, "wide32") == 0) v = 3;
   }
-  return v == 1;
+  return v;
 }
 
 template <int kEpi>
 cudaError_t launch_fp8_gemm(const Fp8Args& a, cudaStream_t st) {
-  return fp8_wide_epilogue() ? launch_fp8_gemm_w<kEpi, 8>(a, st)
-                             : launch_fp8_gemm_w<kEpi, 16>(a, st);
+  switch (fp8_epilogue_kind()) {
+    case 1: return launch_fp8_gemm_w<kEpi, 16, 32, 1>(a, st);
+    case 2: return launch_fp8_gemm_w<kEpi, 8, 16, 2>(a, st);
+    case 3: return launch_fp8_gemm_w<kEpi, 8, 32, 1>(a, st);
+    default: return launch_fp8_gemm_w<kEpi, 16, 16, 1>(a, st);
+  }
 }
 
 }  // namespace

@@ -130,6 +130,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const bool clock_cta = kEpi != kEpiScores && blockIdx.x == 0 && tid == 0 && args.status;
+  ClockMark cm{};
+  if (clock_cta) cm = clock_start();
   const int G1 = args.N + 1;
   const int NT = (args.n_acc / BN) * args.k_splits;  // n-tiles x K splits
   const int KB = args.k_dim / BK;
@@ -472,6 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (clock_cta)
+    clock_stop(cm, reinterpret_cast<unsigned long long*>(
+                       reinterpret_cast<uint8_t*>(args.status) + kClockRecordOffset));
 }
 
 template <int kEpi, int kBN, bool kGather = false>

@@ -51,6 +51,12 @@ void note_text(const char* what);
 // contiguous and one TMA copy (16-byte aligned row pitch) brings them in.
 inline long long scale_ld(long long rows) { return (rows + 3) & ~3LL; }
 
+// Clock record in a workspace head (after the status word, inside its 256
+// bytes, clear of the status word and the schedule counters at bytes 64-75):
+// u64 pairs {SM cycles, ns} summed over launches by the first CTA of
+// the bf16 expert GEMMs (pair 0) and of the FP8 expert GEMMs (pair 1).
+constexpr size_t kClockRecordOffset = 128;
+
 // ---- host helpers (tma_host.cu) ------------------------------------------------
 // 2-D row-major tensor [rows, inner] with a (box_inner x box_rows) box and the
 // 128-byte swizzle; out-of-range rows read as zero.

@@ -25,6 +25,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Clock record of a persistent kernel: one thread's SM cycles (clock64) and
+// wall-clock nanoseconds (globaltimer) from its start to its end, added to a
+// pair of 64-bit counters; cycles / ns over many launches is the SM clock the
+// kernel ran at.
+struct ClockMark {
+  uint64_t c0, t0;
+};
+__device__ __forceinline__ ClockMark clock_start() {
+  return ClockMark{(uint64_t)clock64(), globaltimer_ns()};
+}
+__device__ __forceinline__ void clock_stop(const ClockMark& m, unsigned long long* counters) {
+  const uint64_t c1 = (uint64_t)clock64(), t1 = globaltimer_ns();
+  atomicAdd(counters, (unsigned long long)(c1 - m.c0));
+  atomicAdd(counters + 1, (unsigned long long)(t1 - m.t0));
+}
+
 // ---- mbarrier ---------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -156,3 +156,22 @@ def test_fp8_weight_gradient_entry_point_rejects_bad_arguments(L):
     bf16 = ctypes.byref(L.shape(128, 256, 16, 4, 1, 1, 256, L.DTYPE_BF16))
     assert f.moe_expert_ffn_backward_dw_fp8(bf16, *([ok] * 8), None) == L.ERR_UNSUPPORTED
     assert f.moe_expert_ffn_backward_dw_fp8(e4m3, *([None] * 8), None) == L.ERR_ARG
+
+
+def test_gather_rows_rejects_bad_arguments_before_any_launch(L):
+    f = L.lib().moe_gather_rows
+    fake = ctypes.c_void_p(1 << 20)                        # never dereferenced
+    odd = ctypes.c_void_p((1 << 20) + 8)                   # not 16-byte aligned
+    assert f(fake, 10, fake, 4, 24, fake, None) == L.ERR_ARG      # row bytes not a multiple of 16
+    assert f(fake, 10, fake, -1, 32, fake, None) == L.ERR_ARG     # negative count
+    assert f(None, 10, fake, 4, 32, fake, None) == L.ERR_ARG
+    assert f(fake, 10, None, 4, 32, fake, None) == L.ERR_ARG
+    assert f(odd, 10, fake, 4, 32, fake, None) == L.ERR_ARG
+    assert f(fake, 10, fake, 0, 32, fake, None) == L.OK          # nothing to do
+
+
+def test_gemm_clock_reader_rejects_null(L):
+    import ctypes as C
+    c = (C.c_uint64 * 4)()
+    assert L.lib().moe_read_gemm_clock(None, None, c, 0) == L.ERR_ARG
+    assert L.lib().moe_read_gemm_clock(C.c_void_p(1 << 20), None, None, 0) == L.ERR_ARG

@@ -7,6 +7,8 @@ bf16 layer parity tests (routing and dispatch bit-exact, expert outputs and
 the layer within the bf16 tolerance) in a child process with the variable set.
 Likewise MOE_WGRAD=single selects the one-CTA weight-gradient kernel instead
 of the default CTA-pair one; the weight-gradient parity tests rerun with it.
+MOE_FP8_EPI picks the FP8 GEMM epilogue's TMEM read shape (x32, wide,
+wide32); the FP8 layer and FP8 input-gradient parity tests rerun with each.
 """
 import os
 import subprocess
@@ -36,6 +38,18 @@ def test_one_cta_weight_gradient_kernel():
     env = dict(os.environ, MOE_WGRAD="single")
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
            os.path.join(HERE, "test_gpu_backward.py"), "-k", "dw"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    tail = (r.stdout + r.stderr)[-3000:]
+    assert r.returncode == 0, tail
+    assert " passed" in r.stdout and "failed" not in r.stdout, tail
+
+
+@pytest.mark.parametrize("kind", ["x32", "wide", "wide32"])
+def test_fp8_epilogue_variant(kind):
+    env = dict(os.environ, MOE_FP8_EPI=kind)
+    cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+           os.path.join(HERE, "test_gpu_parity.py"), os.path.join(HERE, "test_gpu_fp8_backward.py"),
+           "-k", "small_fp8 or backward_dx"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
     tail = (r.stdout + r.stderr)[-3000:]
     assert r.returncode == 0, tail
