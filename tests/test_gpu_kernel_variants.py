@@ -7,8 +7,9 @@ bf16 layer parity tests (routing and dispatch bit-exact, expert outputs and
 the layer within the bf16 tolerance) in a child process with the variable set.
 Likewise MOE_WGRAD=single selects the one-CTA weight-gradient kernel instead
 of the default CTA-pair one; the weight-gradient parity tests rerun with it.
-MOE_FP8_EPI picks the FP8 GEMM epilogue's TMEM read shape (x32, wide,
-wide32); the FP8 layer and FP8 input-gradient parity tests rerun with each.
+MOE_FP8_EPI picks the FP8 GEMM epilogue's TMEM read shape (narrow, x32,
+wide32; the default is the eight-warp one); the FP8 layer and FP8
+input-gradient parity tests rerun with each.
 """
 import os
 import subprocess
@@ -44,7 +45,7 @@ def test_one_cta_weight_gradient_kernel():
     assert " passed" in r.stdout and "failed" not in r.stdout, tail
 
 
-@pytest.mark.parametrize("kind", ["x32", "wide", "wide32"])
+@pytest.mark.parametrize("kind", ["narrow", "x32", "wide32"])
 def test_fp8_epilogue_variant(kind):
     env = dict(os.environ, MOE_FP8_EPI=kind)
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
