@@ -218,6 +218,27 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
                             const int32_t* offsets, const void* w13, const void* w2,
                             void* y_perm, void* y_shared, void* ws, void* stream);
 
+/* moe_expert_ffn_combine (BF16 mode only): moe_expert_ffn followed by
+ * moe_combine, with the COMBINE step inside GEMM2's epilogue ([P1] §2.2 runs
+ * DISPATCH -> MLP -> COMBINE within one chunk).  After storing a row of
+ * y_perm or y_shared, the epilogue counts one arrival for (token, 256-column
+ * tile) in the workspace; the token's K+1-th arrival (its K routed rows and
+ * its shared-expert row) forms that tile of
+ *   y[t] = y_shared[t] + sum_k topk_gate[t,k] * y_perm[slot[t,k]]
+ * with fp32 fused multiply-adds in k order and one bf16 rounding: the same
+ * operations in the same order as moe_combine, so y is bit-identical to
+ * moe_expert_ffn + moe_combine.  The shared expert's tiles run first.
+ *   x_perm, offsets, perm_tok, slot   from moe_dispatch
+ *   topk_gate  [T, K] fp32 from moe_route
+ *   x, w13, w2, y_perm, y_shared, ws  as at moe_expert_ffn
+ *   y          [T, d] bf16 out
+ * The arrival counters ([T, d/256] int32 in the workspace) are cleared at the
+ * start of every call.  Returns MOE_ERR_UNSUPPORTED for other dtypes. */
+int moe_expert_ffn_combine(const moe_shape* shape, const void* x_perm, const int32_t* offsets,
+                           const int32_t* perm_tok, const int32_t* slot, const float* topk_gate,
+                           const void* x, const void* w13, const void* w2, void* y_perm,
+                           void* y_shared, void* y, void* ws, void* stream);
+
 /* Backward of the expert FFNs, input gradients ([P1] §2.2: the backward
  * pass runs COMBINE -> MLP_B -> MLP_W -> DISPATCH; this is MLP_B), BF16 mode.
  * With g = a W1^T, u = a W3^T (a = a dispatched row, or an x row for the

@@ -11,7 +11,7 @@ from ._lib import (  # noqa: F401
     moe_expert_ffn_backward_dw_fp8,
     DTYPE_BF16, DTYPE_E4M3, DTYPE_FP32, MoEError, MoEShape, check_shape, lib, moe_bias_update,
     moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_expert_ffn, moe_expert_ffn_gathered,
-    moe_gather_rows,
+    moe_gather_rows, moe_expert_ffn_combine,
     moe_forward, moe_pack_w13, moe_quantize_weights,
     moe_read_device_status, moe_read_gemm_clock, moe_route, moe_route_softmax, moe_workspace_init, shape,
     status_string,

@@ -52,6 +52,7 @@ _SIGS = {
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 10),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 12),
     "moe_expert_ffn_gathered": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 9),
+    "moe_expert_ffn_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 13),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 6),
     "moe_combine_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 7),
     "moe_route_backward": (ctypes.c_int, [ctypes.POINTER(MoEShape)] + [_c_p] * 11),
@@ -236,6 +237,20 @@ def moe_expert_ffn_gathered(s, x, perm_tok, offsets, w13, w2, y_perm, y_shared, 
     _expect(y_shared, x_torch_dtype(s), s.T * s.d, "y_shared")
     _call("moe_expert_ffn_gathered", ctypes.byref(s), _ptr(x), _ptr(perm_tok), _ptr(offsets),
           _ptr(w13), _ptr(w2), _ptr(y_perm), _ptr(y_shared), _ptr(ws), _stream(stream))
+
+
+def moe_expert_ffn_combine(s, x_perm, offsets, perm_tok, slot, topk_gate, x, w13, w2, y_perm,
+                           y_shared, y, ws, stream=None):
+    _expect(w13, w_torch_dtype(s), (s.N + 1) * 2 * s.f * s.d, "w13")
+    _expect(w2, w_torch_dtype(s), (s.N + 1) * s.d * s.f, "w2")
+    _expect(y_perm, x_torch_dtype(s), s.T * s.K * s.d, "y_perm")
+    _expect(y_shared, x_torch_dtype(s), s.T * s.d, "y_shared")
+    _expect(y, x_torch_dtype(s), s.T * s.d, "y")
+    _expect(slot, torch.int32, s.T * s.K, "slot")
+    _expect(topk_gate, torch.float32, s.T * s.K, "topk_gate")
+    _call("moe_expert_ffn_combine", ctypes.byref(s), _ptr(x_perm), _ptr(offsets), _ptr(perm_tok),
+          _ptr(slot), _ptr(topk_gate), _ptr(x), _ptr(w13), _ptr(w2), _ptr(y_perm),
+          _ptr(y_shared), _ptr(y), _ptr(ws), _stream(stream))
 
 
 def backward_workspace_size(s) -> int:

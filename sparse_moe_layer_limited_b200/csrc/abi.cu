@@ -36,6 +36,10 @@ WsLayout ws_layout(const moe_shape& s) {
     L.xq_scales = off;
     off = align256(off + (size_t)scale_ld(s.T) * (s.d / 128) * 4);
   }
+  if (s.dtype == MOE_DTYPE_BF16) {
+    L.arrive = off;
+    off = align256(off + (size_t)s.T * (s.d / 256) * 4);
+  }
   L.total = off;
   return L;
 }
@@ -225,6 +229,22 @@ int moe_expert_ffn_gathered(const moe_shape* shape, const void* x, const int32_t
   if ((rc = ws_check(shape, ws))) return rc;
   return launch_ffn_tc_bf16(*shape, nullptr, perm_tok, offsets, x, w13, w2, y_perm, y_shared,
                             ws, static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_ffn_combine(const moe_shape* shape, const void* x_perm, const int32_t* offsets,
+                           const int32_t* perm_tok, const int32_t* slot, const float* topk_gate,
+                           const void* x, const void* w13, const void* w2, void* y_perm,
+                           void* y_shared, void* y, void* ws, void* stream) {
+  int rc = check(shape);
+  if (rc) return rc;
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!ptr_ok(x_perm) || !ptr_ok(offsets) || !ptr_ok(perm_tok) || !ptr_ok(slot) ||
+      !ptr_ok(topk_gate) || !ptr_ok(x) || !ptr_ok(w13) || !ptr_ok(w2) || !ptr_ok(y_perm) ||
+      !ptr_ok(y_shared) || !ptr_ok(y))
+    return MOE_ERR_ARG;
+  if ((rc = ws_check(shape, ws))) return rc;
+  return launch_ffn_combine_bf16(*shape, x_perm, offsets, perm_tok, slot, topk_gate, x, w13, w2,
+                                 y_perm, y_shared, y, ws, static_cast<cudaStream_t>(stream));
 }
 
 size_t moe_backward_workspace_size(const moe_shape* shape) {

@@ -152,17 +152,29 @@ __global__ void __launch_bounds__(256) scatter_gather_kernel(
   const int nt = min(kChunkTokens, T - t0);
   chunk_slots(idx, chunk_base, c, t0, nt, T, K, N, perm_tok, slot, sidx, sslot);
   if (x_perm == nullptr) return;  // slots only: the expert GEMM gathers the rows itself
-  // gather: warp per token, 16-byte vectors
+  // gather: warp per token, 16-byte vectors, four loads in flight per lane
   constexpr int kElems = 16 / sizeof(XT);
+  constexpr int kUnroll = 4;
   const int nvec = d / kElems;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int tl = warp; tl < nt; tl += 8) {
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t0 + tl) * d);
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 val = __ldg(src + v);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kUnroll) {
+      uint4 val[kUnroll];
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        const int v = v0 + 32 * j;
+        if (v < nvec) val[j] = __ldg(src + v);
+      }
       for (int k = 0; k < K; ++k) {
         const int r = sslot[tl * K + k];
-        if (r >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)r * d)[v] = val;
+        if (r < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * d);
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+          const int v = v0 + 32 * j;
+          if (v < nvec) dst[v] = val[j];
+        }
       }
     }
   }
@@ -185,21 +197,31 @@ __global__ void __launch_bounds__(256) scatter_gather_fp8_kernel(
   const int tiles = d / QB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = lane >> 4, l16 = lane & 15;
+  constexpr int kUnroll = 4;  // tiles per half-warp per pass, their loads in flight together
   for (int tl = warp; tl < nt; tl += 8) {
     const __nv_bfloat16* src = x + (size_t)(t0 + tl) * d;
-    for (int tc0 = 0; tc0 < tiles; tc0 += 2) {  // two tiles per warp pass
-      const int tc = tc0 + half;
-      const bool live = tc < tiles;
-      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (live) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(src + tc * QB) + l16), v);
-      uint2 codes;
-      const float sc = quant_tile_16lanes(v, codes);
-      if (!live) continue;
-      for (int k = 0; k < K; ++k) {
-        const int r = sslot[tl * K + k];
-        if (r < 0) continue;
-        *reinterpret_cast<uint2*>(x_perm + (size_t)r * d + tc * QB + 8 * l16) = codes;
-        if (l16 == 0) x_perm_scales[(size_t)tc * sc_ld + r] = sc;
+    for (int tc0 = 0; tc0 < tiles; tc0 += 2 * kUnroll) {  // eight tiles per warp pass
+      float v[kUnroll][8];
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        const int tc = tc0 + 2 * j + half;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[j][i] = 0.f;
+        if (tc < tiles)
+          bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(src + tc * QB) + l16), v[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < kUnroll; ++j) {
+        const int tc = tc0 + 2 * j + half;
+        uint2 codes;
+        const float sc = quant_tile_16lanes(v[j], codes);  // both halves take part
+        if (tc >= tiles) continue;
+        for (int k = 0; k < K; ++k) {
+          const int r = sslot[tl * K + k];
+          if (r < 0) continue;
+          *reinterpret_cast<uint2*>(x_perm + (size_t)r * d + tc * QB + 8 * l16) = codes;
+          if (l16 == 0) x_perm_scales[(size_t)tc * sc_ld + r] = sc;
+        }
       }
     }
   }

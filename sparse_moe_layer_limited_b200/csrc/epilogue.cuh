@@ -33,6 +33,17 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 8 bf16 packed in 16 bytes -> 8 fp32.
+__device__ __forceinline__ void bf16x8_unpack(const uint4& w, float* v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
 // 8 bf16 (one 16-byte load) -> 8 fp32.
 __device__ __forceinline__ void bf16x8_load(const __nv_bfloat16* src, float* v) {
   const uint4 w = *reinterpret_cast<const uint4*>(src);

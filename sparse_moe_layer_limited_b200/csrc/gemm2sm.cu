@@ -35,6 +35,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "epilogue.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -75,7 +76,6 @@ constexpr size_t pair_smem_bytes(int groups) {
   return 1024 + (size_t)PStages * PStageBytes + 1024 + (size_t)(groups + 1) * 4;
 }
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
 
 // Rows of a group split into near-equal units of at most UMax rows; every unit
 // but the last has `size` rows (a multiple of 16).

@@ -62,7 +62,8 @@ constexpr int kABytes = BM * BK * 2;
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiScores = 2, kEpiSwiGLUBwd = 3 };
+enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiScores = 2, kEpiSwiGLUBwd = 3,
+           kEpiStoreCombine = 4 };
 
 template <int kBN>
 struct TileCfg {
@@ -92,6 +93,16 @@ struct alignas(64) GemmArgs {
   const __nv_bfloat16* aux_routed;
   const __nv_bfloat16* aux_shared;
   uint32_t* status;
+  // store-and-combine epilogue (GEMM2 with the COMBINE step fused): the
+  // token of every routed row, each token's K slots and gates, the output y
+  // [T, d], and one arrival counter per (token, 256-column tile), zero on entry
+  const int32_t* perm_tok;
+  const int32_t* slot;
+  const float* gate;
+  __nv_bfloat16* y;
+  int32_t* arrive;
+  int K;
+  int shared_first;  // 1: the shared expert's tiles come before the routed ones
   int N, T;
   int rows_routed;  // T*K
   int a_shared_row0;
@@ -102,6 +113,66 @@ struct alignas(64) GemmArgs {
   int n_valid; // columns to store (score epilogue)
   int k_splits; // K ranges computed by separate units (score epilogue; else 1)
 };
+
+// COMBINE fused into GEMM2's epilogue (the mhpq.cn article §2.2 runs
+// DISPATCH -> MLP -> COMBINE as one chunk): after storing its row's 256
+// columns of y_perm (or y_shared), a thread counts one arrival for (token,
+// column tile).  A token has K routed rows and its shared-expert row; the
+// K+1-th arrival sees every one of them stored, and its warp then forms
+//   y[t, cols] = y_shared[t] + sum_k gate[t,k] * y_perm[slot[t,k]]
+// in k order with fp32 fused multiply-adds and one bf16 rounding -- the same
+// operations, in the same order, as the standalone combine kernel, so the
+// result is bit-identical.  Each lane handles 8 of the tile's 256 columns.
+// The rows are read through L2 (ld.global.cg): they were written by other
+// CTAs, made visible by the writers' fence before their counter increment and
+// ordered after the last increment by the reader's fence.
+__device__ __forceinline__ void combine_arrivals(const GemmArgs& args, int g, int n, int r,
+                                                 bool valid, int lane) {
+  const int NTd = args.n_acc / 256;
+  int tok = -1;
+  if (valid) {
+    tok = (g < args.N) ? args.perm_tok[args.offsets[g] + r] : r;
+    if (tok < 0 || tok >= args.T) {
+      atomicOr(args.status, kErrBadIndex);
+      tok = -1;
+    }
+  }
+  bool last = false;
+  if (tok >= 0) {
+    __threadfence();
+    last = atomicAdd(&args.arrive[(size_t)tok * NTd + n], 1) == args.K;
+  }
+  unsigned mask = __ballot_sync(0xffffffffu, last);
+  if (mask == 0u) return;
+  __threadfence();
+  const int d = args.n_acc;
+  const int col = n * 256 + 8 * lane;
+  const long long TK = (long long)args.T * args.K;
+  while (mask) {
+    const int src = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    const int t = __shfl_sync(0xffffffffu, tok, src);
+    float acc[8];
+    bf16x8_unpack(__ldcg(reinterpret_cast<const uint4*>(args.out_shared + (size_t)t * d + col)),
+                  acc);
+    for (int k = 0; k < args.K; ++k) {
+      const int sl = __ldg(args.slot + (size_t)t * args.K + k);
+      const bool ok = sl >= 0 && sl < TK;  // a slot outside the rows adds nothing
+      const float gk = ok ? __ldg(args.gate + (size_t)t * args.K + k) : 0.f;
+      float rv[8];
+      bf16x8_unpack(__ldcg(reinterpret_cast<const uint4*>(args.out_routed +
+                                                         (size_t)(ok ? sl : 0) * d + col)),
+                    rv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(gk, rv[i], acc[i]);
+    }
+    uint4 o;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(args.y + (size_t)t * d + col) = o;
+  }
+}
 
 template <int kEpi, int kBN, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
@@ -157,9 +228,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
   }
-  for (int g = tid; g < G1; g += kThreads) {
+  // tiles are laid out group by group in schedule position order; position p
+  // holds group p, or with shared_first group (p + N) mod (N + 1): the shared
+  // expert first, then the routed experts in order
+  auto group_at = [&](int p) { return args.shared_first ? (p + args.N) % G1 : p; };
+  for (int p = tid; p < G1; p += kThreads) {
+    const int g = group_at(p);
     const int rows = (g < args.N) ? args.offsets[g + 1] - args.offsets[g] : args.T;
-    tile_start[g] = rows > 0 ? (rows + BM - 1) / BM : 0;
+    tile_start[p] = rows > 0 ? (rows + BM - 1) / BM : 0;
   }
   tc_fence_before();
   __syncthreads();
@@ -193,9 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
       const int mid = (lo + hi) >> 1;
       if (tile_start[mid] <= tile) lo = mid; else hi = mid;
     }
-    g = lo;
-    mt = (tile_start[g + 1] - tile_start[g]) / NT;
-    const int local = tile - tile_start[g];
+    g = group_at(lo);
+    mt = (tile_start[lo + 1] - tile_start[lo]) / NT;
+    const int local = tile - tile_start[lo];
     n = local / mt;
     m = local - n * mt;
   };
@@ -411,6 +487,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
           if (valid) store_row32(orow + n * BN + c, y);
         }
+      } else if constexpr (kEpi == kEpiStoreCombine) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
+          if (valid) store_row32(orow + n * BN + c, y);
+        }
+        // the accumulator is drained: hand it back before the combine work
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        combine_arrivals(args, g, n, r, valid, lane);
+        continue;
       } else if constexpr (kEpi == kEpiSwiGLUBwd) {
         // the accumulator is dh for hidden features n*BN + c; with g, u the
         // stored gate/up products: dg = dh * u * silu'(g), du = dh * silu(g),
@@ -517,6 +610,22 @@ __global__ void router_split_kernel(const float* __restrict__ R, int N, int d,
 
 }  // namespace
 
+namespace {
+// The COMBINE step fused into GEMM2 (store-and-combine epilogue): null when
+// the combine runs as its own kernel.
+struct FusedCombine {
+  const int32_t* perm_tok;
+  const int32_t* slot;
+  const float* gate;
+  void* y;
+};
+
+int ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* perm_tok,
+                const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                void* y_perm, void* y_shared, void* ws, cudaStream_t st,
+                const FusedCombine* fc);
+}  // namespace
+
 int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* perm_tok,
                        const int32_t* offsets, const void* x, const void* w13, const void* w2,
                        void* y_perm, void* y_shared, void* ws, cudaStream_t st) {
@@ -533,6 +642,23 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* pe
     return launch_ffn_tc_bf16_pair(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
   if (perm_tok == nullptr && kind == 1)
     return launch_ffn_tc_bf16_dual(s, x_perm, offsets, x, w13, w2, y_perm, y_shared, ws, st);
+  return ffn_tc_bf16(s, x_perm, perm_tok, offsets, x, w13, w2, y_perm, y_shared, ws, st,
+                     nullptr);
+}
+
+int launch_ffn_combine_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                            const int32_t* perm_tok, const int32_t* slot, const float* gate,
+                            const void* x, const void* w13, const void* w2, void* y_perm,
+                            void* y_shared, void* y, void* ws, cudaStream_t st) {
+  const FusedCombine fc{perm_tok, slot, gate, y};
+  return ffn_tc_bf16(s, x_perm, nullptr, offsets, x, w13, w2, y_perm, y_shared, ws, st, &fc);
+}
+
+namespace {
+int ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* perm_tok,
+                const int32_t* offsets, const void* x, const void* w13, const void* w2,
+                void* y_perm, void* y_shared, void* ws, cudaStream_t st,
+                const FusedCombine* fc) {
   const WsLayout L = ws_layout(s);
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(w + L.h);
@@ -590,9 +716,27 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* pe
   g2.out_ld = s.d;
   g2.a_rep = 1;
   g2.k_splits = 1;
-  if (launch_gemm<kEpiStore, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (fc == nullptr) {
+    if (launch_gemm<kEpiStore, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  // store-and-combine: arrival counters start at zero; the shared expert's
+  // tiles go first so each token completes with its last routed row
+  int32_t* arrive = reinterpret_cast<int32_t*>(w + L.arrive);
+  if (note_cuda(cudaMemsetAsync(arrive, 0, (size_t)s.T * (s.d / 256) * sizeof(int32_t), st),
+                "fused combine: clear arrival counters") != cudaSuccess)
+    return MOE_ERR_CUDA;
+  g2.perm_tok = fc->perm_tok;
+  g2.slot = fc->slot;
+  g2.gate = fc->gate;
+  g2.y = static_cast<__nv_bfloat16*>(fc->y);
+  g2.arrive = arrive;
+  g2.K = s.K;
+  g2.shared_first = 1;
+  if (launch_gemm<kEpiStoreCombine, 256>(g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
+}  // namespace
 
 int router_k_splits(const moe_shape& s) {
   const int m_tiles = (s.T + BM - 1) / BM;

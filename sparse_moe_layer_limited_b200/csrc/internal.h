@@ -29,6 +29,7 @@ struct WsLayout {
   size_t h_scales = 0;    // fp32 block-major [f/128, scale_ld(T*K + T)] (E4M3)
   size_t xq = 0;          // E4M3 codes of x for the shared expert [T, d]
   size_t xq_scales = 0;   // fp32 block-major [d/128, scale_ld(T)]
+  size_t arrive = 0;      // int32 [T, d/256] arrival counters of the fused combine (BF16)
   size_t total = 0;
 };
 WsLayout ws_layout(const moe_shape& s);
@@ -167,6 +168,12 @@ int launch_ffn_tc_bf16(const moe_shape& s, const void* x_perm, const int32_t* pe
                        const int32_t* offsets, const void* x, const void* w13, const void* w2,
                        void* y_perm, void* y_shared, void* ws, cudaStream_t st);
 // The same two GEMMs on CTA pairs (tcgen05 cta_group::2), gemm2sm.cu.
+// The same GEMMs with the COMBINE step fused into GEMM2's epilogue: y is
+// written directly (bit-identical to the standalone combine).
+int launch_ffn_combine_bf16(const moe_shape& s, const void* x_perm, const int32_t* offsets,
+                            const int32_t* perm_tok, const int32_t* slot, const float* gate,
+                            const void* x, const void* w13, const void* w2, void* y_perm,
+                            void* y_shared, void* y, void* ws, cudaStream_t st);
 int launch_ffn_tc_bf16_dual(const moe_shape& s, const void* x_perm, const int32_t* offsets,
                             const void* x, const void* w13, const void* w2, void* y_perm,
                             void* y_shared, void* ws, cudaStream_t st);

@@ -18,10 +18,15 @@ class MoELayer:
 
     gather (BF16 only): GEMM1 reads each routed row straight from x through
     perm_tok (moe_expert_ffn_gathered) instead of a permuted copy; dispatch
-    then writes no x_perm."""
+    then writes no x_perm.
+
+    fused_combine (BF16 only, not with gather): the combine runs inside
+    GEMM2's epilogue (moe_expert_ffn_combine) instead of as its own kernel;
+    the output is bit-identical."""
 
     def __init__(self, shape: L.MoEShape, router_w, bias, w13, w2, w13_scales=None,
-                 w2_scales=None, gamma: float = 0.001, gather: bool = False):
+                 w2_scales=None, gamma: float = 0.001, gather: bool = False,
+                 fused_combine: bool = False):
         rc = L.check_shape(shape)
         if rc != L.OK:
             raise L.MoEError("moe_check_shape", rc)
@@ -30,6 +35,8 @@ class MoELayer:
         self.w13_scales, self.w2_scales = w13_scales, w2_scales
         self.gamma = float(gamma)
         self.gather = bool(gather) and s.dtype == L.DTYPE_BF16
+        self.fused_combine = (bool(fused_combine) and s.dtype == L.DTYPE_BF16
+                              and not self.gather)
         dev = router_w.device
         i32 = dict(dtype=torch.int32, device=dev)
         xdt = L.x_torch_dtype(s)
@@ -63,11 +70,23 @@ class MoELayer:
                     self.ws, stream)
         L.moe_dispatch(s, x, self.topk_idx, self.counts, self.offsets, self.perm_tok, self.slot,
                        self.x_perm, self.x_perm_scales, self.ws, stream)
-        self.experts(x, stream)
-        L.moe_combine(s, self.y_perm, self.y_shared, self.slot, self.topk_gate, self.y, stream)
+        self.experts_and_combine(x, stream)
         if update_bias:
             L.moe_bias_update(s, self.counts, self.bias, self.gamma, stream)
         return self.y
+
+    def experts_and_combine(self, x, stream=None):
+        """The expert GEMMs and the COMBINE step (one fused launch pair when
+        fused_combine is set); writes self.y."""
+        s = self.shape
+        if self.fused_combine:
+            L.moe_expert_ffn_combine(s, self.x_perm, self.offsets, self.perm_tok, self.slot,
+                                     self.topk_gate, x, self.w13, self.w2, self.y_perm,
+                                     self.y_shared, self.y, self.ws, stream)
+        else:
+            self.experts(x, stream)
+            L.moe_combine(s, self.y_perm, self.y_shared, self.slot, self.topk_gate, self.y,
+                          stream)
 
     def experts(self, x, stream=None):
         """The expert GEMMs on the dispatched rows (gathered from x or read from x_perm)."""
