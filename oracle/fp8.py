@@ -29,8 +29,9 @@ from __future__ import annotations
 import numpy as np
 
 
-def e4m3_decode(codes) -> np.ndarray:
-    """E4M3 bit patterns (uint8) -> float64 values (NaN for S.1111.111)."""
+def _e4m3_value(codes) -> np.ndarray:
+    """The format's definition: E4M3 bit patterns (uint8) -> float64 values
+    (NaN for S.1111.111)."""
     c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     sign = np.where(c >> 7, -1.0, 1.0)
     E = (c >> 3) & 0xF
@@ -40,9 +41,18 @@ def e4m3_decode(codes) -> np.ndarray:
     return sign * mag
 
 
+_E4M3_TABLE = _e4m3_value(np.arange(256, dtype=np.uint8))
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 bit patterns (uint8) -> float64 values (NaN for S.1111.111): the
+    entry of each code in the table of all 256 values the definition gives."""
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
 def e4m3_all_values() -> np.ndarray:
     """Values of all 256 codes, index = code."""
-    return e4m3_decode(np.arange(256, dtype=np.uint8))
+    return _E4M3_TABLE.copy()
 
 
 _POS_VALUES = e4m3_all_values()[:127]          # codes 0x00..0x7E: 0 .. 448, increasing
@@ -50,17 +60,26 @@ _POS_VALUES = e4m3_all_values()[:127]          # codes 0x00..0x7E: 0 .. 448, inc
 
 def e4m3_encode(v) -> np.ndarray:
     """float -> E4M3 code, round to nearest (ties to even mantissa),
-    saturating finite overflow to +-448; NaN -> 0x7F."""
-    v = np.asarray(v, dtype=np.float64)
+    saturating finite overflow (infinities included) to +-448; NaN -> 0x7F.
+    float32 input is rounded in float32 (every step below is exact there),
+    anything else in float64."""
+    v = np.asarray(v)
+    if v.dtype != np.float32:
+        v = v.astype(np.float64)
     a = np.abs(v)
     _, e = np.frexp(a)                         # a = m * 2**e, 0.5 <= m < 1
     step_exp = np.maximum(e - 4, -9)           # 3 mantissa bits; subnormal step 2^-9
     r = np.ldexp(np.rint(np.ldexp(a, -step_exp)), step_exp)
-    r = np.minimum(r, 448.0)
-    code = np.searchsorted(_POS_VALUES, np.nan_to_num(r, nan=0.0)).astype(np.uint8)
-    assert np.all(np.isnan(r) | (_POS_VALUES[np.minimum(code, 126)] == r))
+    r = np.fmin(r, 448.0)                      # saturate (NaN is replaced below)
+    # the code of r: a subnormal r < 2^-6 is (r / 2^-9); a normal
+    # r = (1 + M/8) 2^(E-7) has exponent field E and mantissa M
+    mr, er = np.frexp(r)                       # r = mr 2^er, 0.5 <= mr < 1
+    code = np.where(r >= 2.0 ** -6, ((er + 6) << 3) | (np.rint(mr * 16) - 8).astype(np.int64),
+                    np.rint(r * 512).astype(np.int64)).astype(np.uint8)
     code = np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
-    return np.where(np.isnan(v), np.uint8(0x7F), code).astype(np.uint8)
+    if np.isnan(v).any():
+        code = np.where(np.isnan(v), np.uint8(0x7F), code).astype(np.uint8)
+    return code
 
 
 def e5m2_decode(codes) -> np.ndarray:
