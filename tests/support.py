@@ -149,3 +149,43 @@ def device_weights(cfg: MoEConfig, seed: int = 0):
         out = dict(w13=w13q, w2=w2q, w13_scales=s13, w2_scales=s2)
     torch.cuda.synchronize()
     return out
+
+
+# ---------------------------------------------------------------------------
+# Per-expert oracle jobs in parallel (full-size layers)
+# ---------------------------------------------------------------------------
+
+def _expert_job(args):
+    """Worker: one expert's oracle outputs on its rows (weights regenerated
+    from the seeded generator inside the worker)."""
+    cfg, seed, e, rows, kind = args
+    w = tuple(gen.make_expert_weight(cfg, seed, n, e).astype(np.float64)
+              for n in ("w1", "w3", "w2"))
+    if kind == "fp8":
+        return e, oracle.fp8_swiglu_expert(rows, *w)
+    return e, oracle.swiglu_expert(rows, *w, h_round="bf16")
+
+
+def expert_outputs_parallel(cfg: MoEConfig, jobs: dict, kind: str, seed: int = 0,
+                            workers: int | None = None, timeout: float = 1800.0) -> dict:
+    """{expert: rows [n, d]} -> {expert: oracle outputs [n, d]}, one process
+    per expert job in a pool started with 'spawn' (no CUDA state is inherited);
+    kind 'fp8' runs the E4M3 expert emulation, 'bf16' the expert with h
+    rounded to bf16."""
+    import multiprocessing as mp
+    import os
+    n = workers or max(1, min(16, len(os.sched_getaffinity(0))))
+    items = [(cfg, seed, int(e), np.asarray(r, np.float64), kind) for e, r in jobs.items()]
+    with mp.get_context("spawn").Pool(n) as pool:
+        # bounded: a pool whose workers cannot start would otherwise wait forever
+        return dict(pool.map_async(_expert_job, items, chunksize=1).get(timeout=timeout))
+
+
+def tail_tile_rows(offsets: np.ndarray, e: int, tile: int = 128) -> np.ndarray:
+    """Rows (expert-major) of expert e's last m-tile: the ragged tail the
+    expert GEMMs handle with a partly filled (or M=64) tile."""
+    a, z = int(offsets[e]), int(offsets[e + 1])
+    if z == a:
+        return np.zeros(0, dtype=np.int64)
+    full = (z - a - 1) // tile * tile
+    return np.arange(a + full, z)
