@@ -615,7 +615,10 @@ cudaError_t launch_fp8_gemm_w(const Fp8Args& a, cudaStream_t st) {
 //   x32     16 warps, 32-column loads, one per wait
 //   wide32  8 warps, 32-column loads, one per wait
 // (the 16-warp shapes run at 96 registers a thread and spill; x32 and wide32
-// spill more and measured slower)
+// spill more and measured slower.  The 18-warp CTA cannot have more registers:
+// compiled for 112 a thread, its launch is refused; a 20-warp CTA that moves
+// registers from its control warpgroup to the epilogue with setmaxnreg spills
+// the TMA and MMA loops instead, 0.6-0.8 KB a thread at 32-56 registers)
 int fp8_epilogue_kind() {
   static int v = -1;
   if (v < 0) {

@@ -148,23 +148,41 @@ __device__ __forceinline__ void combine_arrivals(const GemmArgs& args, int g, in
   const int d = args.n_acc;
   const int col = n * 256 + 8 * lane;
   const long long TK = (long long)args.T * args.K;
+  constexpr int kBatch = 8;  // rows whose loads are in flight together
   while (mask) {
     const int src = __ffs(mask) - 1;
     mask &= mask - 1u;
     const int t = __shfl_sync(0xffffffffu, tok, src);
-    float acc[8];
-    bf16x8_unpack(__ldcg(reinterpret_cast<const uint4*>(args.out_shared + (size_t)t * d + col)),
-                  acc);
-    for (int k = 0; k < args.K; ++k) {
-      const int sl = __ldg(args.slot + (size_t)t * args.K + k);
+    // lanes 0..K-1 fetch the token's slots and gates once (kMaxK <= 32)
+    int my_sl = 0;
+    float my_g = 0.f;
+    if (lane < args.K) {
+      const int sl = __ldg(args.slot + (size_t)t * args.K + lane);
       const bool ok = sl >= 0 && sl < TK;  // a slot outside the rows adds nothing
-      const float gk = ok ? __ldg(args.gate + (size_t)t * args.K + k) : 0.f;
-      float rv[8];
-      bf16x8_unpack(__ldcg(reinterpret_cast<const uint4*>(args.out_routed +
-                                                         (size_t)(ok ? sl : 0) * d + col)),
-                    rv);
+      my_sl = ok ? sl : 0;
+      my_g = ok ? __ldg(args.gate + (size_t)t * args.K + lane) : 0.f;
+    }
+    float acc[8];
+    const uint4 sh = __ldcg(reinterpret_cast<const uint4*>(args.out_shared + (size_t)t * d + col));
+    for (int k0 = 0; k0 < args.K; k0 += kBatch) {
+      uint4 rv[kBatch];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(gk, rv[i], acc[i]);
+      for (int j = 0; j < kBatch; ++j) {
+        const int sl = __shfl_sync(0xffffffffu, my_sl, (k0 + j) & 31);
+        if (k0 + j < args.K)
+          rv[j] = __ldcg(reinterpret_cast<const uint4*>(args.out_routed + (size_t)sl * d + col));
+      }
+      if (k0 == 0) bf16x8_unpack(sh, acc);
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const float gk = __shfl_sync(0xffffffffu, my_g, (k0 + j) & 31);
+        if (k0 + j < args.K) {
+          float r8[8];
+          bf16x8_unpack(rv[j], r8);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(gk, r8[i], acc[i]);
+        }
+      }
     }
     uint4 o;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
