@@ -50,6 +50,9 @@ def parse():
     p.add_argument("--fused-combine", choices=["on", "off"], default="off",
                    help="bf16: the combine runs inside GEMM2's epilogue (on) or as its own "
                         "kernel (off); the output is bit-identical")
+    p.add_argument("--only", choices=["backward_fp8"], default=None,
+                   help="run one of the line's measurements alone and print its object "
+                        "(backward_fp8: the FP8 expert backward on the V3 FP8 shapes)")
     p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
     p.add_argument("--N", type=int, default=None, help="override routed experts (profiling)")
     return p.parse_args()
@@ -246,6 +249,12 @@ def main():
         cfg = cfg.with_(N=args.N)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.only == "backward_fp8":
+        import torch
+        out = run_backward_fp8(BY_NAME["v3_fp8"], torch.device("cuda"), calls=max(1, args.steps),
+                               warmup=args.warmup)
+        print(json.dumps({"backward_fp8": out}), flush=True)
+        return out
 
     import torch
 

@@ -35,6 +35,8 @@ WsLayout ws_layout(const moe_shape& s) {
     off = align256(off + (size_t)s.T * s.d);
     L.xq_scales = off;
     off = align256(off + (size_t)scale_ld(s.T) * (s.d / 128) * 4);
+    L.sc_rows = off;
+    off = align256(off + (size_t)s.T * s.K * ((s.d / 128 + 7) / 8 * 8) * 4);
   }
   if (s.dtype == MOE_DTYPE_BF16) {
     L.arrive = off;

@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "fp8_util.cuh"
@@ -182,12 +184,18 @@ __global__ void __launch_bounds__(256) scatter_gather_kernel(
 
 // E4M3 layer: slots as above, then each x row is quantised once per 1x128
 // tile (a half-warp per tile) and its codes and scales are written to the
-// token's K destination rows (scales block-major: [d/128][sc_ld]).
+// token's K destination rows.  Scales: kStaged writes each destination row's
+// scales contiguously into sc_rows ([T*K][sc_stride], eight tiles per pass as
+// two 16-byte stores) for scale_rows_to_blocks_kernel to lay out block-major;
+// otherwise they go straight to the block-major [d/128][sc_ld] array, one
+// 4-byte store per tile and destination row.
+template <bool kStaged>
 __global__ void __launch_bounds__(256) scatter_gather_fp8_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ chunk_base, int T, int d, int K, int N,
     int32_t* __restrict__ perm_tok, int32_t* __restrict__ slot, uint8_t* __restrict__ x_perm,
-    float* __restrict__ x_perm_scales, long long sc_ld) {
+    float* __restrict__ x_perm_scales, long long sc_ld, float* __restrict__ sc_rows,
+    int sc_stride) {
   __shared__ int sidx[kChunkTokens * kMaxK];
   __shared__ int sslot[kChunkTokens * kMaxK];
   const int c = blockIdx.x;
@@ -210,21 +218,71 @@ __global__ void __launch_bounds__(256) scatter_gather_fp8_kernel(
         if (tc < tiles)
           bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(src + tc * QB) + l16), v[j]);
       }
+      float scs[kUnroll];  // this half-warp's tile scales (every lane of the half holds them)
 #pragma unroll
       for (int j = 0; j < kUnroll; ++j) {
         const int tc = tc0 + 2 * j + half;
         uint2 codes;
-        const float sc = quant_tile_16lanes(v[j], codes);  // both halves take part
+        scs[j] = quant_tile_16lanes(v[j], codes);  // both halves take part
         if (tc >= tiles) continue;
         for (int k = 0; k < K; ++k) {
           const int r = sslot[tl * K + k];
           if (r < 0) continue;
           *reinterpret_cast<uint2*>(x_perm + (size_t)r * d + tc * QB + 8 * l16) = codes;
-          if (l16 == 0) x_perm_scales[(size_t)tc * sc_ld + r] = sc;
+          if (!kStaged && l16 == 0) x_perm_scales[(size_t)tc * sc_ld + r] = scs[j];
+        }
+      }
+      if constexpr (kStaged) {
+        // lane 0 writes the pass's eight scales (tiles tc0..tc0+7, half 0 holding
+        // the even ones, half 1 the odd ones) of every destination row; entries
+        // past the last tile land in the row's padding
+        float odd[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) odd[j] = __shfl_sync(0xffffffffu, scs[j], 16);
+        if (lane == 0) {
+          for (int k = 0; k < K; ++k) {
+            const int r = sslot[tl * K + k];
+            if (r < 0) continue;
+            float4* dst = reinterpret_cast<float4*>(sc_rows + (size_t)r * sc_stride + tc0);
+            dst[0] = make_float4(scs[0], odd[0], scs[1], odd[1]);
+            dst[1] = make_float4(scs[2], odd[2], scs[3], odd[3]);
+          }
         }
       }
     }
   }
+}
+
+// sc_rows [rows][stride] -> out [tiles][ld] (block-major), 32 x 32 tiles
+// through shared memory.
+__global__ void __launch_bounds__(256) scale_rows_to_blocks_kernel(
+    const float* __restrict__ rows, int stride, long long nrows, int tiles,
+    float* __restrict__ out, long long ld) {
+  __shared__ float t[32][33];
+  const long long r0 = (long long)blockIdx.x * 32;
+  const int c0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const long long r = r0 + i;
+    const int c = c0 + threadIdx.x;
+    t[i][threadIdx.x] = (r < nrows && c < tiles) ? rows[r * stride + c] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i;
+    const long long r = r0 + threadIdx.x;
+    if (c < tiles && r < nrows) out[(long long)c * ld + r] = t[threadIdx.x][i];
+  }
+}
+
+// MOE_FP8_SCALES=direct writes the dispatch's E4M3 scales straight to the
+// block-major array (read once per process); the default stages them per row
+bool fp8_scales_direct() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("MOE_FP8_SCALES");
+    v = (e != nullptr && std::strcmp(e, "direct") == 0) ? 1 : 0;
+  }
+  return v == 1;
 }
 
 }  // namespace
@@ -250,10 +308,24 @@ cudaError_t launch_dispatch(const moe_shape& s, const void* x, const int32_t* id
     scatter_gather_kernel<__nv_bfloat16><<<nch, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
         slot, static_cast<__nv_bfloat16*>(x_perm));
-  else
-    scatter_gather_fp8_kernel<<<nch, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
-        slot, static_cast<uint8_t*>(x_perm), x_perm_scales, scale_ld((long long)s.T * s.K));
+  else {
+    const long long TK = (long long)s.T * s.K;
+    const int tiles = s.d / QB;
+    const int stride = (tiles + 7) / 8 * 8;
+    float* sc_rows = reinterpret_cast<float*>(w + L.sc_rows);
+    if (fp8_scales_direct()) {
+      scatter_gather_fp8_kernel<false><<<nch, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
+          slot, static_cast<uint8_t*>(x_perm), x_perm_scales, scale_ld(TK), nullptr, stride);
+    } else {
+      scatter_gather_fp8_kernel<true><<<nch, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), idx, chunk_base, s.T, s.d, s.K, s.N, perm_tok,
+          slot, static_cast<uint8_t*>(x_perm), x_perm_scales, scale_ld(TK), sc_rows, stride);
+      scale_rows_to_blocks_kernel<<<dim3((unsigned)((TK + 31) / 32), (unsigned)((tiles + 31) / 32)),
+                                    dim3(32, 8), 0, st>>>(sc_rows, stride, TK, tiles,
+                                                          x_perm_scales, scale_ld(TK));
+    }
+  }
   return cudaGetLastError();
 }
 

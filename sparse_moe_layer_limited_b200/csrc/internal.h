@@ -30,6 +30,7 @@ struct WsLayout {
   size_t xq = 0;          // E4M3 codes of x for the shared expert [T, d]
   size_t xq_scales = 0;   // fp32 block-major [d/128, scale_ld(T)]
   size_t arrive = 0;      // int32 [T, d/256] arrival counters of the fused combine (BF16)
+  size_t sc_rows = 0;     // fp32 [T*K, round8(d/128)] dispatch scales by row (E4M3)
   size_t total = 0;
 };
 WsLayout ws_layout(const moe_shape& s);

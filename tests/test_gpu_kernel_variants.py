@@ -55,3 +55,30 @@ def test_fp8_epilogue_variant(kind):
     tail = (r.stdout + r.stderr)[-3000:]
     assert r.returncode == 0, tail
     assert " passed" in r.stdout and "failed" not in r.stdout, tail
+
+
+def test_fp8_dispatch_direct_scales():
+    """MOE_FP8_SCALES=direct: the dispatch writes its E4M3 scales straight to
+    the block-major array instead of staging them per row; the FP8 layer
+    parity tests (codes and scales bit-exact) rerun with it."""
+    env = dict(os.environ, MOE_FP8_SCALES="direct")
+    cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+           os.path.join(HERE, "test_gpu_parity.py"), "-k", "small_fp8"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    tail = (r.stdout + r.stderr)[-3000:]
+    assert r.returncode == 0, tail
+    assert " passed" in r.stdout and "failed" not in r.stdout, tail
+
+
+@pytest.mark.parametrize("kind", ["wide", "narrow"])
+def test_fp8_weight_gradient_shapes(kind):
+    """MOE_FP8_WGRAD_EPI: the FP8 weight-gradient kernel on 256-column tiles
+    (eight or sixteen epilogue warps) instead of the default 128-column tiles;
+    the FP8 weight-gradient parity test reruns with each."""
+    env = dict(os.environ, MOE_FP8_WGRAD_EPI=kind)
+    cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+           os.path.join(HERE, "test_gpu_fp8_backward.py"), "-k", "dw"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    tail = (r.stdout + r.stderr)[-3000:]
+    assert r.returncode == 0, tail
+    assert " passed" in r.stdout and "failed" not in r.stdout, tail
