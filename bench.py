@@ -251,7 +251,12 @@ def main():
         return run_reference(args, cfg)
     if args.only == "backward_fp8":
         import torch
-        out = run_backward_fp8(BY_NAME["v3_fp8"], torch.device("cuda"), calls=max(1, args.steps),
+        c8 = BY_NAME["v3_fp8"]
+        if args.T:
+            c8 = c8.with_(T=args.T)
+        if args.N:
+            c8 = c8.with_(N=args.N)
+        out = run_backward_fp8(c8, torch.device("cuda"), calls=max(1, args.steps),
                                warmup=args.warmup)
         print(json.dumps({"backward_fp8": out}), flush=True)
         return out

@@ -22,51 +22,102 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
+
+#include "epilogue.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int GBM = 128, GBN = 256, GBK = 128;  // gradient tile rows, columns; K slice
-constexpr int GStages = 4;
-constexpr int GABytes = GBM * GBK;              // 16 KB (one byte per element)
-constexpr int GBBytes = GBN * GBK;              // 32 KB
-constexpr int GStageBytes = GABytes + GBBytes;
-constexpr int GThreads = 576;                   // warp 0 TMA, warp 1 MMA, warps 2-17 epilogue
-constexpr int GEpiWarps = 16;
+constexpr int GBM = 128, GBK = 128;  // gradient tile rows; K slice (one scale tile)
+constexpr int GABytes = GBM * GBK;   // 16 KB (one byte per element)
+// warp 0 TMA, warp 1 MMA, then kEpiW epilogue warps (kEpiW / 4 per TMEM lane quadrant)
+__host__ __device__ constexpr int wgrad_threads(int epi_warps) { return 64 + 32 * epi_warps; }
 constexpr int GScaleSlots = 8;
-constexpr int GScaleSlotBytes = (GBM + GBN) * 4;  // row scales, then column scales
-constexpr size_t GSmemBytes = 1024 + (size_t)GStages * GStageBytes +
-                              (size_t)GScaleSlots * GScaleSlotBytes + 512;
-static_assert(GSmemBytes <= 232448, "FP8 weight-gradient kernel exceeds the shared memory");
 constexpr uint64_t GTimeoutNs = 2000000000ull;
+
+// Tile configuration by gradient-tile width kBN (256 or 128 columns): the 512
+// TMEM columns hold 512 / kBN slice buffers, so a narrower tile gives the MMA
+// more slices of slack and each epilogue thread fewer running sums
+// The 128-column tiles store their gradient through shared memory by TMA
+// (eight epilogue warps, one 32-row x 64-column 128B-swizzled staging buffer
+// each); the 256-column tiles store rows directly.
+template <int kBN>
+struct WgTile {
+  static constexpr int kBufs = 512 / kBN;
+  static constexpr int kBBytes = kBN * GBK;
+  static constexpr int kStageBytes = GABytes + kBBytes;
+  static constexpr bool kTmaStore = kBN == 128;
+  static constexpr int kStages = kBN == 256 ? 4 : 5;
+  static constexpr int kStgBytes = kTmaStore ? 8 * 32 * 128 : 0;  // all epilogue warps
+  static constexpr int kScaleSlotBytes = (GBM + kBN) * 4;  // row scales, then column scales
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kStgBytes +
+                                       (size_t)GScaleSlots * kScaleSlotBytes + 512;
+  static_assert(kSmemBytes <= 232448, "FP8 weight-gradient kernel exceeds the shared memory");
+};
 
 struct alignas(64) Fp8WgradArgs {
   CUtensorMap tmL;   // left codes [M_total, R] E5M2 (the gradient), box {128, 128}
-  CUtensorMap tmR;   // right codes [N_total, R] E4M3 (the activation), box {128, 256}
+  CUtensorMap tmR;   // right codes [N_total, R] E4M3 (the activation), box {128, kBN}
   CUtensorMap tmSL;  // left scales [R/128, ld] fp32, box {128, 1}
-  CUtensorMap tmSR;  // right scales [R/128, ld] fp32, box {256, 1}
+  CUtensorMap tmSR;  // right scales [R/128, ld] fp32, box {kBN, 1}
+  CUtensorMap tmOut; // gradient [G1 * M_total, N_total] bf16, box {64, 32}, 128B swizzle
   const int32_t* colbase;  // [G1 + 1] column block of each group, multiples of 128
   __nv_bfloat16* out;      // [G1, M_total, N_total]
   uint32_t* status;
   int G1, M_total, N_total;
 };
 
-__global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
+// {m0, m1} = {a0 * s, a1 * s} as one packed fp32x2 multiply
+__device__ __forceinline__ void fmul2_s(float& m0, float& m1, float a0, float a1, float s) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "mul.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(m0), "=f"(m1)
+      : "f"(a0), "f"(a1), "f"(s));
+}
+// {acc0, acc1} += {x0 * s0, x1 * s1} as one packed fp32x2 fused multiply-add
+__device__ __forceinline__ void ffma2_v(float& acc0, float& acc1, float x0, float x1, float s0,
+                                       float s1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "f"(x0), "f"(x1), "f"(s0), "f"(s1));
+}
+
+// kBN-column gradient tiles; kEpiW epilogue warps, each reading its slice
+// columns 16 at a time with kInFlight TMEM loads per wait
+template <int kBN, int kEpiW, int kInFlight>
+__global__ void __launch_bounds__(wgrad_threads(kEpiW), 1) fp8_wgrad_kernel(
     const __grid_constant__ Fp8WgradArgs args) {
+  static_assert(kEpiW == 16 || kEpiW == 8, "four or two epilogue warps per lane quadrant");
+  using C = WgTile<kBN>;
+  static_assert(!C::kTmaStore || kEpiW == 8, "one staging buffer per epilogue warp, eight warps");
+  constexpr int GBN = kBN;
+  constexpr int GStages = C::kStages;
+  constexpr int GStageBytes = C::kStageBytes;
+  constexpr int GScaleSlotBytes = C::kScaleSlotBytes;
+  constexpr int kBufs = C::kBufs;
+  constexpr int GEpiWarps = kEpiW;
+  constexpr int kSub = kEpiW / 4;      // epilogue warps per lane quadrant
+  constexpr int kCols = GBN / kSub;    // gradient columns per warp
+  constexpr int kLoads = kCols / 16;
+  static_assert(kLoads % kInFlight == 0, "loads split evenly into waits");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* sc_ring = reinterpret_cast<float*>(base + (size_t)GStages * GStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)GStages * GStageBytes +
+  uint8_t* staging = base + (size_t)GStages * GStageBytes;  // 1024-aligned (stage sizes)
+  float* sc_ring = reinterpret_cast<float*>(staging + C::kStgBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + C::kStgBytes +
                                                (size_t)GScaleSlots * GScaleSlotBytes);
   uint64_t* full = bars;                       // [GStages]
   uint64_t* empty = full + GStages;            // [GStages]
-  uint64_t* sfull = empty + GStages;           // [2] slice buffer written
-  uint64_t* sempty = sfull + 2;                // [2] slice buffer drained (16 warps)
-  uint64_t* scfull = sempty + 2;               // [GScaleSlots] scale slot landed
-  uint64_t* scempty = scfull + GScaleSlots;    // [GScaleSlots] scale slot read (16 warps)
+  uint64_t* sfull = empty + GStages;           // [kBufs] slice buffer written
+  uint64_t* sempty = sfull + kBufs;            // [kBufs] slice buffer drained (epilogue warps)
+  uint64_t* scfull = sempty + kBufs;           // [GScaleSlots] scale slot landed
+  uint64_t* scempty = scfull + GScaleSlots;    // [GScaleSlots] scale slot read (epilogue warps)
   uint64_t* drain = scempty + GScaleSlots;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -79,7 +130,7 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kBufs; ++a) {
       mbar_init(&sfull[a], 1);
       mbar_init(&sempty[a], GEpiWarps);
     }
@@ -91,7 +142,7 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 2 * GBN);
+    tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -168,7 +219,7 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
         int g, m, n, kb0, kcnt;
         decode(u, g, m, n, kb0, kcnt);
         for (int kb = 0; kb < kcnt; ++kb, ++slice) {
-          const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
+          const uint32_t sb = slice % kBufs, sph = (slice / kBufs) & 1u;
           if (!mbar_wait_bounded(&sempty[sb], sph ^ 1u, args.status, GTimeoutNs) ||
               !mbar_wait_bounded(&full[stage], phase, args.status, GTimeoutNs)) {
             ok = false;
@@ -193,8 +244,8 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
       mbar_wait_bounded(drain, 0, args.status, GTimeoutNs / 8);
     }
   } else {
-    // warps 2..17: warp w reads TMEM lanes 32*(w%4)..+31; the four warps of a
-    // quadrant own the 64 columns 64*sub.. of the tile
+    // warps 2..kEpiW+1: warp w reads TMEM lanes 32*(w%4)..+31; the kSub warps
+    // of a quadrant own the kCols columns kCols*sub.. of the tile
     const int q = warp & 3;
     const int sub = (warp - 2) >> 2;
     const int row = q * 32 + lane;
@@ -203,11 +254,11 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       int g, m, n, kb0, kcnt;
       decode(u, g, m, n, kb0, kcnt);
-      float acc[64];
+      float acc[kCols];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
       for (int kb = 0; kb < kcnt; ++kb, ++slice) {
-        const uint32_t sb = slice & 1u, sph = (slice >> 1) & 1u;
+        const uint32_t sb = slice % kBufs, sph = (slice / kBufs) & 1u;
         const uint32_t cs = slice % GScaleSlots, cph = (slice / GScaleSlots) & 1u;
         if (!mbar_wait_bounded(&scfull[cs], cph, args.status, GTimeoutNs) ||
             !mbar_wait_bounded(&sfull[sb], sph, args.status, GTimeoutNs)) {
@@ -217,17 +268,29 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
         tc_fence_after();
         const float* slot = sc_ring + cs * (GScaleSlotBytes / 4);
         const float s_row = slot[row];
-        const float* s_col = slot + GBM + 64 * sub;
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * GBN + 64 * sub;
+        const float* s_col = slot + GBM + kCols * sub;
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * GBN + kCols * sub;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t p[16];
-          tmem_ld16(taddr + 16 * c, p);
+        for (int c0 = 0; c0 < kLoads; c0 += kInFlight) {
+          uint32_t p[kInFlight][16];
+#pragma unroll
+          for (int j = 0; j < kInFlight; ++j) tmem_ld16(taddr + 16 * (c0 + j), p[j]);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            acc[16 * c + i] = fmaf(__uint_as_float(p[i]), s_row * s_col[16 * c + i],
-                                   acc[16 * c + i]);
+          for (int j = 0; j < kInFlight; ++j) {
+            const int c = c0 + j;
+            // pairs of columns: their two scale products by one packed multiply,
+            // then one packed fused multiply-add (two round-to-nearest fp32 ops
+            // each, the same results as the scalar fmul and fmaf)
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              const float2 sc = *reinterpret_cast<const float2*>(s_col + 16 * c + i);
+              float m0, m1;
+              fmul2_s(m0, m1, sc.x, sc.y, s_row);
+              ffma2_v(acc[16 * c + i], acc[16 * c + i + 1], __uint_as_float(p[j][i]),
+                      __uint_as_float(p[j][i + 1]), m0, m1);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -238,36 +301,96 @@ __global__ void __launch_bounds__(GThreads, 1) fp8_wgrad_kernel(
       }
       if (!ok) break;
       // an expert without rows stores zeros
-      __nv_bfloat16* orow = args.out +
-                            ((size_t)g * args.M_total + (size_t)m * GBM + row) * args.N_total +
-                            (size_t)n * GBN + 64 * sub;
+      if constexpr (C::kTmaStore) {
+        // 64-column pieces: bf16 into this warp's swizzled staging buffer (the
+        // 16-byte chunks of row `lane` XOR-permuted like the TMA's 128-byte
+        // swizzle), then one TMA store of 32 rows x 64 columns
+        uint8_t* stg = staging + (size_t)(warp - 2) * (32 * 128);
+        const int grow = g * args.M_total + m * GBM + q * 32;
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        uint4 w;
-        __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&w);
+        for (int c = 0; c < kCols; c += 64) {
+          if (lane == 0) bulk_wait_read_all();  // the previous piece has left the buffer
+          __syncwarp();
+          uint8_t* my_row = stg + lane * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          hb[i] = __floats2bfloat162_rn(acc[8 * v + 2 * i], acc[8 * v + 2 * i + 1]);
-        reinterpret_cast<uint4*>(orow)[v] = w;
+          for (int jj = 0; jj < 8; ++jj) {
+            const float* a8 = acc + c + 8 * jj;
+            *reinterpret_cast<uint4*>(my_row + ((jj ^ (lane & 7)) << 4)) =
+                make_uint4(bf16x2_bits(a8[0], a8[1]), bf16x2_bits(a8[2], a8[3]),
+                           bf16x2_bits(a8[4], a8[5]), bf16x2_bits(a8[6], a8[7]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&args.tmOut, stg, n * GBN + kCols * sub + c, grow);
+            bulk_commit_group();
+          }
+        }
+      } else {
+        __nv_bfloat16* orow = args.out +
+                              ((size_t)g * args.M_total + (size_t)m * GBM + row) * args.N_total +
+                              (size_t)n * GBN + kCols * sub;
+#pragma unroll
+        for (int v = 0; v < kCols / 8; ++v) {
+          uint4 w;
+          __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            hb[i] = __floats2bfloat162_rn(acc[8 * v + 2 * i], acc[8 * v + 2 * i + 1]);
+          reinterpret_cast<uint4*>(orow)[v] = w;
+        }
       }
+    }
+    if constexpr (C::kTmaStore) {
+      if (lane == 0) bulk_wait_all();  // every store has completed before the CTA exits
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * GBN);
+    tmem_dealloc(tmem_base, 512);
   }
 }
 
-cudaError_t launch_fp8_wgrad(const Fp8WgradArgs& a, cudaStream_t st) {
-  cudaError_t e = note_cuda(cudaFuncSetAttribute(fp8_wgrad_kernel,
+template <int kBN, int kEpiW, int kInFlight>
+cudaError_t launch_fp8_wgrad_w(const Fp8WgradArgs& a, cudaStream_t st) {
+  auto kernel = fp8_wgrad_kernel<kBN, kEpiW, kInFlight>;
+  constexpr size_t smem = WgTile<kBN>::kSmemBytes;
+  cudaError_t e = note_cuda(cudaFuncSetAttribute(kernel,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)GSmemBytes),
+                                                 (int)smem),
                             "fp8 weight-gradient GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
-  fp8_wgrad_kernel<<<num_sms(), GThreads, GSmemBytes, st>>>(a);
+  kernel<<<num_sms(), wgrad_threads(kEpiW), smem, st>>>(a);
   return note_cuda(cudaGetLastError(), "fp8 weight-gradient GEMM launch");
+}
+
+// Gradient tile and epilogue shape, chosen once per process by
+// MOE_FP8_WGRAD_EPI:
+//   unset   128-column tiles, four slice buffers, eight epilogue warps with all
+//           four 16-column loads of a slice in flight (64 running sums a thread)
+//   wide    256-column tiles, two slice buffers, eight warps, one load in flight
+//           (128 running sums a thread)
+//   narrow  256-column tiles, sixteen warps, one load in flight
+int fp8_wgrad_kind() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("MOE_FP8_WGRAD_EPI");
+    v = 0;
+    if (e != nullptr && std::strcmp(e, "wide") == 0) v = 1;
+    if (e != nullptr && std::strcmp(e, "narrow") == 0) v = 2;
+  }
+  return v;
+}
+int fp8_wgrad_tile_cols() { return fp8_wgrad_kind() == 0 ? 128 : 256; }
+
+cudaError_t launch_fp8_wgrad(const Fp8WgradArgs& a, cudaStream_t st) {
+  switch (fp8_wgrad_kind()) {
+    case 1: return launch_fp8_wgrad_w<256, 8, 1>(a, st);
+    case 2: return launch_fp8_wgrad_w<256, 16, 1>(a, st);
+    default: return launch_fp8_wgrad_w<128, 8, 4>(a, st);
+  }
 }
 
 }  // namespace
@@ -311,6 +434,7 @@ int launch_ffn_bwd_dw_e4m3(const moe_shape& s, const int32_t* perm_tok, const in
 
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t KT = (uint64_t)(R / GBK);
+  const uint32_t GBN = (uint32_t)fp8_wgrad_tile_cols();
   // dW2_e [d, f] = dYT_e HT_e^T
   Fp8WgradArgs a2{};
   bool ok = make_map(&a2.tmL, w + B.dytq, U8, 1, R, s.d, GBK, GBM) &&
@@ -323,6 +447,10 @@ int launch_ffn_bwd_dw_e4m3(const moe_shape& s, const int32_t* perm_tok, const in
        make_map(&a13.tmR, w + B.atq, U8, 1, R, s.d, GBK, GBN) &&
        make_map_f32_rows(&a13.tmSL, f32(B.dguts), ld_2f, KT, GBM) &&
        make_map_f32_rows(&a13.tmSR, f32(B.ats), ld_d, KT, GBN);
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t G1 = (uint64_t)s.N + 1;
+  ok = ok && make_map(&a2.tmOut, dw2, BF, 2, s.f, G1 * s.d, 64, 32) &&
+       make_map(&a13.tmOut, dw13, BF, 2, s.d, G1 * twof, 64, 32);
   if (!ok) {
     note_text("fp8 weight-gradient GEMM: tensor-map encoding failed");
     return MOE_ERR_CUDA;
