@@ -310,6 +310,8 @@ def main():
         }
         if r.get("softmax_route"):
             line["softmax_route"] = r["softmax_route"]
+        if r.get("graph"):
+            line["graph_replay"] = r["graph"]
         for k, v in extra.items():
             line[k] = {"workload": workload_name(v["cfg"]),
                        "value": world * v["cfg"].T * v["steps"] / (v["total_ms"] / 1e3),
@@ -660,6 +662,27 @@ def run_layer_backward(cfg, dev, calls=10, warmup=3):
     return out
 
 
+def graph_step_timing(layer, x, steps, warmup=3):
+    """The same layer step (route -> bias update) captured in one CUDA graph
+    and replayed `steps` times after `warmup` replays, CUDA events around the
+    replays: the step without host launch overhead."""
+    import torch
+    layer.capture(x)
+    for _ in range(warmup):
+        layer.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        layer.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"ms_per_step": ms, "value": x.shape[0] / (ms / 1e3), "unit": "tokens/s",
+            "note": "one CUDA graph per step (route, dispatch, experts, combine, bias update), "
+                    "replayed back to back"}
+
+
 def softmax_route_baseline(M, s, x, router, layer, cfg, stream, reps=20):
     """The conventional softmax top-K router (moe_route_softmax) on the same
     input, for contrast with the method's routing: time per call (CUDA events,
@@ -817,10 +840,12 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
 
     e2e_ms = None
     baseline = None
+    graph = None
     if e2e:
         e2e_ms = run_e2e(M, s, layer, x, w13, w2, s13, s2, cfg, steps, stream)
         if cfg.dtype != "fp32":  # the softmax router takes bf16 activations
             baseline = softmax_route_baseline(M, s, x, router, layer, cfg, stream)
+        graph = graph_step_timing(layer, x, steps)
 
     total_ms, e2e_ms = reduce_max([total_ms, e2e_ms or 0.0], pg, dev)
 
@@ -896,7 +921,7 @@ def run_layer(cfg, dev, steps, warmup, pg, local, e2e=False):
             roof["traffic_note"] = ("bytes per experts phase (GEMM1 + GEMM2), ncu capture of "
                                     "this workload scaled by the experts hit")
     return {"cfg": cfg, "steps": steps, "total_ms": total_ms, "e2e_ms": e2e_ms,
-            "softmax_route": baseline,
+            "softmax_route": baseline, "graph": graph,
             "phases_ms": {p: statistics.mean(v) for p, v in per_phase.items()},
             "roofline": roof,
             "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step, "flops": fl, "bytes": by},

@@ -283,12 +283,15 @@ __global__ void __launch_bounds__(wgrad_threads(kEpiW), 1) fp8_wgrad_kernel(
             // then one packed fused multiply-add (two round-to-nearest fp32 ops
             // each, the same results as the scalar fmul and fmaf)
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              const float2 sc = *reinterpret_cast<const float2*>(s_col + 16 * c + i);
-              float m0, m1;
+            for (int i = 0; i < 16; i += 4) {
+              const float4 sc = *reinterpret_cast<const float4*>(s_col + 16 * c + i);
+              float m0, m1, m2, m3;
               fmul2_s(m0, m1, sc.x, sc.y, s_row);
+              fmul2_s(m2, m3, sc.z, sc.w, s_row);
               ffma2_v(acc[16 * c + i], acc[16 * c + i + 1], __uint_as_float(p[j][i]),
                       __uint_as_float(p[j][i + 1]), m0, m1);
+              ffma2_v(acc[16 * c + i + 2], acc[16 * c + i + 3], __uint_as_float(p[j][i + 2]),
+                      __uint_as_float(p[j][i + 3]), m2, m3);
             }
           }
         }
@@ -368,8 +371,9 @@ cudaError_t launch_fp8_wgrad_w(const Fp8WgradArgs& a, cudaStream_t st) {
 
 // Gradient tile and epilogue shape, chosen once per process by
 // MOE_FP8_WGRAD_EPI:
-//   unset   128-column tiles, four slice buffers, eight epilogue warps with all
-//           four 16-column loads of a slice in flight (64 running sums a thread)
+//   unset   128-column tiles, four slice buffers, eight epilogue warps with two
+//           16-column loads in flight (64 running sums a thread; four in
+//           flight measured the same and spills)
 //   wide    256-column tiles, two slice buffers, eight warps, one load in flight
 //           (128 running sums a thread)
 //   narrow  256-column tiles, sixteen warps, one load in flight
@@ -389,7 +393,7 @@ cudaError_t launch_fp8_wgrad(const Fp8WgradArgs& a, cudaStream_t st) {
   switch (fp8_wgrad_kind()) {
     case 1: return launch_fp8_wgrad_w<256, 8, 1>(a, st);
     case 2: return launch_fp8_wgrad_w<256, 16, 1>(a, st);
-    default: return launch_fp8_wgrad_w<128, 8, 4>(a, st);
+    default: return launch_fp8_wgrad_w<128, 8, 2>(a, st);
   }
 }
 

@@ -143,6 +143,30 @@ class MoELayer:
                                 stream)
         return out
 
+    def capture(self, x, update_bias: bool = True):
+        """Record one forward (route, dispatch, experts, combine and, with
+        update_bias, the bias update) on the buffer x into a CUDA graph, so
+        that replay() reruns the whole step with one launch from the host.
+        One eager forward runs first (it also moves the bias once) so that
+        every launch-time set-up happens outside the capture.  The graph keeps
+        x's address: copy each new batch into x before replay().  Returns the
+        graph."""
+        side = torch.cuda.Stream(x.device)
+        side.wait_stream(torch.cuda.current_stream(x.device))
+        with torch.cuda.stream(side):
+            self.forward(x, update_bias)
+        torch.cuda.current_stream(x.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(x, update_bias)
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        """Rerun the captured step; returns self.y."""
+        self._graph.replay()
+        return self.y
+
     def backward_status(self, clear: bool = False) -> int:
         """Status word of the backward workspace (0 = no device-side problem)."""
         B = getattr(self, "_bwd", None)
