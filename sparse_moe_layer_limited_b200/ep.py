@@ -25,7 +25,8 @@ the layer:
 Inside one NVSwitch node every peer is reached at the same bandwidth, so the
 group limit constrains nothing here; it stays part of the routing rule.
 
-The exchange uses torch.distributed collectives (NCCL between GPUs).  The
+The exchange uses torch.distributed collectives (NCCL between GPUs; with
+gloo, device tensors are staged through host memory).  The
 per-rank computation is behind a small operations interface: the library's
 CUDA kernels (``LibraryOps``) on the product path.  The host-side planning
 (send splits, the regroup tables) is plain integer work in NumPy.
@@ -181,6 +182,28 @@ def local_shape(shape, W: int):
     return L.shape(shape.T, shape.d, n, k, 1, 1, shape.f, shape.dtype)
 
 
+def _all_to_all(dist, group, out, inp, out_splits=None, in_splits=None):
+    """all_to_all_single; with a backend that exchanges host memory only
+    (gloo), device tensors go through host copies."""
+    if inp.is_cuda and dist.get_backend(group) == "gloo":
+        o = torch.empty(out.shape, dtype=out.dtype)
+        dist.all_to_all_single(o, inp.cpu(), output_split_sizes=out_splits,
+                               input_split_sizes=in_splits, group=group)
+        out.copy_(o)
+        return
+    dist.all_to_all_single(out, inp, output_split_sizes=out_splits, input_split_sizes=in_splits,
+                           group=group)
+
+
+def _all_reduce(dist, group, t):
+    if t.is_cuda and dist.get_backend(group) == "gloo":
+        h = t.cpu()
+        dist.all_reduce(h, group=group)
+        t.copy_(h)
+        return
+    dist.all_reduce(t, group=group)
+
+
 class ExpertParallelMoE:
     """One rank of the expert-parallel layer.  `ops` carries the per-rank
     steps (the library's kernels by default: ``LibraryOps``); `group` is the
@@ -202,21 +225,19 @@ class ExpertParallelMoE:
         counts, x_perm = ops.route_dispatch(x)
         # per-expert counts: rank r's counts of rank q's experts go to q
         cnt = torch.empty_like(counts)
-        dist.all_to_all_single(cnt, counts, group=self.group)
+        _all_to_all(dist, self.group, cnt, counts)
         cnt_h = cnt.cpu().numpy().reshape(W, -1)
         sends = send_splits(counts.cpu().numpy(), W)
         plan = regroup_plan(cnt_h)
         self.last_plan = plan
         R = ops.set_plan(plan)
         n_send = sum(sends)
-        dist.all_to_all_single(ops.recv[:R], x_perm[:n_send], output_split_sizes=plan["recv_splits"],
-                               input_split_sizes=sends, group=self.group)
+        _all_to_all(dist, self.group, ops.recv[:R], x_perm[:n_send], plan["recv_splits"], sends)
         y_back = ops.experts(R, x)
-        dist.all_to_all_single(ops.y_perm[:n_send], y_back[:R], output_split_sizes=sends,
-                               input_split_sizes=plan["recv_splits"], group=self.group)
+        _all_to_all(dist, self.group, ops.y_perm[:n_send], y_back[:R], sends, plan["recv_splits"])
         y = ops.combine()
         if update_bias:
             counts_all = counts.clone()
-            dist.all_reduce(counts_all, group=self.group)
+            _all_reduce(dist, self.group, counts_all)
             ops.bias_update(counts_all, x.shape[0] * W, self.gamma)
         return y

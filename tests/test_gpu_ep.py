@@ -4,9 +4,20 @@ expert-parallel forward on one rank.
 With one rank (NCCL, world size 1) every collective is a copy to itself and
 the regroup is the identity, so ExpertParallelMoE over the library's kernels
 must reproduce MoELayer's output and bias bit for bit; this runs every
-kernel and every collective call of the expert-parallel path.  The exchange
-between two ranks is covered on CPU (tests/test_ep_cpu.py)."""
+kernel and every collective call of the expert-parallel path.
+
+With two ranks, two processes share the GPU and exchange through gloo: the
+collectives run on the host, so no kernel of one rank ever waits on the
+other's.  Each rank holds half of the routed experts; every row an expert
+receives is computed by the same kernel as in the single-GPU layer, so each
+rank's output must equal MoELayer's on that rank's batch bit for bit, the
+regroup sends every row to exactly one rank, and both ranks end with the
+bias the oracle's update gives for the two batches' summed counts.  The
+exchange between ranks is also covered on CPU against the oracle
+(tests/test_ep_cpu.py)."""
+import os
 import socket
+import sys
 
 import numpy as np
 import pytest
@@ -72,3 +83,88 @@ def test_expert_parallel_single_rank_equals_layer():
         assert M.moe_read_device_status(ops.ws_loc) == 0
     finally:
         dist.destroy_process_group()
+
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _two_rank_worker(rank, world, port, dtype, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import sparse_moe_layer_limited_b200 as M
+    from sparse_moe_layer_limited_b200 import ep
+    from synth import CONFIGS, gen
+    from tests import support as S
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        cfg = CONFIGS[1].with_(T=300, d=256, N=16, K=4, G=4, topG=2, f=256, dtype=dtype)
+        R, b = gen.make_router(cfg), gen.make_bias(cfg)
+        x, _ = S.tie_free_x(cfg, R, b, batch=rank)          # each rank its own batch
+        W = S.device_weights(cfg)
+        s = S.moe_shape(cfg)
+        Rd = torch.from_numpy(R).cuda()
+        bd = torch.from_numpy(np.asarray(b, np.float32)).cuda()
+        lo, hi = ep.expert_range(cfg.N, world, rank)
+        keep = list(range(lo, hi)) + [cfg.N]                # this rank's experts + shared
+        w13 = W["w13"][keep].contiguous()
+        w2 = W["w2"][keep].contiguous()
+        ops = ep.LibraryOps(s, ep.local_shape(s, world), Rd, bd.clone(), w13, w2)
+        epl = ep.ExpertParallelMoE(ops, cfg.N, gamma=cfg.gamma)
+        layer = M.MoELayer(s, Rd, bd.clone(), W["w13"], W["w2"], gamma=cfg.gamma)
+        xd = S.to_dev_x(x, cfg)
+        out = dict(equal=[], recv=[], counts=None, bias=None)
+        for step in range(2):                 # step 1 routes with the updated bias
+            layer.bias.copy_(ops.bias)
+            y_ep = epl.forward(xd).clone()
+            y_ref = layer.forward(xd, update_bias=False).clone()
+            torch.cuda.synchronize()
+            out["equal"].append(bool(torch.equal(y_ep, y_ref)))
+            out["recv"].append(sum(epl.last_plan["recv_splits"]))
+            if step == 0:
+                out["counts"] = layer.counts.cpu().numpy().astype(np.int64)
+                out["bias"] = ops.bias.cpu().numpy()
+        out["status"] = [int(layer.device_status()), int(M.moe_read_device_status(ops.ws)),
+                         int(M.moe_read_device_status(ops.ws_loc))]
+        q.put((rank, out))
+    except Exception as e:  # report instead of leaving the parent's queue read to time out
+        q.put((rank, dict(error=repr(e))))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_expert_parallel_two_ranks_one_gpu(dtype):
+    import oracle
+    import torch.multiprocessing as mp
+    from synth import CONFIGS
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_two_rank_worker, args=(r, 2, port, dtype, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        res = dict(q.get(timeout=600) for _ in procs)
+    finally:
+        for p in procs:
+            p.join(timeout=120)
+    for r in (0, 1):
+        assert "error" not in res[r], res[r]
+        assert res[r]["equal"] == [True, True], res[r]["equal"]
+        assert res[r]["status"] == [0, 0, 0]
+    for p in procs:
+        assert p.exitcode == 0
+    cfg = CONFIGS[1].with_(T=300, d=256, N=16, K=4, G=4, topG=2, f=256, dtype=dtype)
+    for step in (0, 1):                               # every routed row went to one rank
+        assert res[0]["recv"][step] + res[1]["recv"][step] == 2 * cfg.T * cfg.K
+    b0 = gen.make_bias(cfg)
+    want_b = oracle.bias_update(b0, res[0]["counts"] + res[1]["counts"], 2 * cfg.T, cfg.K,
+                                cfg.gamma)
+    np.testing.assert_array_equal(res[0]["bias"], want_b)
+    np.testing.assert_array_equal(res[1]["bias"], want_b)
