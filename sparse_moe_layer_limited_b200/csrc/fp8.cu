@@ -164,6 +164,9 @@ struct alignas(64) Fp8Args {
   CUtensorMap tmB;
   CUtensorMap tmS_routed;  // activation scales [KB][ld] (row index as in tmA_routed), box {132, 1}
   CUtensorMap tmS_shared;  // the same for tmA_shared's rows
+  CUtensorMap tmY_routed;  // store epilogue: y_routed [rows_routed, out_ld] bf16, box {16, 32},
+  CUtensorMap tmY_shared;  // 32-byte swizzle; y_shared [T, out_ld] (built by the launcher)
+  int y_tma;               // 1: the maps above are valid
   const int32_t* offsets;
   const float* sw;         // [(N+1) * n_acc / 128, KB] weight block scales
   uint8_t* q_routed;       // GEMM1: h codes, row (offsets[g] + r)
@@ -185,9 +188,15 @@ struct alignas(64) Fp8Args {
   int out_ld;  // f (GEMM1 codes) or d (GEMM2)
 };
 
-constexpr size_t fp8_smem_bytes(int groups) {
-  return 1024 + (size_t)FStages * FStageBytes + (size_t)FScaleSlots * FScaleSlotBytes + 512 +
-         2 * 4 * FBM * 4 + (size_t)(groups + 1) * 4;
+// Store epilogue staging: per epilogue warp two 1 KB pieces (32 rows x 16
+// bf16 columns) in the TMA's 32-byte swizzle, one filled while the other is
+// being stored.
+constexpr int FStgPiece = 1024;
+constexpr int FStgBytes = 8 * 2 * FStgPiece;
+
+constexpr size_t fp8_smem_bytes(int groups, bool staging) {
+  return 1024 + (size_t)FStages * FStageBytes + (staging ? FStgBytes : 0) +
+         (size_t)FScaleSlots * FScaleSlotBytes + 512 + 2 * 4 * FBM * 4 + (size_t)(groups + 1) * 4;
 }
 
 // a0 += x0 * s and a1 += x1 * s as one packed fp32x2 FMA (two independent
@@ -213,11 +222,15 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
   constexpr int kCols = FBN / kSub;        // accumulator columns per warp
   constexpr int kFeat = (FBN / 2) / kSub;  // GEMM1: hidden features per warp
   static_assert((kCols / kLd) % (2 * kInFlight) == 0, "gate and up halves split evenly");
+  // the bf16 store epilogue writes full 32-row groups by TMA (eight-warp shape)
+  constexpr bool kTmaY = kEpi == kFEpiStore && kEpiW == 8;
+  constexpr size_t kStg = kTmaY ? FStgBytes : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* sc_ring = reinterpret_cast<float*>(base + (size_t)FStages * FStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)FStages * FStageBytes +
+  uint8_t* staging = base + (size_t)FStages * FStageBytes;  // 1024-aligned
+  float* sc_ring = reinterpret_cast<float*>(staging + kStg);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + kStg +
                                                (size_t)FScaleSlots * FScaleSlotBytes);
   uint64_t* full = bars;                  // [FStages]
   uint64_t* empty = bars + FStages;       // [FStages]
@@ -443,14 +456,14 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
         const float sA = sa * slot_sc[FScaleBox + wA], sB = sa * slot_sc[FScaleBox + wB];
         __syncwarp();
         if (lane == 0) mbar_arrive(&scempty[cs]);
+        // load c (kLd columns) of this warp: GEMM1 gate loads first, then up
+        constexpr int kLoads = kCols / kLd;
         if (!mbar_wait_bounded(&sfull[sb], sph, args.status, FTimeoutNs)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + sb * FBN;
-        // load c (kLd columns) of this warp: GEMM1 gate loads first, then up
-        constexpr int kLoads = kCols / kLd;
 #pragma unroll
         for (int c0 = 0; c0 < kLoads; c0 += kInFlight) {
           uint32_t p[kInFlight][kLd];
@@ -469,6 +482,13 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
               tmem_ld16(taddr + col, p[j]);
           }
           tmem_wait_ld();
+          if (c0 + kInFlight == kLoads) {
+            // the whole slice is in registers: hand the buffer back to the
+            // MMA before the last multiply-adds
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[sb]);
+          }
 #pragma unroll
           for (int j = 0; j < kInFlight; ++j) {
             const int c = c0 + j;
@@ -479,9 +499,6 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
                     __uint_as_float(p[j][i + 1]), sc);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[sb]);
       }
       if (!ok) break;
 
@@ -565,7 +582,42 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
           }
         }
       } else {
-        if (valid) {
+        // a warp whose 32 rows all lie inside the group stores them by TMA;
+        // the ragged last rows of a group take the row stores below
+        const int r0 = m * FBM + q * 32;
+        bool tma_rows = false;
+        if constexpr (kTmaY) {
+          tma_rows = args.y_tma != 0 && r0 + 32 <= rows_g &&
+                     (g == args.N || args.offsets[g] + r0 + 32 <= args.rows_routed);
+          if (tma_rows) {
+            uint8_t* stg = staging + (size_t)(warp - 2) * (2 * FStgPiece);
+            const CUtensorMap* ym = (g < args.N) ? &args.tmY_routed : &args.tmY_shared;
+            const int yrow = ((g < args.N) ? args.offsets[g] : 0) + r0;
+            const int ycol = n * FBN + kCols * sub;
+            const int sw = (lane >> 2) & 1;  // the 32-byte swizzle of row `lane`
+#pragma unroll
+            for (int c = 0; c < kCols / 16; ++c) {
+              uint8_t* buf = stg + (c & 1) * FStgPiece;
+              if (lane == 0) bulk_wait_read_but_one();  // this piece's buffer is free
+              __syncwarp();
+              uint8_t* my = buf + lane * 32;
+              const float* a = acc + 16 * c;
+              *reinterpret_cast<uint4*>(my + (sw << 4)) =
+                  make_uint4(bf16x2_bits(a[0], a[1]), bf16x2_bits(a[2], a[3]),
+                             bf16x2_bits(a[4], a[5]), bf16x2_bits(a[6], a[7]));
+              *reinterpret_cast<uint4*>(my + ((sw ^ 1) << 4)) =
+                  make_uint4(bf16x2_bits(a[8], a[9]), bf16x2_bits(a[10], a[11]),
+                             bf16x2_bits(a[12], a[13]), bf16x2_bits(a[14], a[15]));
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(ym, buf, ycol + 16 * c, yrow);
+                bulk_commit_group();
+              }
+            }
+          }
+        }
+        if (!tma_rows && valid) {
           __nv_bfloat16* yrow =
               ((g < args.N) ? args.y_routed + ((long long)args.offsets[g] + r) * args.out_ld
                             : args.y_shared + (long long)r * args.out_ld) +
@@ -582,6 +634,10 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
         }
       }
     }
+    // the staging buffers must outlive the stores that read them
+    if constexpr (kTmaY) {
+      if (lane == 0) bulk_wait_all();
+    }
   }
 
   tc_fence_before();
@@ -596,14 +652,31 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
 }
 
 template <int kEpi, int kEpiW, int kLd, int kInFlight>
-cudaError_t launch_fp8_gemm_w(const Fp8Args& a, cudaStream_t st) {
-  const size_t smem = fp8_smem_bytes(a.N + 1);
+cudaError_t launch_fp8_gemm_w(const Fp8Args& a0, cudaStream_t st) {
+  constexpr bool kTmaY = kEpi == kFEpiStore && kEpiW == 8;
+  const size_t smem = fp8_smem_bytes(a0.N + 1, kTmaY);
   auto kernel = grouped_gemm_fp8_kernel<kEpi, kEpiW, kLd, kInFlight>;
   cudaError_t e = note_cuda(cudaFuncSetAttribute(kernel,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem),
                             "fp8 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
+  Fp8Args a = a0;
+  a.y_tma = 0;
+  if constexpr (kTmaY) {
+    // TMA stores need 16-byte aligned outputs; otherwise every row takes the
+    // row stores
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const bool aligned = (reinterpret_cast<uintptr_t>(a.y_routed) % 16 == 0) &&
+                         (reinterpret_cast<uintptr_t>(a.y_shared) % 16 == 0) &&
+                         ((size_t)a.out_ld * 2) % 16 == 0;
+    if (aligned &&
+        make_map_swizzled(&a.tmY_routed, a.y_routed, BF, 2, a.out_ld, a.rows_routed, 16, 32,
+                          CU_TENSOR_MAP_SWIZZLE_32B) &&
+        make_map_swizzled(&a.tmY_shared, a.y_shared, BF, 2, a.out_ld, a.T, 16, 32,
+                          CU_TENSOR_MAP_SWIZZLE_32B))
+      a.y_tma = 1;
+  }
   kernel<<<num_sms(), fp8_threads(kEpiW), smem, st>>>(a);
   return note_cuda(cudaGetLastError(), "fp8 GEMM launch");
 }
@@ -618,7 +691,10 @@ cudaError_t launch_fp8_gemm_w(const Fp8Args& a, cudaStream_t st) {
 // spill more and measured slower.  The 18-warp CTA cannot have more registers:
 // compiled for 112 a thread, its launch is refused; a 20-warp CTA that moves
 // registers from its control warpgroup to the epilogue with setmaxnreg spills
-// the TMA and MMA loops instead, 0.6-0.8 KB a thread at 32-56 registers)
+// the TMA and MMA loops instead, 0.6-0.8 KB a thread at 32-56 registers.  A
+// 12-warp CTA with a 88/208 setmaxnreg split and four loads in flight, and a
+// ring of four 128-column slice buffers fed by N=128 MMAs, were both exact
+// and slower: the slice handshake, not the read shape, bounds the kernel)
 int fp8_epilogue_kind() {
   static int v = -1;
   if (v < 0) {

@@ -64,6 +64,10 @@ constexpr size_t kClockRecordOffset = 128;
 // 128-byte swizzle; out-of-range rows read as zero.
 bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t elem_bytes,
               uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows);
+// The same with a chosen swizzle and no L2 promotion (used for TMA stores).
+bool make_map_swizzled(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt,
+                       size_t elem_bytes, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                       uint32_t box_rows, CUtensorMapSwizzle swizzle);
 // `rank`-D tensor (2..5) given by its dims (innermost first), the byte strides of
 // dims 1..rank-1 and the box; 128-byte swizzle, out-of-range elements read as zero.
 bool make_map_nd(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int rank,

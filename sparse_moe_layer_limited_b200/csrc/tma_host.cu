@@ -39,6 +39,21 @@ bool make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, size_t 
   return r == CUDA_SUCCESS;
 }
 
+bool make_map_swizzled(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt,
+                       size_t elem_bytes, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                       uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_map_nd(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int rank,
                  const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
