@@ -5,7 +5,13 @@
 
 namespace moe {
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.f + expf(-v)); }
+// silu(v) = v / (1 + e^-v) with the hardware exponential and an approximate
+// divide (relative error ~1e-6, far below bf16 and E4M3 rounding): the
+// tensor-core epilogues evaluate it for every hidden feature on the path
+// between the MMA and the next tile.  For v below about -87, 1 + e^-v
+// overflows or passes 2^126 and the quotient is 0, where the exact value is
+// under 1e-36 in magnitude.
+__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
 // SwiGLU backward for one hidden feature: with dh the gradient of
 // h = silu(g) * u, dg = dh * u * silu'(g) (silu'(g) = s (1 + g (1 - s)),

@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(fp8_threads(kEpiW), 1) grouped_gemm_fp8_kernel
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < kFeat; ++i) {
-          acc[i] = silu_f(acc[i]) * acc[kFeat + i];
+          acc[i] = silu_fast(acc[i]) * acc[kFeat + i];
           amax = fmaxf(amax, fabsf(acc[i]));
         }
         // the row's 1x128 tile spans the kSub warps of this quadrant

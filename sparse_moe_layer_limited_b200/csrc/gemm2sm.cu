@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(PThreads, 1) pair_gemm_bf16_kernel(
             const float gt = up_lane ? other : __uint_as_float(v[k]);
             const float upv = up_lane ? __uint_as_float(v[8 + k]) : other;
             if (tb + k < U.ntok)
-              o[(long long)k * args.out_ld] = __float2bfloat16_rn(silu_f(gt) * upv);
+              o[(long long)k * args.out_ld] = __float2bfloat16_rn(silu_fast(gt) * upv);
           }
         } else {
           const int feat = U.nf * 2 * PW + PW * (int)rank + 32 * q + lane;

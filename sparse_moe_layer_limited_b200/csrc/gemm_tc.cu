@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           float h[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            h[i] = silu_f(__uint_as_float(ga[i])) * __uint_as_float(up[i]);
+            h[i] = silu_fast(__uint_as_float(ga[i])) * __uint_as_float(up[i]);
           if (valid) store_row32(orow + n * (BN / 2) + c, h);
         }
       } else if constexpr (kEpi == kEpiStore) {

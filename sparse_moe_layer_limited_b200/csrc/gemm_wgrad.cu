@@ -123,8 +123,8 @@ __global__ void __launch_bounds__(kTileThreads) transpose_groups_kernel(
         __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          h[e] = __floats2bfloat162_rn(silu_f(gt[2 * e]) * up[2 * e],
-                                       silu_f(gt[2 * e + 1]) * up[2 * e + 1]);
+          h[e] = __floats2bfloat162_rn(silu_fast(gt[2 * e]) * up[2 * e],
+                                       silu_fast(gt[2 * e + 1]) * up[2 * e + 1]);
       } else {
         v = __ldg(reinterpret_cast<const uint4*>(row + f0 + p * 8));
       }
