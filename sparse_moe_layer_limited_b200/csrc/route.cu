@@ -39,13 +39,36 @@ __device__ __forceinline__ bool better(float v, int i, float w, int j) {
   return v > w || (v == w && i < j);
 }
 
+// Unsigned keys in the order of the floats (NaN never occurs here); -0 is
+// taken as +0 first, so equal floats have equal keys.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// The warp's best (v, i) under `better` (largest v, then smallest i), on
+// every lane: two warp-wide reductions (max of the value keys, then min of
+// the indices holding that value).  i >= 0.
 __device__ __forceinline__ void warp_argmax(float& v, int& i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    float w = __shfl_xor_sync(0xffffffffu, v, o);
-    int j = __shfl_xor_sync(0xffffffffu, i, o);
-    if (better(w, j, v, i)) { v = w; i = j; }
-  }
+  const uint32_t k = order_key(v);
+  const uint32_t kmax = __reduce_max_sync(0xffffffffu, k);
+  i = (int)__reduce_min_sync(0xffffffffu, k == kmax ? (uint32_t)i : 0xffffffffu);
+  v = key_float(kmax);
+}
+
+// The two largest of the 32 lanes' (largest, second largest) pairs, on every
+// lane: the largest first value, then the largest of the other lanes' first
+// values and that lane's second value.
+__device__ __forceinline__ void warp_top2(float& m1, float& m2, int lane) {
+  const uint32_t k1 = order_key(m1);
+  const uint32_t kmax = __reduce_max_sync(0xffffffffu, k1);
+  const uint32_t owner = __reduce_min_sync(0xffffffffu, k1 == kmax ? (uint32_t)lane : 32u);
+  const uint32_t k2 = __reduce_max_sync(0xffffffffu, (uint32_t)lane == owner ? order_key(m2) : k1);
+  m1 = key_float(kmax);
+  m2 = key_float(k2);
 }
 
 // Merge two (largest, second largest) pairs.
@@ -86,12 +109,7 @@ __device__ __forceinline__ void select_token(const float (&s)[kEPL], const float
 #pragma unroll
     for (int j = 0; j < kEPL; ++j)
       if (grp[j] == g) top2_merge(m1, m2, sb[j], -INFINITY);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float b1 = __shfl_xor_sync(0xffffffffu, m1, o);
-      const float b2 = __shfl_xor_sync(0xffffffffu, m2, o);
-      top2_merge(m1, m2, b1, b2);
-    }
+    warp_top2(m1, m2, lane);
     const float score = (gs >= 2) ? m1 + m2 : m1;
     if (lane == g) my_gscore = score;
   }
