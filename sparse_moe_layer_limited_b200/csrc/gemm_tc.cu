@@ -65,14 +65,24 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 enum Epi { kEpiSwiGLU = 0, kEpiStore = 1, kEpiScores = 2, kEpiSwiGLUBwd = 3,
            kEpiStoreCombine = 4 };
 
+// Row-store epilogues (GEMM1 h, GEMM2 y) write full 32-row groups by TMA:
+// per epilogue warp two 2 KB pieces (32 rows x 32 bf16 columns) of shared
+// memory in the TMA's 64-byte swizzle, one filled while the other is stored.
+constexpr int kOutPiece = 2048;
+constexpr int kOutStgBytes = 4 * 2 * kOutPiece;
+template <int kEpi, int kBN>
+__host__ __device__ constexpr bool tma_out() {
+  return (kEpi == kEpiStore || kEpi == kEpiSwiGLU) && kBN == 256;
+}
+
 template <int kBN>
 struct TileCfg {
   static constexpr int kBBytes = kBN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * kBN;  // two accumulators
-  static constexpr size_t smem_bytes(int groups, bool gather) {
-    return 1024 + (size_t)kStages * kStageBytes + 256 + (gather ? (size_t)BM * 8 : 0) +
-           (size_t)(groups + 1) * 4;
+  static constexpr size_t smem_bytes(int groups, bool gather, bool staging) {
+    return 1024 + (size_t)kStages * kStageBytes + (staging ? kOutStgBytes : 0) + 256 +
+           (gather ? (size_t)BM * 8 : 0) + (size_t)(groups + 1) * 4;
   }
 };
 
@@ -80,6 +90,9 @@ struct alignas(64) GemmArgs {
   CUtensorMap tmA_routed;  // routed rows (unused when a_rows is set)
   CUtensorMap tmA_shared;
   CUtensorMap tmB;
+  CUtensorMap tmOut_routed;  // row-store epilogues: out_routed [rows_routed, out_ld] bf16 and
+  CUtensorMap tmOut_shared;  // out_shared [T, out_ld], box {32, 32}, 64-byte swizzle
+  int out_tma;               // 1: the two maps above are valid (set by the launcher)
   const int32_t* offsets;
   const int32_t* a_rows;  // when set: routed A row r of a group is a_src row a_rows[offsets[g] + r]
   const __nv_bfloat16* a_src;  // gathered rows' source (x), a_ld elements per row
@@ -201,10 +214,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   constexpr int kTmemCols = TileCfg<kBN>::kTmemCols;
   static_assert(kEpi != kEpiSwiGLU || kBN == 256, "SwiGLU tiles pair 128 gate + 128 up columns");
   (void)kBBytes;
+  constexpr bool kTmaOut = tma_out<kEpi, kBN>();
+  constexpr size_t kStg = kTmaOut ? kOutStgBytes : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)kStages * kStageBytes);
+  uint8_t* staging = base + (size_t)kStages * kStageBytes;  // 1024-aligned
+  (void)staging;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)kStages * kStageBytes + kStg);
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
   uint64_t* tfull = bars + 2 * kStages;  // [2]
@@ -213,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   // gathered tiles: the source address of each of the tile's 128 rows
   const char** rowptr =
-      reinterpret_cast<const char**>(base + (size_t)kStages * kStageBytes + 256);
-  int* tile_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + 256 +
+      reinterpret_cast<const char**>(base + (size_t)kStages * kStageBytes + kStg + 256);
+  int* tile_start = reinterpret_cast<int*>(base + (size_t)kStages * kStageBytes + kStg + 256 +
                                            (kGather ? BM * 8 : 0));
 
   const int tid = threadIdx.x;
@@ -481,6 +498,40 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           (g < args.N) ? args.out_routed + (size_t)(args.offsets[g] + r) * args.out_ld
                        : args.out_shared + (size_t)r * args.out_ld;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      // a warp whose 32 rows (of a 128-row tile) all lie inside the group
+      // stores them by TMA; the others take the row stores
+      bool tma_rows = false;
+      const CUtensorMap* omap = (g < args.N) ? &args.tmOut_routed : &args.tmOut_shared;
+      const int orow0 = ((g < args.N) ? args.offsets[g] : 0) + m * BM + q * 32;
+      if constexpr (kTmaOut) {
+        const int r0 = m * BM + q * 32;
+        tma_rows = args.out_tma != 0 && !m64 && r0 + 32 <= rows_g &&
+                   (g == args.N || args.offsets[g] + r0 + 32 <= args.rows_routed);
+      }
+      // one 32-column piece of this warp's rows -> staging -> TMA store
+      auto store_piece = [&](const float* y, int piece, int col) {
+        uint8_t* buf = staging + (size_t)(warp - 2) * (2 * kOutPiece) + (piece & 1) * kOutPiece;
+        if (lane == 0) bulk_wait_read_but_one();  // the store that last read buf is done
+        __syncwarp();
+        uint8_t* my = buf + lane * 64;
+        const int sw = (lane >> 1) & 3;  // the 64-byte swizzle of row `lane`
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const float* a = y + 8 * c4;
+          *reinterpret_cast<uint4*>(my + ((c4 ^ sw) << 4)) =
+              make_uint4(bf16x2_bits(a[0], a[1]), bf16x2_bits(a[2], a[3]),
+                         bf16x2_bits(a[4], a[5]), bf16x2_bits(a[6], a[7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(omap, buf, col, orow0);
+          bulk_commit_group();
+        }
+      };
+      (void)store_piece;
+      (void)omap;
+      (void)orow0;
       if constexpr (kEpi == kEpiSwiGLU) {
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
@@ -492,7 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             h[i] = silu_fast(__uint_as_float(ga[i])) * __uint_as_float(up[i]);
-          if (valid) store_row32(orow + n * (BN / 2) + c, h);
+          if (tma_rows)
+            store_piece(h, c / 32, n * (BN / 2) + c);
+          else if (valid)
+            store_row32(orow + n * (BN / 2) + c, h);
         }
       } else if constexpr (kEpi == kEpiStore) {
 #pragma unroll 1
@@ -503,7 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
           float y[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
-          if (valid) store_row32(orow + n * BN + c, y);
+          if (tma_rows)
+            store_piece(y, c / 32, n * BN + c);
+          else if (valid)
+            store_row32(orow + n * BN + c, y);
         }
       } else if constexpr (kEpi == kEpiStoreCombine) {
 #pragma unroll 1
@@ -577,6 +634,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    // the staging buffers must outlive the stores that read them
+    if constexpr (kTmaOut) {
+      if (lane == 0) bulk_wait_all();
+    }
   }
 
   // ---- teardown ------------------------------------------------------------------
@@ -592,13 +653,30 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_bf16_kernel(
 }
 
 template <int kEpi, int kBN, bool kGather = false>
-cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
-  const size_t smem = TileCfg<kBN>::smem_bytes(a.N + 1, kGather);
+cudaError_t launch_gemm(const GemmArgs& a0, cudaStream_t st) {
+  constexpr bool kTmaOut = tma_out<kEpi, kBN>();
+  const size_t smem = TileCfg<kBN>::smem_bytes(a0.N + 1, kGather, kTmaOut);
   cudaError_t e = note_cuda(cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kEpi, kBN, kGather>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem),
                             "bf16 GEMM: set shared-memory size");
   if (e != cudaSuccess) return e;
+  GemmArgs a = a0;
+  a.out_tma = 0;
+  if constexpr (kTmaOut) {
+    // TMA stores need 16-byte aligned outputs; otherwise every row takes the
+    // row stores
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const bool aligned = (reinterpret_cast<uintptr_t>(a.out_routed) % 16 == 0) &&
+                         (reinterpret_cast<uintptr_t>(a.out_shared) % 16 == 0) &&
+                         ((size_t)a.out_ld * 2) % 16 == 0;
+    if (aligned &&
+        make_map_swizzled(&a.tmOut_routed, a.out_routed, BF, 2, a.out_ld, a.rows_routed, 32, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B) &&
+        make_map_swizzled(&a.tmOut_shared, a.out_shared, BF, 2, a.out_ld, a.T, 32, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
+      a.out_tma = 1;
+  }
   grouped_gemm_bf16_kernel<kEpi, kBN, kGather><<<num_sms(), kThreads, smem, st>>>(a);
   return note_cuda(cudaGetLastError(), "bf16 GEMM launch");
 }

@@ -326,21 +326,34 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Z
 
 // prob_sum[e]: the selection CTAs' partials summed in a fixed order (eight
 // running sums over the CTAs b = j mod 8, then added j = 0..7), so the result
-// does not depend on scheduling.
-__global__ void prob_sum_kernel(const float* __restrict__ part, int nblocks, int N,
-                                float* __restrict__ prob_sum) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= N) return;
-  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int b = 0;
-  for (; b + 8 <= nblocks; b += 8)
+// does not depend on scheduling.  Block: 32 experts (lanes) x the eight sums
+// (warps); each sum takes its CTAs in increasing order, eight loads ahead.
+__global__ void __launch_bounds__(256) prob_sum_kernel(const float* __restrict__ part,
+                                                       int nblocks, int N,
+                                                       float* __restrict__ prob_sum) {
+  __shared__ float run[8][32];
+  const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  float a = 0.f;
+  if (e < N) {
+    for (int b = j; b < nblocks; b += 64) {
+      float v[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a[j] += part[(size_t)(b + j) * N + e];
-  for (int j = 0; b + j < nblocks; ++j) a[j] += part[(size_t)(b + j) * N + e];
-  float sum = 0.f;
+      for (int u = 0; u < 8; ++u)
+        v[u] = (b + 8 * u < nblocks) ? part[(size_t)(b + 8 * u) * N + e] : 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) sum += a[j];
-  prob_sum[e] = sum;
+      for (int u = 0; u < 8; ++u)
+        if (b + 8 * u < nblocks) a += v[u];
+    }
+  }
+  run[j][lane] = a;
+  __syncthreads();
+  if (j == 0 && e < N) {
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sum += run[q][lane];
+    prob_sum[e] = sum;
+  }
 }
 
 }  // namespace
@@ -383,7 +396,8 @@ int launch_route_softmax(const moe_shape& s, const void* x, const float* router,
   // one group kept of one: plain top-K over all experts
   select_kernel<true><<<nb, 256, 0, st>>>(Z, splits, nullptr, s.T, s.N, s.K, 1, 1, idx, gate,
                                           counts, part, status);
-  if (prob_sum != nullptr) prob_sum_kernel<<<1, 256, 0, st>>>(part, nb, s.N, prob_sum);
+  if (prob_sum != nullptr)
+    prob_sum_kernel<<<(s.N + 31) / 32, 256, 0, st>>>(part, nb, s.N, prob_sum);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
