@@ -88,7 +88,7 @@ def test_expert_parallel_single_rank_equals_layer():
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _two_rank_worker(rank, world, port, dtype, q):
+def _two_rank_worker(rank, world, port, dtype, q, replicas=0):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import datetime
@@ -104,6 +104,9 @@ def _two_rank_worker(rank, world, port, dtype, q):
     try:
         cfg = CONFIGS[1].with_(T=300, d=256, N=16, K=4, G=4, topG=2, f=256, dtype=dtype)
         R, b = gen.make_router(cfg), gen.make_bias(cfg)
+        if replicas:  # three hot experts, so that the placement makes replicas
+            b = np.asarray(b, np.float32).copy()
+            b[[1, 2, 9]] += np.float32(0.3)
         x, _ = S.tie_free_x(cfg, R, b, batch=rank)          # each rank its own batch
         W = S.device_weights(cfg)
         s = S.moe_shape(cfg)
@@ -113,11 +116,13 @@ def _two_rank_worker(rank, world, port, dtype, q):
         keep = list(range(lo, hi)) + [cfg.N]                # this rank's experts + shared
         w13 = W["w13"][keep].contiguous()
         w2 = W["w2"][keep].contiguous()
-        ops = ep.LibraryOps(s, ep.local_shape(s, world), Rd, bd.clone(), w13, w2)
-        epl = ep.ExpertParallelMoE(ops, cfg.N, gamma=cfg.gamma)
+        ops = ep.LibraryOps(s, ep.local_shape(s, world, replicas), Rd, bd.clone(), w13, w2,
+                            replicas=replicas)
+        epl = ep.ExpertParallelMoE(ops, cfg.N, gamma=cfg.gamma, redundant=replicas,
+                                   replan_every=1 if replicas else 0)
         layer = M.MoELayer(s, Rd, bd.clone(), W["w13"], W["w2"], gamma=cfg.gamma)
         xd = S.to_dev_x(x, cfg)
-        out = dict(equal=[], recv=[], counts=None, bias=None)
+        out = dict(equal=[], recv=[], counts=None, bias=None, hosted=None)
         for step in range(2):                 # step 1 routes with the updated bias
             layer.bias.copy_(ops.bias)
             y_ep = epl.forward(xd).clone()
@@ -128,6 +133,7 @@ def _two_rank_worker(rank, world, port, dtype, q):
             if step == 0:
                 out["counts"] = layer.counts.cpu().numpy().astype(np.int64)
                 out["bias"] = ops.bias.cpu().numpy()
+                out["hosted"] = epl.hosted
         out["status"] = [int(layer.device_status()), int(M.moe_read_device_status(ops.ws)),
                          int(M.moe_read_device_status(ops.ws_loc))]
         q.put((rank, out))
@@ -138,15 +144,20 @@ def _two_rank_worker(rank, world, port, dtype, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-def test_expert_parallel_two_ranks_one_gpu(dtype):
+@pytest.mark.parametrize("dtype,replicas", [("bf16", 0), ("fp32", 0), ("bf16", 2)])
+def test_expert_parallel_two_ranks_one_gpu(dtype, replicas):
+    """replicas=2: after the first step the three hot experts (and one more)
+    get copies on the other rank, so the second step splits their rows
+    between two GPUs' worth of slots and moves their weights first."""
     import oracle
     import torch.multiprocessing as mp
+    from sparse_moe_layer_limited_b200 import ep
     from synth import CONFIGS
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_two_rank_worker, args=(r, 2, port, dtype, q)) for r in range(2)]
+    procs = [ctx.Process(target=_two_rank_worker, args=(r, 2, port, dtype, q, replicas))
+             for r in range(2)]
     for p in procs:
         p.start()
     try:
@@ -164,6 +175,13 @@ def test_expert_parallel_two_ranks_one_gpu(dtype):
     for step in (0, 1):                               # every routed row went to one rank
         assert res[0]["recv"][step] + res[1]["recv"][step] == 2 * cfg.T * cfg.K
     b0 = gen.make_bias(cfg)
+    if replicas:
+        b0 = np.asarray(b0, np.float32).copy()
+        b0[[1, 2, 9]] += np.float32(0.3)
+        placed = res[0]["hosted"]
+        assert placed == res[1]["hosted"]
+        assert placed == ep.place_redundant(res[0]["counts"] + res[1]["counts"], cfg.N, 2, replicas)
+        assert all(e >= 0 for h in placed for e in h[cfg.N // 2:])
     want_b = oracle.bias_update(b0, res[0]["counts"] + res[1]["counts"], 2 * cfg.T, cfg.K,
                                 cfg.gamma)
     np.testing.assert_array_equal(res[0]["bias"], want_b)
