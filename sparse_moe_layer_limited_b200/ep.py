@@ -31,9 +31,10 @@ per-rank computation is behind a small operations interface: the library's
 CUDA kernels (``LibraryOps``) on the product path.  The host-side planning
 (send splits, the regroup tables) is plain integer work in NumPy.
 
-Redundant experts: the pages' inference deployment (the V3 deployment
-walk-through, decoding stage; gkm0120.cn notes Q10) places extra copies of
-high-load experts on other GPUs and adjusts the placement as the load moves.
+Redundant experts: the inference deployment in the DeepSeek-V3
+walk-through (kaiyunto.com), deployment section (decoding stage), and the
+"解读 DeepSeek-V3" notes (gkm0120.cn), Q10, place extra copies of high-load
+experts on other GPUs and adjust the placement as the load moves.
 Here every rank keeps r replica slots beside its N/W primary experts.
 `place_redundant` fills the W*r slots greedily from the node-wide counts:
 the expert with the highest load per copy receives another copy on the
