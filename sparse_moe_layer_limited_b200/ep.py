@@ -186,15 +186,10 @@ def send_tables(counts, hosted, sender: int, n_primary: int):
             sendcnt[q, i] = m
             start[(q, i)] = pos
             pos += m
-    order = []
-    for q in range(W):
-        for i in range(S):
-            m = int(sendcnt[q, i])
-            if m:
-                a = start[(q, i)]
-                order.extend(range(a, a + m))
-    return dict(sendcnt=sendcnt, sends=[int(v) for v in sendcnt.sum(axis=1)],
-                order=np.asarray(order, dtype=np.int64))
+    parts = [np.arange(start[(q, i)], start[(q, i)] + sendcnt[q, i], dtype=np.int64)
+             for q in range(W) for i in range(S) if sendcnt[q, i]]
+    order = np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+    return dict(sendcnt=sendcnt, sends=[int(v) for v in sendcnt.sum(axis=1)], order=order)
 
 
 def exchange_replica_weights(dist, group, w13, w2, hosted, old_hosted, n_primary: int):
@@ -220,14 +215,12 @@ def exchange_replica_weights(dist, group, w13, w2, hosted, old_hosted, n_primary
         mine = [(i, e) for i, e in need[q] if e // n_primary == rank]
         for _, e in mine:
             j = e - rank * n_primary
-            send_parts += [w13[j].reshape(-1), w2[j].reshape(-1)]
+            send_parts += [w13[j].view(-1), w2[j].view(-1)]
         send_sizes.append(len(mine) * per_block)
     recv_list = [(i, e) for i, e in need[rank]]
     recv_sizes = [sum(1 for _, e in recv_list if e // n_primary == p) * per_block
                   for p in range(W)]
-    if sum(send_sizes) == 0 and sum(recv_sizes) == 0:
-        # every rank still takes part in the collective
-        pass
+    # every rank takes part in the collective, also with nothing to move
     send = (torch.cat(send_parts) if send_parts
             else torch.empty(0, dtype=w13.dtype, device=w13.device))
     recv = torch.empty(sum(recv_sizes), dtype=w13.dtype, device=w13.device)
@@ -237,8 +230,8 @@ def exchange_replica_weights(dist, group, w13, w2, hosted, old_hosted, n_primary
         for i, e in recv_list:
             if e // n_primary != p:
                 continue
-            w13[i].reshape(-1).copy_(recv[pos:pos + blk13])
-            w2[i].reshape(-1).copy_(recv[pos + blk13:pos + per_block])
+            w13[i].view(-1).copy_(recv[pos:pos + blk13])     # view: the slot itself
+            w2[i].view(-1).copy_(recv[pos + blk13:pos + per_block])
             pos += per_block
 
 
