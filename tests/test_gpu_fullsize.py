@@ -101,6 +101,9 @@ def test_v3_bf16_passes_and_sampled_outputs(M):
             np.testing.assert_array_equal(layer.offsets.cpu().numpy(), d["offsets"])
             np.testing.assert_array_equal(layer.perm_tok.cpu().numpy(), d["perm_tok"])
             np.testing.assert_array_equal(layer.slot.cpu().numpy(), d["slot"])
+            # every dispatched row is its token's row, bit for bit (65,536 rows)
+            pt = torch.from_numpy(d["perm_tok"].astype(np.int64)).to(xd.device)
+            assert torch.equal(layer.x_perm[:len(pt)], xd[pt])
             # every expert's ragged last m-tile, and the whole output of 64 tokens
             _check_tails_and_tokens(layer, x, r, d, cfg, y, "bf16", 1e-2)
         b = b_next

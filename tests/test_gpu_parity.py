@@ -91,11 +91,17 @@ def _layer(M, cfg, x, R, b, W):
     return layer, xd
 
 
-def _check_dispatch(layer, r):
+def _check_dispatch(layer, r, xd=None):
+    """offsets, perm_tok and slot equal the oracle's; with the device input
+    xd, every dispatched row (bf16 or fp32) is its token's row bit for bit."""
+    import torch
     d = oracle.dispatch(r["idx"], layer.shape.N)
     np.testing.assert_array_equal(layer.offsets.cpu().numpy(), d["offsets"])
     np.testing.assert_array_equal(layer.perm_tok.cpu().numpy(), d["perm_tok"])
     np.testing.assert_array_equal(layer.slot.cpu().numpy(), d["slot"])
+    if xd is not None and layer.x_perm is not None and layer.x_perm.dtype == xd.dtype:
+        pt = torch.from_numpy(d["perm_tok"].astype(np.int64)).to(xd.device)
+        assert torch.equal(layer.x_perm[:len(pt)], xd[pt])
     return d
 
 
@@ -111,7 +117,7 @@ def test_tiny_fp32_layer_full(M):
     r = ref["route"]
     _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
                  layer.counts.cpu().numpy())
-    _check_dispatch(layer, r)
+    _check_dispatch(layer, r, xd)
     err = S.rel_fro(y, ref["y"])
     assert err <= TOL["fp32"], err
     nb = oracle.bias_update(b, r["counts"], cfg.T, cfg.K, cfg.gamma)
@@ -137,7 +143,7 @@ def test_small_bf16_layer_full(M, T):
     r = ref["route"]
     _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
                  layer.counts.cpu().numpy())
-    d = _check_dispatch(layer, r)
+    d = _check_dispatch(layer, r, xd)
     # per-expert rows of the grouped GEMM output
     get = S.host_weights(cfg)
     yp = layer.y_perm.float().cpu().numpy()
@@ -201,7 +207,7 @@ def test_mid_bf16_layer_full(M):
     r = oracle.route(x, R, b, cfg.G, cfg.topG, cfg.K)
     _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
                  layer.counts.cpu().numpy())
-    d = _check_dispatch(layer, r)
+    d = _check_dispatch(layer, r, xd)
     ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
                              h_round="bf16")
     err = S.rel_fro(y, ref["y"])
@@ -260,7 +266,7 @@ def test_small_fp8_layer_full(M, T):
     r = ref["route"]
     _check_route(cfg, r, layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
                  layer.counts.cpu().numpy())
-    d = _check_dispatch(layer, r)
+    d = _check_dispatch(layer, r, xd)
     # dispatched rows are quantised per 1x128 tile exactly as the oracle does
     codes, scales = oracle.quant_rows_1x128(x[d["perm_tok"]])
     np.testing.assert_array_equal(layer.x_perm.view(torch.uint8).cpu().numpy(), codes)
@@ -341,7 +347,7 @@ def test_layer_k13_same_node_budget(M):
                              h_round="bf16")
     _check_route(cfg, ref["route"], layer.topk_idx.cpu().numpy(),
                  layer.topk_gate.cpu().numpy(), layer.counts.cpu().numpy())
-    _check_dispatch(layer, ref["route"])
+    _check_dispatch(layer, ref["route"], xd)
     assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
     assert layer.device_status() == 0
 
@@ -357,7 +363,7 @@ def test_layer_all_experts_every_token(M):
     ref = oracle.moe_forward(x, R, b, S.host_weights(cfg), cfg.G, cfg.topG, cfg.K,
                              h_round="bf16")
     assert np.all(layer.counts.cpu().numpy() == cfg.T)
-    _check_dispatch(layer, ref["route"])
+    _check_dispatch(layer, ref["route"], xd)
     assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
     assert layer.device_status() == 0
 
@@ -376,6 +382,6 @@ def test_layer_with_idle_experts(M):
                              h_round="bf16")
     counts = layer.counts.cpu().numpy()
     assert counts[8:].sum() == 0 and counts.sum() == cfg.T * cfg.K
-    _check_dispatch(layer, ref["route"])
+    _check_dispatch(layer, ref["route"], xd)
     assert S.rel_fro(y, ref["y"]) <= TOL["bf16"]
     assert layer.device_status() == 0
