@@ -41,7 +41,10 @@ def _inputs(cfg):
     return x, r
 
 
-def _dispatch_both(M, cfg, x, r, slots_only=False):
+def _dispatch_both(M, cfg, x, r, slots_only=False, statuses=None):
+    """moe_dispatch (with a workspace) and moe_dispatch_noalloc on the same
+    inputs, outputs pre-filled with -7; with `statuses` a list, the
+    workspace call's device status word is appended to it."""
     import torch
     s = S.moe_shape(cfg)
     xd = S.to_dev_x(x, cfg)
@@ -57,6 +60,8 @@ def _dispatch_both(M, cfg, x, r, slots_only=False):
         if which == "ws":
             ws = torch.zeros(M.workspace_size(s), dtype=torch.uint8, device="cuda")
             M.moe_dispatch(s, xd, idx, counts, off, perm, slot, xp_arg, None, ws)
+            if statuses is not None:
+                statuses.append(M.moe_read_device_status(ws))
         else:
             rc = M.lib().moe_dispatch_noalloc(
                 ctypes.byref(s), ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(idx.data_ptr()),
@@ -109,3 +114,36 @@ def test_noalloc_at_its_largest_shape_and_slots_only():
         np.testing.assert_array_equal(s2, d["slot"])
         if slots_only:
             assert not x2.any()            # the rows were not copied
+
+
+MOE_DEV_BAD_INDEX = 4  # the device status bit for an expert index outside [0, N)
+
+
+@pytest.mark.gpu
+def test_noalloc_bad_expert_index_stays_in_bounds():
+    """One (token, k) pair names expert N, outside [0, N).  moe_dispatch
+    reports it in its workspace status; moe_dispatch_noalloc, whose status
+    word cannot be read back, must still write only in bounds: both leave
+    that pair's slot untouched (-7) and place no row for it, and every other
+    pair's slot and row, perm_tok and the offsets agree between the two."""
+    import sparse_moe_layer_limited_b200 as M
+    cfg = CONFIGS[1].with_(T=1000, d=256, N=8, K=2, G=2, topG=1, f=256)
+    x, r = _inputs(cfg)
+    idx = r["idx"].astype(np.int32).copy()
+    counts = r["counts"].astype(np.int64).copy()
+    t_bad, k_bad = 3, 1
+    counts[idx[t_bad, k_bad]] -= 1         # counts describe the valid pairs only
+    idx[t_bad, k_bad] = cfg.N
+    statuses = []
+    (o1, p1, s1, x1), (o2, p2, s2, x2) = _dispatch_both(M, cfg, x, dict(r, idx=idx, counts=counts),
+                                                        statuses=statuses)
+    assert statuses[0] & MOE_DEV_BAD_INDEX
+    TK1 = cfg.T * cfg.K - 1                # rows placed: every pair but the bad one
+    np.testing.assert_array_equal(o2, o1)
+    assert o1[cfg.N] == TK1
+    np.testing.assert_array_equal(p2[:TK1], p1[:TK1])
+    assert p1[TK1] == -7 and p2[TK1] == -7  # the row past the placed ones is not written
+    np.testing.assert_array_equal(s2, s1)
+    assert s1[t_bad, k_bad] == -7 and s2[t_bad, k_bad] == -7
+    np.testing.assert_array_equal(x2[:TK1], x1[:TK1])
+    np.testing.assert_array_equal(x1[:TK1], x[p1[:TK1]].astype(np.float32))
