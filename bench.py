@@ -270,8 +270,10 @@ def main():
     main_res = run_layer(cfg, dev, args.steps, max(3, args.warmup), pg, local, e2e=True)
     extra = {}
     if not args.no_extra and not (args.T or args.N):
-        # the FP8 layer and the decode workload, reported beside the bf16 headline
+        # the FP8 layer, the decode workload and the mid-size bf16 layer,
+        # reported beside the bf16 headline
         extra["fp8"] = run_layer(BY_NAME["v3_fp8"], dev, max(5, args.steps // 5), 3, pg, local)
+        extra["mid"] = run_layer(BY_NAME["mid_bf16"], dev, max(20, args.steps), 3, pg, local)
         extra["decode"] = run_layer(BY_NAME["decode_zipf"], dev, max(20, args.steps), 3, pg,
                                     local)
     bwd = layer_bwd = bwd_fp8 = None
