@@ -18,6 +18,8 @@ pytestmark = pytest.mark.gpu
 CASES = {
     "tiny_fp32": CONFIGS[0],
     "small_bf16": CONFIGS[1].with_(T=300, d=256, N=16, K=4, G=4, topG=2, f=256),
+    # more than eight selected experts: the gate kernel's wide instantiation
+    "k13_bf16": CONFIGS[1].with_(T=200, d=256, N=64, K=13, G=8, topG=4, f=256),
 }
 
 
