@@ -50,9 +50,10 @@ def parse():
     p.add_argument("--fused-combine", choices=["on", "off"], default="off",
                    help="bf16: the combine runs inside GEMM2's epilogue (on) or as its own "
                         "kernel (off); the output is bit-identical")
-    p.add_argument("--only", choices=["backward_fp8"], default=None,
+    p.add_argument("--only", choices=["backward", "backward_fp8"], default=None,
                    help="run one of the line's measurements alone and print its object "
-                        "(backward_fp8: the FP8 expert backward on the V3 FP8 shapes)")
+                        "(backward: the bf16 expert backward on --config's shapes; "
+                        "backward_fp8: the FP8 expert backward on the V3 FP8 shapes)")
     p.add_argument("--T", type=int, default=None, help="override tokens (profiling runs)")
     p.add_argument("--N", type=int, default=None, help="override routed experts (profiling)")
     return p.parse_args()
@@ -249,6 +250,12 @@ def main():
         cfg = cfg.with_(N=args.N)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.only == "backward":
+        import torch
+        out = run_backward(cfg, torch.device("cuda"), calls=max(1, args.steps),
+                           warmup=args.warmup)
+        print(json.dumps({"backward_dx": out}), flush=True)
+        return out
     if args.only == "backward_fp8":
         import torch
         c8 = BY_NAME["v3_fp8"]

@@ -354,9 +354,14 @@ cudaError_t launch_wgrad(const WgradArgs& a, cudaStream_t st) {
 // same 128 x 256 outputs, and each CTA's TMEM holds its 128 rows of the tile.
 // The gradient rows are multiples of 256 (d and 2f are), so no unit is ragged.
 // Barriers: full (leader; both CTAs' copies land on it), empty and tfull (each
-// CTA; the leader's commits are multicast), tempty (leader; the 16 epilogue
-// warps of the pair).  Both CTAs reach the final cluster barrier, so neither
-// exits while its peer may still signal it.
+// CTA; the leader's commits are multicast), edone (each CTA; its eight
+// epilogue warps have read the accumulator) and tempty (leader; one arrive per
+// use from the peer CTA's warp 1, which forwards its edone).  The leader's MMA
+// thread waits on its own edone and on tempty, so one cluster-scope arrive per
+// accumulator use crosses the pair instead of one per epilogue warp: the
+// release fence each of those arrives carries was the epilogue's largest
+// stall.  Both CTAs reach the final cluster barrier, so neither exits while
+// its peer may still signal it.
 constexpr int QStages = 5;
 constexpr int QHalfBytes = WBM * WBK * 2;     // 16 KB: 128 rows x 64 K
 constexpr int QStageBytes = 2 * QHalfBytes;   // left rows + right rows
@@ -377,7 +382,8 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_pair_kernel(
   uint64_t* tfull = empty + QStages;   // [2] each CTA
   uint64_t* tempty = tfull + 2;        // [2] leader
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* edone = drain + 1;         // [2] each CTA: its eight epilogue warps have read
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(edone + 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -393,7 +399,8 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_pair_kernel(
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 16);
+      mbar_init(&tempty[a], 1);   // the peer CTA's forwarded release
+      mbar_init(&edone[a], 8);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -464,7 +471,8 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_pair_kernel(
         int g, n, m, kb0, kcnt;
         decode(u, g, n, m, kb0, kcnt);
         const int acc = local & 1;
-        if (!mbar_wait_cluster_bounded(&tempty[acc], ((local >> 1) & 1) ^ 1u, args.status,
+        if (!mbar_wait_bounded(&edone[acc], ((local >> 1) & 1) ^ 1u, args.status, WTimeoutNs) ||
+            !mbar_wait_cluster_bounded(&tempty[acc], ((local >> 1) & 1) ^ 1u, args.status,
                                        WTimeoutNs))
           break;
         tc_fence_after();
@@ -491,13 +499,22 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_pair_kernel(
       }
       mma_commit_2sm(drain);
       mbar_wait_bounded(drain, 0, args.status, WTimeoutNs / 8);
+    } else if (!leader && lane == 0) {
+      // forward each accumulator release of this CTA's epilogue warps to the
+      // leader with one cluster-scope arrive
+      const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+      int local = 0;
+      for (int u = pair; u < total; u += npairs, ++local) {
+        const int acc = local & 1;
+        if (!mbar_wait_bounded(&edone[acc], (local >> 1) & 1, args.status, WTimeoutNs)) break;
+        mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
+      }
     }
   } else {
     // each CTA drains its 128 rows of the tile exactly as the one-CTA kernel
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     uint8_t* stg0 = staging + (size_t)(warp - 2) * 2 * WStgBytes;
-    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int local = 0;
     for (int u = pair; u < total; u += npairs, ++local) {
       int g, n, m, kb0, kcnt;
@@ -542,7 +559,7 @@ __global__ void __launch_bounds__(WThreads, 1) wgrad_pair_kernel(
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
+      if (lane == 0) mbar_arrive(&edone[acc]);
     }
     if (lane == 0) bulk_wait_all();
   }
