@@ -75,21 +75,27 @@ __global__ void colbase_kernel(const int32_t* __restrict__ offsets, int N, int T
 // from `shared`; with `perm_tok`, dispatched row r is row perm_tok[r] of
 // `routed`) -> dst [C, R]: group g's rows go, in order, to its columns
 // colbase[g] .. colbase[g] + rows_g - 1, and its padding columns up to
-// colbase[g + 1] get zeros.  One 64 x 64 tile per CTA (tile_transpose.cuh);
-// the colbase values are multiples of 64 (the padding is 64 or 128), so a
-// column tile lies in one group.
+// colbase[g + 1] get zeros.  A CTA moves kGroupTiles 64 x 64 tiles
+// (tile_transpose.cuh) of the same 64 columns and consecutive features: all
+// their 16-byte loads are issued before any shared-memory write, so each
+// thread keeps 2 * kGroupTiles loads in flight.  The colbase values are
+// multiples of 64 (the padding is 64 or 128), so a column tile lies in one
+// group.
 // kSwiGLUH: the source holds the packed gate/up products [rows, 2f] and the
 // value moved is h = silu(g) * u of feature c (C = f), rounded to bf16.
+constexpr int kGroupTiles = 4;
+constexpr int kItems = kTile * 8 / kTileThreads;  // 16-byte items per thread per tile
+
 template <bool kSwiGLUH>
 __global__ void __launch_bounds__(kTileThreads) transpose_groups_kernel(
     const __nv_bfloat16* __restrict__ routed, const __nv_bfloat16* __restrict__ shared, int TK,
     int T, int N, int C, int src_ld, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ perm_tok, const int32_t* __restrict__ colbase, long long ld,
     __nv_bfloat16* __restrict__ dst) {
-  __shared__ alignas(16) uint8_t sm[kTileBytes];
+  __shared__ alignas(16) uint8_t sm[kGroupTiles][kTileBytes];
   __shared__ int s_group;
   const long long col0 = (long long)blockIdx.y * kTile;
-  const int f0 = blockIdx.x * kTile;
+  const int fb = blockIdx.x * kGroupTiles * kTile;
   const int G1 = N + 1;
   if (col0 >= colbase[G1]) return;  // past the last group's block
   if (threadIdx.x == 0) {
@@ -106,36 +112,60 @@ __global__ void __launch_bounds__(kTileThreads) transpose_groups_kernel(
   const long long count = g < N ? (long long)offsets[g + 1] - offsets[g] : T;
   const long long limit = g < N ? TK : (long long)TK + T;  // a group's rows stay below
   const long long local0 = col0 - colbase[g];
-  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
-    const int i = it >> 3, p = it & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  // this thread's source rows (the same in every tile of the CTA)
+  const __nv_bfloat16* rowp[kItems];
+#pragma unroll
+  for (int j = 0; j < kItems; ++j) {
+    const int i = (threadIdx.x + j * kTileThreads) >> 3;
     const long long r = first + local0 + i;
     const long long src = (perm_tok != nullptr && r >= 0 && r < TK) ? perm_tok[r] : r;
     const bool src_ok = perm_tok == nullptr || r >= TK || (src >= 0 && src < T);
-    if (local0 + i < count && r >= 0 && r < limit && src_ok && f0 + p * 8 + 8 <= C) {
-      const __nv_bfloat16* row =
-          r < TK ? routed + (size_t)src * src_ld : shared + (size_t)(r - TK) * src_ld;
-      if constexpr (kSwiGLUH) {
-        const int col = (f0 / 128) * 256 + (f0 % 128) + p * 8;
-        float gt[8], up[8];
-        bf16x8_load(row + col, gt);
-        bf16x8_load(row + col + 128, up);
-        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+    rowp[j] = (local0 + i < count && r >= 0 && r < limit && src_ok)
+                  ? (r < TK ? routed + (size_t)src * src_ld : shared + (size_t)(r - TK) * src_ld)
+                  : nullptr;
+  }
+  uint4 v[kGroupTiles][kItems];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          h[e] = __floats2bfloat162_rn(silu_fast(gt[2 * e]) * up[2 * e],
-                                       silu_fast(gt[2 * e + 1]) * up[2 * e + 1]);
-      } else {
-        v = __ldg(reinterpret_cast<const uint4*>(row + f0 + p * 8));
+  for (int t = 0; t < kGroupTiles; ++t) {
+    const int f0 = fb + t * kTile;
+#pragma unroll
+    for (int j = 0; j < kItems; ++j) {
+      const int p = (threadIdx.x + j * kTileThreads) & 7;
+      v[t][j] = make_uint4(0u, 0u, 0u, 0u);
+      if (rowp[j] != nullptr && f0 + p * 8 + 8 <= C) {
+        if constexpr (kSwiGLUH) {
+          const int col = (f0 / 128) * 256 + (f0 % 128) + p * 8;
+          float gt[8], up[8];
+          bf16x8_load(rowp[j] + col, gt);
+          bf16x8_load(rowp[j] + col + 128, up);
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v[t][j]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            h[e] = __floats2bfloat162_rn(silu_fast(gt[2 * e]) * up[2 * e],
+                                         silu_fast(gt[2 * e + 1]) * up[2 * e + 1]);
+        } else {
+          v[t][j] = __ldg(reinterpret_cast<const uint4*>(rowp[j] + f0 + p * 8));
+        }
       }
     }
-    tile_put(sm, i, p, v);
   }
+#pragma unroll
+  for (int t = 0; t < kGroupTiles; ++t)
+#pragma unroll
+    for (int j = 0; j < kItems; ++j) {
+      const int it = threadIdx.x + j * kTileThreads;
+      tile_put(sm[t], it >> 3, it & 7, v[t][j]);
+    }
   __syncthreads();
-  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
-    const int c = it >> 3, q = it & 7;
-    if (f0 + c < C && col0 + q * 8 + 8 <= ld)
-      *reinterpret_cast<uint4*>(dst + (size_t)(f0 + c) * ld + col0 + q * 8) = tile_get(sm, c, q);
+#pragma unroll
+  for (int t = 0; t < kGroupTiles; ++t) {
+    const int f0 = fb + t * kTile;
+    for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
+      const int c = it >> 3, q = it & 7;
+      if (f0 + c < C && col0 + q * 8 + 8 <= ld)
+        *reinterpret_cast<uint4*>(dst + (size_t)(f0 + c) * ld + col0 + q * 8) =
+            tile_get(sm[t], c, q);
+    }
   }
 }
 
@@ -640,7 +670,8 @@ cudaError_t launch_group_transposes(const moe_shape& s, int pad, const void* a_r
   const unsigned col_tiles = (unsigned)(R / kTile);
   auto layout = [&](auto kernel, const __nv_bfloat16* routed, const int32_t* perm,
                     const __nv_bfloat16* shared, int C, int src_ld, __nv_bfloat16* dst) {
-    kernel<<<dim3(C / kTile, col_tiles), kTileThreads, 0, st>>>(
+    const unsigned f_blocks = (unsigned)((C / kTile + kGroupTiles - 1) / kGroupTiles);
+    kernel<<<dim3(f_blocks, col_tiles), kTileThreads, 0, st>>>(
         routed, shared, TK, s.T, s.N, C, src_ld, offsets, perm, colbase, R, dst);
   };
   layout(transpose_groups_kernel<false>, bf(a_routed), a_perm, bf(x), s.d, s.d, AT);
