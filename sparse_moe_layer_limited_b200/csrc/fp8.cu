@@ -104,7 +104,12 @@ __global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ x, long long
 }
 
 // ---- 128x128 weight quantisation ---------------------------------------------------
-// One CTA (128 threads) per block; thread t handles row t of the block.
+// One CTA (128 threads) per block.  Sixteen lanes cover one 128-column row of
+// the block with 16-byte loads (8 values each), so a warp reads two whole
+// 256-byte rows per instruction; warp w takes rows 32w .. 32w+31, two at a
+// time, and keeps its 16 loads in registers for the second pass.  The block's
+// max-abs is reduced over the lanes and warps, then each lane writes its 8
+// codes of each of its rows (8 bytes; 128 contiguous bytes per row).
 __global__ void __launch_bounds__(128) quant_blocks_kernel(const __nv_bfloat16* __restrict__ w,
                                                            int cols, long long blocks_r,
                                                            int blocks_c,
@@ -114,13 +119,15 @@ __global__ void __launch_bounds__(128) quant_blocks_kernel(const __nv_bfloat16* 
   const long long b = blockIdx.x;
   const long long br = b / blocks_c;
   const int bc = (int)(b - br * blocks_c);
-  const int t = threadIdx.x;
-  const __nv_bfloat16* row = w + (br * QB + t) * (long long)cols + (long long)bc * QB;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int half = lane >> 4, l16 = lane & 15;  // row parity within a pair, 16-byte piece
+  const long long row0 = br * QB + warp * 32 + half;  // this lane's first row
+  const __nv_bfloat16* src = w + row0 * (long long)cols + (long long)bc * QB + 8 * l16;
   float amax = 0.f;
   uint4 raw[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    raw[i] = reinterpret_cast<const uint4*>(row)[i];
+  for (int i = 0; i < 16; ++i) {  // rows row0 + 2i
+    raw[i] = __ldg(reinterpret_cast<const uint4*>(src + (long long)(2 * i) * cols));
     float f[8];
     bf16x8_to_f32(raw[i], f);
 #pragma unroll
@@ -128,13 +135,13 @@ __global__ void __launch_bounds__(128) quant_blocks_kernel(const __nv_bfloat16* 
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if ((t & 31) == 0) red[t >> 5] = amax;
+  if (lane == 0) red[warp] = amax;
   __syncthreads();
   amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   const bool zero = amax == 0.f;
   const float scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
   const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
-  uint8_t* qrow = q + (br * QB + t) * (long long)cols + (long long)bc * QB;
+  uint8_t* dst = q + row0 * (long long)cols + (long long)bc * QB + 8 * l16;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float f[8];
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(128) quant_blocks_kernel(const __nv_bfloat16* 
           w2[p] |= (uint32_t)c2 << (16 * qq);
         }
     }
-    reinterpret_cast<uint2*>(qrow)[i] = make_uint2(w2[0], w2[1]);
+    *reinterpret_cast<uint2*>(dst + (long long)(2 * i) * cols) = make_uint2(w2[0], w2[1]);
   }
   if (t == 0) sc[br * blocks_c + bc] = scale;
 }
