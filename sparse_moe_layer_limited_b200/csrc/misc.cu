@@ -160,25 +160,48 @@ cudaError_t launch_pack_w13(const moe_shape& s, const void* w1, const void* w3, 
 }
 
 // [B, R, C] bf16 -> [B, C, R] in 64 x 64 tiles (tile_transpose.cuh); R and
-// C are multiples of 64 (the bf16 shape rules make d, f and 2f so).
+// C are multiples of 64 (the bf16 shape rules make d, f and 2f so).  A CTA
+// moves kRowTiles tiles of the same 64 rows and consecutive columns, with all
+// its 16-byte loads issued before any shared-memory write (2 * kRowTiles
+// loads in flight per thread).
 namespace {
+constexpr int kRowTiles = 4;
+constexpr int kTItems = kTile * 8 / kTileThreads;  // 16-byte items per thread per tile
+
 __global__ void __launch_bounds__(kTileThreads) transpose_tiles_kernel(
     const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int R, int C) {
-  __shared__ alignas(16) uint8_t sm[kTileBytes];
+  __shared__ alignas(16) uint8_t sm[kRowTiles][kTileBytes];
   const size_t b = blockIdx.z;
-  const int r0 = blockIdx.y * kTile, c0 = blockIdx.x * kTile;
-  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
-    const int i = it >> 3, p = it & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r0 + i < R && c0 + p * 8 + 8 <= C)
-      v = __ldg(reinterpret_cast<const uint4*>(src + (b * R + r0 + i) * C + c0 + p * 8));
-    tile_put(sm, i, p, v);
+  const int r0 = blockIdx.y * kTile, cb = blockIdx.x * kRowTiles * kTile;
+  uint4 v[kRowTiles][kTItems];
+#pragma unroll
+  for (int t = 0; t < kRowTiles; ++t) {
+    const int c0 = cb + t * kTile;
+#pragma unroll
+    for (int j = 0; j < kTItems; ++j) {
+      const int it = threadIdx.x + j * kTileThreads;
+      const int i = it >> 3, p = it & 7;
+      v[t][j] = make_uint4(0u, 0u, 0u, 0u);
+      if (r0 + i < R && c0 + p * 8 + 8 <= C)
+        v[t][j] = __ldg(reinterpret_cast<const uint4*>(src + (b * R + r0 + i) * C + c0 + p * 8));
+    }
   }
+#pragma unroll
+  for (int t = 0; t < kRowTiles; ++t)
+#pragma unroll
+    for (int j = 0; j < kTItems; ++j) {
+      const int it = threadIdx.x + j * kTileThreads;
+      tile_put(sm[t], it >> 3, it & 7, v[t][j]);
+    }
   __syncthreads();
-  for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
-    const int c = it >> 3, q = it & 7;
-    if (c0 + c < C && r0 + q * 8 + 8 <= R)
-      *reinterpret_cast<uint4*>(dst + (b * C + c0 + c) * R + r0 + q * 8) = tile_get(sm, c, q);
+#pragma unroll
+  for (int t = 0; t < kRowTiles; ++t) {
+    const int c0 = cb + t * kTile;
+    for (int it = threadIdx.x; it < kTile * 8; it += kTileThreads) {
+      const int c = it >> 3, q = it & 7;
+      if (c0 + c < C && r0 + q * 8 + 8 <= R)
+        *reinterpret_cast<uint4*>(dst + (b * C + c0 + c) * R + r0 + q * 8) = tile_get(sm[t], c, q);
+    }
   }
 }
 }  // namespace
@@ -188,9 +211,10 @@ cudaError_t launch_transpose_weights(const moe_shape& s, const void* w13, const 
   if (s.d % kTile != 0 || (2 * s.f) % kTile != 0 || s.f % kTile != 0)
     return cudaErrorInvalidValue;
   const unsigned E = (unsigned)(s.N + 1);
-  transpose_tiles_kernel<<<dim3(s.d / kTile, 2 * s.f / kTile, E), kTileThreads, 0, st>>>(
+  const auto blocks = [](int C) { return (unsigned)((C / kTile + kRowTiles - 1) / kRowTiles); };
+  transpose_tiles_kernel<<<dim3(blocks(s.d), 2 * s.f / kTile, E), kTileThreads, 0, st>>>(
       static_cast<const __nv_bfloat16*>(w13), static_cast<__nv_bfloat16*>(w13t), 2 * s.f, s.d);
-  transpose_tiles_kernel<<<dim3(s.f / kTile, s.d / kTile, E), kTileThreads, 0, st>>>(
+  transpose_tiles_kernel<<<dim3(blocks(s.f), s.d / kTile, E), kTileThreads, 0, st>>>(
       static_cast<const __nv_bfloat16*>(w2), static_cast<__nv_bfloat16*>(w2t), s.d, s.f);
   return cudaGetLastError();
 }
