@@ -26,6 +26,10 @@ __device__ __forceinline__ void to_f32x8(const uint4& v, float (&o)[8]) {
   }
 }
 
+// KM > 0 (K <= KM): a thread loads its piece of all K rows before the first
+// multiply-add, so K loads are in flight; KM = 0 takes the rows one by one.
+// Either way the sums run in k order from y_shared.
+template <int KM>
 __global__ void __launch_bounds__(128) combine_bf16_kernel(const __nv_bfloat16* __restrict__ y_perm,
                                                            const __nv_bfloat16* __restrict__ y_sh,
                                                            const int32_t* __restrict__ slot,
@@ -45,13 +49,30 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(const __nv_bfloat16* 
   const int nvec = d / 8;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float acc[8];
-    to_f32x8(__ldg(reinterpret_cast<const uint4*>(y_sh + (size_t)t * d) + v), acc);
-    for (int k = 0; k < K; ++k) {
-      float r[8];
-      to_f32x8(__ldg(reinterpret_cast<const uint4*>(y_perm + (size_t)ss[k] * d) + v), r);
-      const float g = sg[k];
+    if constexpr (KM > 0) {
+      uint4 raw[KM];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, r[i], acc[i]);
+      for (int k = 0; k < KM; ++k)
+        if (k < K) raw[k] = __ldg(reinterpret_cast<const uint4*>(y_perm + (size_t)ss[k] * d) + v);
+      to_f32x8(__ldg(reinterpret_cast<const uint4*>(y_sh + (size_t)t * d) + v), acc);
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        if (k >= K) break;
+        float r[8];
+        to_f32x8(raw[k], r);
+        const float g = sg[k];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, r[i], acc[i]);
+      }
+    } else {
+      to_f32x8(__ldg(reinterpret_cast<const uint4*>(y_sh + (size_t)t * d) + v), acc);
+      for (int k = 0; k < K; ++k) {
+        float r[8];
+        to_f32x8(__ldg(reinterpret_cast<const uint4*>(y_perm + (size_t)ss[k] * d) + v), r);
+        const float g = sg[k];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, r[i], acc[i]);
+      }
     }
     uint4 out;
     __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&out);
@@ -131,10 +152,16 @@ cudaError_t launch_combine(const moe_shape& s, const void* y_perm, const void* y
     combine_f32_kernel<<<s.T, 128, 0, st>>>(static_cast<const float*>(y_perm),
                                             static_cast<const float*>(y_shared), slot, gate,
                                             s.T, s.d, s.K, static_cast<float*>(y));
+  else if (s.K <= 8)
+    combine_bf16_kernel<8><<<s.T, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm),
+                                                static_cast<const __nv_bfloat16*>(y_shared), slot,
+                                                gate, s.T, s.d, s.K,
+                                                static_cast<__nv_bfloat16*>(y));
   else
-    combine_bf16_kernel<<<s.T, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm),
-                                             static_cast<const __nv_bfloat16*>(y_shared), slot,
-                                             gate, s.T, s.d, s.K, static_cast<__nv_bfloat16*>(y));
+    combine_bf16_kernel<0><<<s.T, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm),
+                                                static_cast<const __nv_bfloat16*>(y_shared), slot,
+                                                gate, s.T, s.d, s.K,
+                                                static_cast<__nv_bfloat16*>(y));
   return cudaGetLastError();
 }
 
