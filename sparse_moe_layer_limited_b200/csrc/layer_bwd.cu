@@ -26,6 +26,19 @@ struct Act;
 template <>
 struct Act<__nv_bfloat16> {
   static constexpr int V = 8;
+  // one 16-byte vector as loaded, and its V values as fp32
+  __device__ static uint4 raw(const __nv_bfloat16* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  __device__ static void cvt(const uint4& w, float* o) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      o[2 * i] = f.x;
+      o[2 * i + 1] = f.y;
+    }
+  }
   __device__ static void load(const __nv_bfloat16* p, float* o) {
     const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
@@ -57,6 +70,13 @@ struct Act<__nv_bfloat16> {
 template <>
 struct Act<float> {
   static constexpr int V = 4;
+  __device__ static uint4 raw(const float* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ static void cvt(const uint4& w, float* o) {
+    o[0] = __uint_as_float(w.x);
+    o[1] = __uint_as_float(w.y);
+    o[2] = __uint_as_float(w.z);
+    o[3] = __uint_as_float(w.w);
+  }
   __device__ static void load(const float* p, float* o) {
     const float4 w = __ldg(reinterpret_cast<const float4*>(p));
     o[0] = w.x;
@@ -77,7 +97,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ---- COMBINE backward: one CTA of 128 threads per token -----------------------------
-template <typename T>
+// KM > 0 (K <= KM): one pass over d; each thread loads its piece of dy_t once
+// and of all K rows of y_perm before the multiply-adds (K loads in flight),
+// and keeps the K partial dots.  KM = 0: one pass per k.  Each dgate_k is the
+// same fixed reduction either way: this thread's multiply-adds in v order,
+// then the warp's shuffle tree, then the four warps' sums in a fixed pairing.
+template <typename T, int KM>
 __global__ void __launch_bounds__(128) combine_bwd_kernel(
     const T* __restrict__ dy, const T* __restrict__ y_perm, const int32_t* __restrict__ slot,
     const float* __restrict__ gate, int ntok, int d, int K, T* __restrict__ dy_perm,
@@ -85,7 +110,7 @@ __global__ void __launch_bounds__(128) combine_bwd_kernel(
   constexpr int V = Act<T>::V;
   __shared__ int ss[kMaxK];
   __shared__ float sg[kMaxK];
-  __shared__ float red[4];
+  __shared__ float red[4][KM > 0 ? KM : 1];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < K) {
@@ -97,31 +122,74 @@ __global__ void __launch_bounds__(128) combine_bwd_kernel(
   __syncthreads();
   const int nvec = d / V;
   const T* dyt = dy + (size_t)t * d;
-  for (int k = 0; k < K; ++k) {
-    const int r = ss[k];
-    const float g = sg[k];
-    float part = 0.f;
-    if (r >= 0) {
-      const T* yr = y_perm + (size_t)r * d;
-      T* out = dy_perm + (size_t)r * d;
-      for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-        float a[V], b[V], o[V];
-        Act<T>::load(dyt + v * V, a);
-        Act<T>::load(yr + v * V, b);
+  if constexpr (KM > 0) {
+    int rk[KM];
+    float part[KM];
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      rk[k] = k < K ? ss[k] : -1;
+      part[k] = 0.f;
+    }
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      float a[V];
+      uint4 braw[KM];
+      Act<T>::load(dyt + v * V, a);
+#pragma unroll
+      for (int k = 0; k < KM; ++k)
+        if (rk[k] >= 0) braw[k] = Act<T>::raw(y_perm + (size_t)rk[k] * d + v * V);
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        if (rk[k] < 0) continue;
+        const float g = sg[k];
+        float b[V], o[V];
+        Act<T>::cvt(braw[k], b);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-          part = fmaf(a[i], b[i], part);
+          part[k] = fmaf(a[i], b[i], part[k]);
           o[i] = g * a[i];
         }
-        Act<T>::store(out + v * V, o);
+        Act<T>::store(dy_perm + (size_t)rk[k] * d + v * V, o);
       }
     }
-    part = warp_sum(part);
-    if (lane == 0) red[warp] = part;
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      const float w = warp_sum(part[k]);
+      if (lane == 0) red[warp][k] = w;
+    }
     __syncthreads();
-    if (threadIdx.x == 0)
-      dgate[(size_t)t * K + k] = r >= 0 ? (red[0] + red[1]) + (red[2] + red[3]) : 0.f;
-    __syncthreads();
+    if (threadIdx.x < K) {
+      const int k = threadIdx.x;
+      dgate[(size_t)t * K + k] =
+          ss[k] >= 0 ? (red[0][k] + red[1][k]) + (red[2][k] + red[3][k]) : 0.f;
+    }
+  } else {
+    for (int k = 0; k < K; ++k) {
+      const int r = ss[k];
+      const float g = sg[k];
+      float part = 0.f;
+      if (r >= 0) {
+        const T* yr = y_perm + (size_t)r * d;
+        T* out = dy_perm + (size_t)r * d;
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+          float a[V], b[V], o[V];
+          Act<T>::load(dyt + v * V, a);
+          Act<T>::load(yr + v * V, b);
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            part = fmaf(a[i], b[i], part);
+            o[i] = g * a[i];
+          }
+          Act<T>::store(out + v * V, o);
+        }
+      }
+      part = warp_sum(part);
+      if (lane == 0) red[warp][0] = part;
+      __syncthreads();
+      if (threadIdx.x == 0)
+        dgate[(size_t)t * K + k] =
+            r >= 0 ? (red[0][0] + red[1][0]) + (red[2][0] + red[3][0]) : 0.f;
+      __syncthreads();
+    }
   }
 }
 
@@ -291,9 +359,14 @@ template <typename T>
 cudaError_t combine_bwd(const moe_shape& s, const void* dy, const void* y_perm,
                         const int32_t* slot, const float* gate, void* dy_perm, float* dgate,
                         cudaStream_t st) {
-  combine_bwd_kernel<T><<<s.T, 128, 0, st>>>(static_cast<const T*>(dy),
-                                             static_cast<const T*>(y_perm), slot, gate, s.T, s.d,
-                                             s.K, static_cast<T*>(dy_perm), dgate);
+  if (s.K <= 8)
+    combine_bwd_kernel<T, 8><<<s.T, 128, 0, st>>>(static_cast<const T*>(dy),
+                                                  static_cast<const T*>(y_perm), slot, gate, s.T,
+                                                  s.d, s.K, static_cast<T*>(dy_perm), dgate);
+  else
+    combine_bwd_kernel<T, 0><<<s.T, 128, 0, st>>>(static_cast<const T*>(dy),
+                                                  static_cast<const T*>(y_perm), slot, gate, s.T,
+                                                  s.d, s.K, static_cast<T*>(dy_perm), dgate);
   return cudaGetLastError();
 }
 
