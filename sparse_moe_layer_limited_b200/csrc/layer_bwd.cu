@@ -196,7 +196,10 @@ __global__ void __launch_bounds__(128) combine_bwd_kernel(
 // ---- gate backward per token: one warp per token ------------------------------------
 // Lane k (k < K) holds the selected expert idx[t,k], its recomputed logit and
 // affinity; the K dot products x_t . e_i and the output row run over d in
-// 4-wide pieces, lanes interleaved (coalesced).
+// 4-wide pieces, lanes interleaved (coalesced).  For K <= 8 the output row
+// takes the K experts and their dz from lists built once, and each lane loads
+// its pieces of all K router rows before the first multiply-add (the same
+// k-order sums).
 template <typename T>
 __global__ void __launch_bounds__(256) route_bwd_token_kernel(
     const T* __restrict__ x, const float* __restrict__ R, const int32_t* __restrict__ idx,
@@ -239,6 +242,33 @@ __global__ void __launch_bounds__(256) route_bwd_token_kernel(
   const float dz = mine ? s * (1.f - s) * (dg - m) / S : 0.f;
   if (lane < K) dz_out[(size_t)t * K + lane] = dz;
   float* out = dx_route + (size_t)t * d;
+  if (K <= 8) {
+    int ek[8];
+    float wk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      ek[k] = __shfl_sync(0xffffffffu, my_e, k);
+      wk[k] = __shfl_sync(0xffffffffu, dz, k);
+      if (k >= K) ek[k] = -1;
+    }
+    for (int j = lane * 4; j < d; j += 128) {
+      float4 rv[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (ek[k] >= 0) rv[k] = __ldg(reinterpret_cast<const float4*>(R + (size_t)ek[k] * d + j));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (ek[k] < 0) continue;
+        acc.x = fmaf(wk[k], rv[k].x, acc.x);
+        acc.y = fmaf(wk[k], rv[k].y, acc.y);
+        acc.z = fmaf(wk[k], rv[k].z, acc.z);
+        acc.w = fmaf(wk[k], rv[k].w, acc.w);
+      }
+      *reinterpret_cast<float4*>(out + j) = acc;
+    }
+    return;
+  }
   for (int j0 = 0; j0 < d; j0 += 128) {  // the same trip count in every lane (shuffles)
     const int j = j0 + lane * 4;
     const bool in = j < d;
